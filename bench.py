@@ -1,0 +1,410 @@
+"""Benchmark of the B200 routed-expert FFN layer (DeepSeek-V4.1-Flash shape).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+One step = one whole layer invocation (router, top-k, permutation, gate/up and
+down grouped GEMMs, combine) on one batch of T synthetic tokens with the
+weights resident in HBM. Prints one JSON line on rank 0.
+
+  value      tokens/s over all ranks, timed with CUDA events around K steps
+             (barrier + synchronize on both sides, max over ranks)
+  e2e        the same metric through moe_forward_host: the step's x copied
+             host->device and y copied back inside the timed region
+  roofline   the dominant kernel's algorithmic bytes per launch / its mean
+             launch time (CUDA events recorded by the library on the launch
+             stream during the timed steps) against the measured HBM peak
+  cpu_baseline  the float64 CPU oracle on a bounded sample of the same
+             workload on this host's cores
+
+Multi-GPU: the layer does not shard across GPUs in this build ("replicas
+only"): every rank runs its own replica on its own tokens; no collective is on
+the data path (one all-reduce of the elapsed time, for the max over ranks).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from routed_expert_ffn_sqrtsoftplus_b200 import synth  # noqa: E402
+
+L2_BYTES = 126 * 1024 * 1024
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=200)
+    p.add_argument("--warmup", type=int, default=10)
+    p.add_argument("--workload", default="flash_decode", choices=sorted(synth.WORKLOADS))
+    p.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    p.add_argument("--tokens", type=int, default=None, help="override T of the workload")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--cpu-seconds", type=float, default=15.0, help="budget of the CPU baseline sample")
+    return p.parse_args()
+
+
+# ----------------------------------------------------------------------------- distributed
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(v: float, world: int) -> float:
+    if world == 1:
+        return v
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ----------------------------------------------------------------------------- clocks
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML while the timed region runs."""
+
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+               0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
+
+    def __init__(self, index: int, period_s: float = 0.02):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self.period, self.index = period_s, index
+        self._stop = threading.Event()
+        self._t = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self.nv = None
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                r = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for bit, name in self.REASONS.items():
+                    if r & bit and name != "gpu_idle":
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.nv is not None:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self._t is not None:
+            self._t.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# ----------------------------------------------------------------------------- workload
+def build_layer(wl, device):
+    d = synth.make_layer(wl, device=device)
+    mxq = None
+    if wl.expert_dtype == "mxfp4":
+        from routed_expert_ffn_sqrtsoftplus_b200 import quantize_mxfp4
+        mxq = {}
+        for n, s in (("w1", "s1"), ("w3", "s3"), ("w2", "s2")):
+            mxq[n], mxq[s] = quantize_mxfp4(d[n])
+    return d, mxq
+
+
+def algorithmic(wl, idx: np.ndarray, T: int):
+    """Bytes and FLOPs one step must move / do (weights read once, x in, y out)."""
+    H, I, E, S, k = wl.H, wl.I, wl.E, wl.n_shared, wl.k
+    U = len(np.unique(idx))
+    if wl.expert_dtype == "mxfp4":
+        routed = (3 * H * I) // 2 + (3 * H * I) // 32
+        routed13 = (2 * I * H) // 2 + (2 * I * H) // 32
+    else:
+        routed = 3 * H * I * 2
+        routed13 = 2 * I * H * 2
+    shared = 3 * H * I * 2
+    shared13 = 2 * I * H * 2
+    step_bytes = U * routed + S * shared + E * H * 2 + 2 * T * H * 2
+    rows = T * k + S * T
+    step_flops = 2 * T * E * H + rows * 3 * 2 * H * I
+    gateup_bytes = U * routed13 + S * shared13 + rows * H * 2 + rows * I * 2
+    gateup_flops = rows * 2 * 2 * H * I
+    return dict(U=U, step_bytes=step_bytes, step_flops=step_flops, gateup_bytes=gateup_bytes,
+                gateup_flops=gateup_flops, rows=rows)
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), float(p["bf16_tflops"]), float(p.get("bf16_tflops_sustained", p["bf16_tflops"])), "measured"
+    except Exception:
+        return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+def recorded_traffic(workload: str, kernel: str):
+    """DRAM bytes per launch from a committed ncu summary, if the kernel source is unchanged since."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)
+        ent = rec[workload][kernel]
+        src = os.path.join(ROOT, "routed_expert_ffn_sqrtsoftplus_b200", "csrc", ent["source"])
+        with open(src, "rb") as f:
+            h = hashlib.sha256(f.read()).hexdigest()[:16]
+        return ent["bytes_per_launch"] if h == ent["source_sha256_16"] else None
+    except Exception:
+        return None
+
+
+# ----------------------------------------------------------------------------- CPU oracle baseline
+def cpu_oracle_sample(wl, d, mxq, tokens, budget_s):
+    """Time the float64 oracle on `tokens` (one token at a time, streaming each
+    expert's weights from the device and upcasting them, until budget_s)."""
+    from oracle import moe as om
+    from oracle import mx as omx
+
+    def f64(t):
+        return t.detach().cpu().to(torch.float64).numpy()
+
+    wg = f64(d["wg"])
+    bias = None if d.get("bias") is None else f64(d["bias"])
+    if mxq is None:
+        routed = lambda e: (f64(d["w1"][e]), f64(d["w3"][e]), f64(d["w2"][e]))
+    else:
+        dq = lambda n, s, e: omx.dequantize_mxfp4_packed(mxq[n][e].cpu().numpy(), mxq[s][e].cpu().numpy())
+        routed = lambda e: (dq("w1", "s1", e), dq("w3", "s3", e), dq("w2", "s2", e))
+    shared = lambda j: (f64(d["sh_w1"][j]), f64(d["sh_w3"][j]), f64(d["sh_w2"][j]))
+    ex = om.ExpertSource(routed, shared, wl.E, wl.n_shared, routed_is_mx=mxq is not None)
+    done = 0
+    t0 = time.perf_counter()
+    for t in tokens:
+        x = f64(d["x"][t:t + 1])
+        om.moe_forward(x, wg, ex, wl.k, wl.route_scale, wl.swiglu_limit, bias=bias)
+        done += 1
+        if time.perf_counter() - t0 > budget_s:
+            break
+    dt = time.perf_counter() - t0
+    return done, dt
+
+
+def cpu_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count()
+
+
+# ----------------------------------------------------------------------------- main arms
+def run_ours(args, world, rank, local):
+    import routed_expert_ffn_sqrtsoftplus_b200 as moe
+    from routed_expert_ffn_sqrtsoftplus_b200 import build
+    if rank == 0:
+        build.build()
+    barrier(world)
+    wl = synth.WORKLOADS[args.workload]
+    if args.tokens:
+        wl = wl.with_tokens(args.tokens)
+    T = wl.T
+    dev = torch.device("cuda", local)
+    d, mxq = build_layer(wl, dev)
+    layer = moe.MoELayer.from_layer(d, top_k=wl.k, max_tokens=T, route_scale=wl.route_scale,
+                                    swiglu_limit=wl.swiglu_limit, mx=mxq)
+    x = d["x"]
+    y = torch.empty_like(x)
+    stream = torch.cuda.current_stream()
+    # routing of this batch, for the algorithmic byte count
+    _, idx, _ = layer.forward_with_routing(x)
+    torch.cuda.synchronize()
+    alg = algorithmic(wl, idx.cpu().numpy(), T)
+
+    for _ in range(args.warmup):
+        layer.forward(x, out=y)
+    torch.cuda.synchronize()
+    assert layer.status() == moe.MOE_OK
+
+    # ---- device-timed region
+    layer.profile_begin(args.steps)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        ev0.record(stream)
+        for _ in range(args.steps):
+            layer.forward(x, out=y)
+        ev1.record(stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    prof = layer.profile_end()
+    st = layer.status()
+    if st != moe.MOE_OK:
+        raise RuntimeError(f"device status {st} after the timed steps")
+    ms = ev0.elapsed_time(ev1)
+    ms = max_over_ranks(ms, world)
+    ms_per_step = ms / args.steps
+    value = world * T * args.steps / (ms / 1e3)
+
+    # ---- end-to-end through host buffers
+    xh = x.cpu().pin_memory()
+    yh = torch.empty_like(xh).pin_memory()
+    e2e_steps = max(3, min(args.steps, 50))
+    for _ in range(2):
+        layer.forward_host(xh, yh)
+    torch.cuda.synchronize()
+    barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        layer.forward_host(xh, yh)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
+    e2e_value = world * T * e2e_steps / (e2e_ms / 1e3)
+
+    hbm, tc, tc_sus, src = peaks()
+    # dominant kernel = the one with the largest share of device time
+    kern = max(prof, key=lambda n: prof[n][0])
+    k_ms, k_launch = prof[kern]
+    k_avg_s = k_ms / k_launch / 1e3
+    launches = sum(c for _, c in prof.values())
+    if kern == "gemm_gateup":
+        a_bytes, a_flops = alg["gateup_bytes"], alg["gateup_flops"]
+    else:
+        a_bytes, a_flops = alg["step_bytes"], alg["step_flops"]
+    t_hbm = a_bytes / (hbm * 1e9)
+    t_tc = a_flops / (tc * 1e12)
+    if t_hbm >= t_tc:
+        roof = {"bound": "hbm", "achieved": a_bytes / k_avg_s / 1e9, "peak": hbm, "unit": "GB/s"}
+    else:
+        roof = {"bound": "tensor", "achieved": a_flops / k_avg_s / 1e12, "peak": tc, "unit": "TFLOP/s"}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["traffic"] = recorded_traffic(wl.name, kern)
+    roof["kernel"] = kern
+    roof["peak_source"] = f"{src} (MEASURED_PEAKS.json)" if src == "measured" else "fallback"
+    step_s = ms_per_step / 1e3
+    layer_roof = {"bytes": alg["step_bytes"], "flops": alg["step_flops"],
+                  "hbm_frac": alg["step_bytes"] / step_s / (hbm * 1e9),
+                  "tensor_frac": alg["step_flops"] / step_s / (tc * 1e12),
+                  "distinct_experts": alg["U"]}
+
+    out = {
+        "metric": "MoE layer tokens/s (Flash shape, BF16 & MXFP4) + % of HBM/tensor roofline",
+        "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16" if wl.expert_dtype == "bf16" else "mxfp4xmxfp8",
+        "data": "synthetic (seeded N(0,1/fan_in) BF16 weights, N(0,1) tokens)",
+        "config": {"workload": wl.name, "T": T, "hidden": wl.H, "inter": wl.I, "n_routed": wl.E,
+                   "n_shared": wl.n_shared, "top_k": wl.k, "route_scale": wl.route_scale,
+                   "swiglu_limit": wl.swiglu_limit, "expert_dtype": wl.expert_dtype,
+                   "parallelism": f"replicas x{world}",
+                   "l2": f"no flush: each step streams {alg['step_bytes'] / 1e9:.2f} GB of weights > 126 MB L2"},
+        "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": T * wl.H * 2,
+                "d2h_bytes_per_step": T * wl.H * 2},
+        "roofline": roof,
+        "layer_roofline": layer_roof,
+        "kernels_ms_per_step": {n: v[0] / args.steps for n, v in sorted(prof.items())},
+        "gpu_launches": launches,
+        "clocks": clk.summary(),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rng = np.random.default_rng(0)
+        toks = rng.permutation(T)
+        n, dt = cpu_oracle_sample(wl, d, mxq, toks, args.cpu_seconds)
+        out["cpu_baseline"] = {"value": n / dt, "unit": "tokens/s", "cores": cpu_cores(), "kind": "oracle",
+                               "sample": f"{n} of {T} tokens, one at a time; each hit expert's weights copied "
+                                         f"from the device and upcast to float64 inside the timing"}
+    layer.close()
+    return out
+
+
+def run_reference(args, world, rank, local):
+    """The float64 CPU oracle as the reference arm, on rank 0 only."""
+    wl = synth.WORKLOADS[args.workload]
+    if args.tokens:
+        wl = wl.with_tokens(args.tokens)
+    if rank != 0:
+        return None
+    dev = torch.device("cuda", local)
+    d, mxq = build_layer(wl, dev)
+    total_budget = 150.0
+    per_step = max(0.2, total_budget / max(1, args.steps + args.warmup))
+    rng = np.random.default_rng(1)
+    done_t, dt_t = 0, 0.0
+    for i in range(args.warmup + args.steps):
+        toks = rng.integers(0, wl.T, size=1)
+        n, dt = cpu_oracle_sample(wl, d, mxq, toks, per_step)
+        if i >= args.warmup:
+            done_t += n
+            dt_t += dt
+    value = done_t / dt_t
+    return {
+        "impl": "reference",
+        "metric": "MoE layer tokens/s (Flash shape, BF16 & MXFP4) + % of HBM/tensor roofline",
+        "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * dt_t / max(1, args.steps), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": wl.name, "T": wl.T, "hidden": wl.H, "inter": wl.I, "n_routed": wl.E,
+                   "top_k": wl.k, "expert_dtype": wl.expert_dtype},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cpu_cores(), "kind": "oracle",
+                         "sample": "one token per step, its routed experts and the shared expert streamed "
+                                   "from the device and upcast to float64"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    args = parse()
+    world, rank, local = dist_setup(args)
+    try:
+        out = run_reference(args, world, rank, local) if args.impl == "reference" else run_ours(args, world, rank, local)
+        if rank == 0 and out is not None:
+            print(json.dumps(out), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,239 @@
+/*
+ * moe.h - C ABI of the B200 (sm_100a) DeepSeek-V4.1-Flash routed-expert FFN layer.
+ *
+ * The layer (DeepSeek V4.1 inference/config.json: "n_routed_experts" 384,
+ * "n_shared_experts" 1, "n_activated_experts" 6, "dim" 5120, "moe_inter_dim"
+ * 2304, "score_func" "sqrtsoftplus", "route_scale" 1.5, "swiglu_limit" 10.0,
+ * "expert_dtype" "fp4"; MAX DeepseekV41Config fields of the same meaning):
+ *
+ *   z_e  = x . Wg_e (+ b_e)                     router logits, e < E
+ *   s_e  = sqrt(softplus(z_e))                  "sqrtsoftplus" score
+ *   sel  = the top_k experts by s_e (ties: lower index first), descending
+ *   w_j  = route_scale * s_sel(j) / sum_j s_sel(j)
+ *   f(x) = W2 (silu(min(W1 x, L)) * clamp(W3 x, -L, L)),   L = swiglu_limit
+ *   y    = sum_{shared} f_sh(x) + sum_j w_j f_sel(j)(x)
+ *
+ * The pages name the score function and the clamp but print no formula; the
+ * lines above are the plainest reading and the one the library computes.
+ *
+ * Conventions for every entry point
+ *   - Device pointers are CUDA device (or managed) addresses on the device that
+ *     was current when the handle was created; host pointers are noted as such.
+ *   - Every matrix is row-major [out, in]: the input (reduction) dimension is
+ *     contiguous. BF16 is IEEE bfloat16 bit patterns in uint16 storage.
+ *   - A stream argument is a cudaStream_t (NULL = legacy default stream). Work is
+ *     enqueued on it and the call returns without synchronising unless the entry
+ *     point says otherwise.
+ *   - Argument errors are detected before anything is enqueued and returned as a
+ *     status; no entry point aborts the process or prints.
+ *   - Device-side bounded waits that run out record MOE_ERR_TIMEOUT in the
+ *     handle's status word, read by moe_get_status().
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define MOE_ABI_VERSION 1
+
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+struct CUstream_st;
+typedef struct CUstream_st* moe_stream_t; /* == cudaStream_t */
+
+typedef struct moe_handle moe_handle;
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1, /* null pointer, bad size, T > max_tokens, misaligned pointer */
+  MOE_ERR_UNSUPPORTED = 2, /* valid but outside what the kernels implement (see moe_config) */
+  MOE_ERR_OOM = 3,         /* device allocation failed inside moe_create */
+  MOE_ERR_CUDA = 4,        /* a CUDA runtime call or kernel launch failed */
+  MOE_ERR_TIMEOUT = 5,     /* a device-side bounded wait ran out (reported by moe_get_status) */
+  MOE_ERR_DEVICE = 6       /* a device-side consistency check failed (reported by moe_get_status) */
+} moe_status;
+
+typedef enum {
+  MOE_DT_BF16 = 0, /* routed experts in BF16 */
+  MOE_DT_MXFP4 = 1 /* routed experts in MXFP4: E2M1 values + one E8M0 scale per 32 along K */
+} moe_expert_dtype;
+
+/*
+ * Layer shape and constants (MAX DeepseekV41Config: hidden_size,
+ * moe_intermediate_size, n_routed_experts, n_shared_experts,
+ * num_experts_per_tok, routed_scaling_factor, swiglu_limit).
+ *
+ * Supported: hidden % 128 == 0, inter % 128 == 0, 1 <= top_k <= n_routed <= 512,
+ * 0 <= n_shared <= 4, 1 <= max_tokens <= 65536, route_scale > 0 and finite,
+ * swiglu_limit >= 0 (INFINITY disables both clamps). Anything else returns
+ * MOE_ERR_UNSUPPORTED (shape) or MOE_ERR_INVALID_ARG (NaN, negative, zero).
+ */
+typedef struct {
+  int32_t hidden;       /* H */
+  int32_t inter;        /* I, expert width (routed and shared) */
+  int32_t n_routed;     /* E */
+  int32_t n_shared;     /* shared experts, weight 1 each */
+  int32_t top_k;        /* k */
+  int32_t max_tokens;   /* largest T a forward may pass; sizes the workspace */
+  float route_scale;    /* rho */
+  float swiglu_limit;   /* L */
+  int32_t expert_dtype; /* moe_expert_dtype of the routed experts */
+} moe_config;
+
+/*
+ * Weights, all device pointers, read during moe_create only (the library keeps
+ * its own repacked copy; the caller may free its buffers once the create
+ * stream has completed).
+ *   router_w     BF16 [E, H]
+ *   router_bias  fp32 [E] added to the logits (selection and weights), or NULL
+ *   BF16 experts:  w1, w3 BF16 [E, I, H]; w2 BF16 [E, H, I]; s1 = s3 = s2 = NULL
+ *   MXFP4 experts: w1, w3 uint8 [E, I, H/2]; w2 uint8 [E, H, I/2]: E2M1 pairs,
+ *                  element 2j in the low nibble of byte j (float4_e2m1fnx2);
+ *                  s1, s3 uint8 [E, I, H/32]; s2 uint8 [E, H, I/32]: E8M0
+ *                  scales (2^(code-127)), code 0xFF (NaN) is rejected.
+ *   sh_w1, sh_w3 BF16 [n_shared, I, H]; sh_w2 BF16 [n_shared, H, I] (always BF16)
+ * Every pointer must be 16-byte aligned.
+ */
+typedef struct {
+  const void* router_w;
+  const float* router_bias;
+  const void* w1;
+  const void* w3;
+  const void* w2;
+  const uint8_t* s1;
+  const uint8_t* s3;
+  const uint8_t* s2;
+  const void* sh_w1;
+  const void* sh_w3;
+  const void* sh_w2;
+} moe_weights;
+
+/*
+ * Create a layer on the current device: validate, allocate the repacked
+ * weights and the workspace for cfg->max_tokens tokens, and enqueue the weight
+ * repack on `stream` (the analogue of the MAX pipeline's one-time routed-expert
+ * upload, DeepseekV41Model.load_model). On success *out owns all device memory
+ * it allocated. On failure *out is NULL and nothing is leaked.
+ */
+MOE_API moe_status moe_create(const moe_config* cfg, const moe_weights* w, moe_stream_t stream,
+                      moe_handle** out);
+
+/*
+ * One layer invocation on T token rows.
+ *   x        BF16 [T, H] device, 16-byte aligned
+ *   y        BF16 [T, H] device, 16-byte aligned (may not alias x)
+ *   topk_idx int32 [T, k] device or NULL: selected experts, descending score
+ *   topk_w   fp32  [T, k] device or NULL: their weights (sum = route_scale)
+ * 0 <= T <= max_tokens; T == 0 enqueues nothing. Allocates nothing and does not
+ * synchronise. Calls on one handle must be ordered (one stream at a time): the
+ * workspace is shared between calls.
+ */
+MOE_API moe_status moe_forward(moe_handle* h, const void* x, int32_t T, void* y, int32_t* topk_idx,
+                       float* topk_w, moe_stream_t stream);
+
+/*
+ * moe_forward on HOST buffers: copies x (BF16 [T, H], host, ideally pinned)
+ * into a handle-owned device staging buffer, runs the layer, and copies y
+ * (and topk_idx / topk_w when not NULL, host [T, k]) back, all enqueued on
+ * `stream`. The host buffers must stay valid until the stream reaches the end
+ * of the copies; synchronise the stream before reading them.
+ */
+MOE_API moe_status moe_forward_host(moe_handle* h, const void* x_host, int32_t T, void* y_host,
+                            int32_t* topk_idx_host, float* topk_w_host, moe_stream_t stream);
+
+/* Synchronise the device, then report and clear the device-side status word
+ * (MOE_OK, MOE_ERR_TIMEOUT or MOE_ERR_DEVICE); MOE_ERR_CUDA if the sync failed. */
+MOE_API moe_status moe_get_status(moe_handle* h);
+
+/* Static string for a status code. */
+MOE_API const char* moe_status_string(moe_status s);
+
+/* Free everything the handle owns (synchronises the device first). NULL is a no-op. */
+MOE_API void moe_destroy(moe_handle* h);
+
+/* MOE_ABI_VERSION of the loaded library. */
+MOE_API int32_t moe_abi_version(void);
+
+/* ------------------------------------------------------------------------
+ * Utilities (not part of the layer's arithmetic path)
+ * ---------------------------------------------------------------------- */
+
+/*
+ * Quantise BF16 [rows, cols] (device) to MXFP4 with the OCP MX v1.0 rule: per
+ * block of 32 along cols, scale = 2^(floor(log2(amax)) - 2) clamped to the E8M0
+ * range (all-zero block: code 0), elements rounded to nearest-even E2M1 and
+ * saturated at +-6. Writes packed [rows, cols/2] (low nibble = even element)
+ * and scales [rows, cols/32]. cols % 32 == 0. Enqueued on `stream`.
+ */
+MOE_API moe_status moe_quantize_mxfp4(const void* src_bf16, int64_t rows, int32_t cols, uint8_t* dst_packed,
+                              uint8_t* dst_scales, moe_stream_t stream);
+
+/* Internal buffers of the LAST forward that moe_inspect can copy out. */
+typedef enum {
+  MOE_BUF_LOGITS = 0,   /* fp32 [T, E] router logits before refinement (approximate) */
+  MOE_BUF_TOPK_IDX = 1, /* int32 [T, k] */
+  MOE_BUF_TOPK_W = 2,   /* fp32 [T, k] */
+  MOE_BUF_COUNTS = 3,   /* int32 [E + n_shared] rows per group (routed experts, then shared) */
+  MOE_BUF_OFFSETS = 4,  /* int32 [E + n_shared + 1] first row of each group */
+  MOE_BUF_PERM = 5,     /* int32 [T*k] flat slot t*k+j of each routed row (expert-major) */
+  MOE_BUF_INV = 6,      /* int32 [T*k] row of each flat slot */
+  MOE_BUF_H = 7,        /* BF16 [T*k + n_shared*T, I] SwiGLU output rows (group order) */
+  MOE_BUF_XQ = 8,       /* MXFP4 layers: uint8 E4M3 [T, H] MXFP8 codes of x */
+  MOE_BUF_XQ_SCALES = 9 /* MXFP4 layers: uint8 E8M0 [T, H/32] */
+} moe_buffer;
+
+/*
+ * Copy `bytes` from the start of internal buffer `what` to dst (host or device;
+ * cudaMemcpyAsync with cudaMemcpyDefault on `stream`). bytes must not exceed the
+ * buffer's size for max_tokens. For tests and debugging.
+ */
+MOE_API moe_status moe_inspect(moe_handle* h, int32_t what, void* dst, size_t bytes, moe_stream_t stream);
+
+/* Limit, in nanoseconds, of every device-side wait of this handle's kernels
+ * (default 2e9). A smaller value makes a stuck wait return sooner. */
+MOE_API moe_status moe_set_wait_timeout(moe_handle* h, uint64_t timeout_ns);
+
+/*
+ * Launch one kernel whose only job is an mbarrier wait that nothing completes,
+ * bounded by timeout_ns; it records MOE_ERR_TIMEOUT in the handle's status word
+ * and returns. Proves the bounded-wait path without hanging the device.
+ */
+MOE_API moe_status moe_selftest_wait_timeout(moe_handle* h, uint64_t timeout_ns, moe_stream_t stream);
+
+/* Sizes of what the handle owns. */
+typedef struct {
+  uint64_t weight_bytes;     /* repacked router + expert weights */
+  uint64_t workspace_bytes;  /* per-forward scratch for max_tokens */
+  int32_t num_sms;           /* SMs the persistent kernels are sized for */
+  int32_t last_tokens;       /* T of the last forward */
+} moe_info;
+
+MOE_API moe_status moe_get_info(moe_handle* h, moe_info* out);
+
+/*
+ * Per-kernel device timing. moe_profile_begin(h, max_calls) makes the next
+ * max_calls forwards record a CUDA event pair around every kernel they launch
+ * (on the forward's stream). moe_profile_end(h, ms, launches, n) synchronises,
+ * adds up the elapsed time per kernel kind over the recorded forwards into
+ * ms[0..n) and the launch counts into launches[0..n), and stops recording.
+ * Kinds are indexed as moe_kernel_name() names them.
+ */
+MOE_API moe_status moe_profile_begin(moe_handle* h, int32_t max_calls);
+MOE_API moe_status moe_profile_end(moe_handle* h, double* ms, int64_t* launches, int32_t n);
+MOE_API int32_t moe_num_kernel_kinds(void);
+MOE_API const char* moe_kernel_name(int32_t kind);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_B200_H */

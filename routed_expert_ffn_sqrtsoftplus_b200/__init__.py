@@ -1,0 +1,290 @@
+"""B200 (sm_100a) DeepSeek-V4.1-Flash routed-expert FFN layer with sqrtsoftplus routing.
+
+A thin ctypes binding of the C ABI in include/moe.h. It only marshals torch
+tensors into pointers and streams: every step of the layer runs in the CUDA
+kernels of libmoe_b200.so. There is no CPU fallback; if the library is missing
+or no CUDA device is present the calls raise.
+
+    from routed_expert_ffn_sqrtsoftplus_b200 import MoELayer
+    layer = MoELayer(hidden=5120, inter=2304, n_routed=384, n_shared=1, top_k=6,
+                     max_tokens=32, router_w=wg, w1=w1, w3=w3, w2=w2,
+                     sh_w1=s1, sh_w3=s3, sh_w2=s2)
+    y = layer(x)                       # x, y: BF16 [T, 5120] on the GPU
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "_lib", "libmoe_b200.so")
+
+MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_OOM, MOE_ERR_CUDA, MOE_ERR_TIMEOUT, MOE_ERR_DEVICE = range(7)
+MOE_DT_BF16, MOE_DT_MXFP4 = 0, 1
+
+# moe_buffer ids
+BUF_LOGITS, BUF_TOPK_IDX, BUF_TOPK_W, BUF_COUNTS, BUF_OFFSETS, BUF_PERM, BUF_INV, BUF_H, BUF_XQ, BUF_XQ_SCALES = range(10)
+
+EXPORTED = ("moe_create", "moe_forward", "moe_forward_host", "moe_get_status", "moe_status_string",
+            "moe_destroy", "moe_abi_version", "moe_quantize_mxfp4", "moe_inspect", "moe_set_wait_timeout",
+            "moe_selftest_wait_timeout", "moe_get_info", "moe_profile_begin", "moe_profile_end",
+            "moe_num_kernel_kinds", "moe_kernel_name")
+
+
+class MoEError(RuntimeError):
+    def __init__(self, status: int, what: str = ""):
+        self.status = status
+        name = _status_name(status)
+        super().__init__(f"{what}: {name}" if what else name)
+
+
+class _Config(ctypes.Structure):
+    _fields_ = [("hidden", ctypes.c_int32), ("inter", ctypes.c_int32), ("n_routed", ctypes.c_int32),
+                ("n_shared", ctypes.c_int32), ("top_k", ctypes.c_int32), ("max_tokens", ctypes.c_int32),
+                ("route_scale", ctypes.c_float), ("swiglu_limit", ctypes.c_float),
+                ("expert_dtype", ctypes.c_int32)]
+
+
+class _Weights(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in ("router_w", "router_bias", "w1", "w3", "w2", "s1", "s3", "s2",
+                                              "sh_w1", "sh_w3", "sh_w2")]
+
+
+class _Info(ctypes.Structure):
+    _fields_ = [("weight_bytes", ctypes.c_uint64), ("workspace_bytes", ctypes.c_uint64),
+                ("num_sms", ctypes.c_int32), ("last_tokens", ctypes.c_int32)]
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded libmoe_b200.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                               "`python -m routed_expert_ffn_sqrtsoftplus_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        P, I32, U64, I64 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_uint64, ctypes.c_int64
+        sig = {
+            "moe_create": (I32, [ctypes.POINTER(_Config), ctypes.POINTER(_Weights), P, ctypes.POINTER(P)]),
+            "moe_forward": (I32, [P, P, I32, P, P, P, P]),
+            "moe_forward_host": (I32, [P, P, I32, P, P, P, P]),
+            "moe_get_status": (I32, [P]),
+            "moe_status_string": (ctypes.c_char_p, [I32]),
+            "moe_destroy": (None, [P]),
+            "moe_abi_version": (I32, []),
+            "moe_quantize_mxfp4": (I32, [P, I64, I32, P, P, P]),
+            "moe_inspect": (I32, [P, I32, P, ctypes.c_size_t, P]),
+            "moe_set_wait_timeout": (I32, [P, U64]),
+            "moe_selftest_wait_timeout": (I32, [P, U64, P]),
+            "moe_get_info": (I32, [P, ctypes.POINTER(_Info)]),
+            "moe_profile_begin": (I32, [P, I32]),
+            "moe_profile_end": (I32, [P, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(I64), I32]),
+            "moe_num_kernel_kinds": (I32, []),
+            "moe_kernel_name": (ctypes.c_char_p, [I32]),
+        }
+        for name, (res, args) in sig.items():
+            f = getattr(L, name)
+            f.restype = res
+            f.argtypes = args
+        _lib = L
+    return _lib
+
+
+def _status_name(s: int) -> str:
+    try:
+        return lib().moe_status_string(s).decode()
+    except Exception:
+        return f"status {s}"
+
+
+def _check(status: int, what: str):
+    if status != MOE_OK:
+        raise MoEError(status, what)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _need(t: torch.Tensor, name: str, dtype, shape=None, device_type="cuda"):
+    if t.device.type != device_type:
+        raise ValueError(f"{name} must be on {device_type}")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+
+
+def kernel_names():
+    L = lib()
+    return [L.moe_kernel_name(i).decode() for i in range(L.moe_num_kernel_kinds())]
+
+
+def quantize_mxfp4(w: torch.Tensor, stream=None):
+    """BF16 [..., K] (CUDA) -> (packed E2M1 uint8 [..., K/2], E8M0 uint8 [..., K/32]) on the device."""
+    _need(w, "w", torch.bfloat16)
+    K = w.shape[-1]
+    rows = w.numel() // K
+    packed = torch.empty(w.shape[:-1] + (K // 2,), dtype=torch.uint8, device=w.device)
+    scales = torch.empty(w.shape[:-1] + (K // 32,), dtype=torch.uint8, device=w.device)
+    _check(lib().moe_quantize_mxfp4(_ptr(w), rows, K, _ptr(packed), _ptr(scales), _stream(stream)),
+           "moe_quantize_mxfp4")
+    return packed, scales
+
+
+class MoELayer:
+    """One routed-expert FFN layer resident on the current CUDA device."""
+
+    def __init__(self, *, hidden: int, inter: int, n_routed: int, n_shared: int, top_k: int, max_tokens: int,
+                 router_w: torch.Tensor, w1: torch.Tensor, w3: torch.Tensor, w2: torch.Tensor,
+                 sh_w1: Optional[torch.Tensor] = None, sh_w3: Optional[torch.Tensor] = None,
+                 sh_w2: Optional[torch.Tensor] = None, router_bias: Optional[torch.Tensor] = None,
+                 s1: Optional[torch.Tensor] = None, s3: Optional[torch.Tensor] = None,
+                 s2: Optional[torch.Tensor] = None, route_scale: float = 1.5, swiglu_limit: float = 10.0,
+                 expert_dtype: str = "bf16", stream=None):
+        self._h = ctypes.c_void_p(None)
+        L = lib()
+        H, I, E, S = hidden, inter, n_routed, n_shared
+        _need(router_w, "router_w", torch.bfloat16, (E, H))
+        if router_bias is not None:
+            _need(router_bias, "router_bias", torch.float32, (E,))
+        if expert_dtype == "bf16":
+            _need(w1, "w1", torch.bfloat16, (E, I, H)); _need(w3, "w3", torch.bfloat16, (E, I, H))
+            _need(w2, "w2", torch.bfloat16, (E, H, I))
+            dt = MOE_DT_BF16
+        elif expert_dtype == "mxfp4":
+            _need(w1, "w1", torch.uint8, (E, I, H // 2)); _need(w3, "w3", torch.uint8, (E, I, H // 2))
+            _need(w2, "w2", torch.uint8, (E, H, I // 2))
+            for n, t, shp in (("s1", s1, (E, I, H // 32)), ("s3", s3, (E, I, H // 32)), ("s2", s2, (E, H, I // 32))):
+                if t is None:
+                    raise ValueError(f"{n} is required for MXFP4 experts")
+                _need(t, n, torch.uint8, shp)
+            dt = MOE_DT_MXFP4
+        else:
+            raise ValueError("expert_dtype must be 'bf16' or 'mxfp4'")
+        if S > 0:
+            _need(sh_w1, "sh_w1", torch.bfloat16, (S, I, H)); _need(sh_w3, "sh_w3", torch.bfloat16, (S, I, H))
+            _need(sh_w2, "sh_w2", torch.bfloat16, (S, H, I))
+        self.cfg = _Config(H, I, E, S, top_k, max_tokens, float(route_scale), float(swiglu_limit), dt)
+        wts = _Weights(_ptr(router_w), _ptr(router_bias), _ptr(w1), _ptr(w3), _ptr(w2), _ptr(s1), _ptr(s3),
+                       _ptr(s2), _ptr(sh_w1), _ptr(sh_w3), _ptr(sh_w2))
+        st = _stream(stream)
+        _check(L.moe_create(ctypes.byref(self.cfg), ctypes.byref(wts), st, ctypes.byref(self._h)), "moe_create")
+        # The library copied the weights on `st`; wait so the caller may free its tensors.
+        torch.cuda.synchronize()
+        self.hidden, self.inter, self.n_routed, self.n_shared, self.top_k = H, I, E, S, top_k
+        self.max_tokens = max_tokens
+
+    # ------------------------------------------------------------------ forward
+    def forward(self, x: torch.Tensor, out: Optional[torch.Tensor] = None, topk_idx: Optional[torch.Tensor] = None,
+                topk_w: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+        T = x.shape[0]
+        _need(x, "x", torch.bfloat16, (T, self.hidden))
+        if out is None:
+            out = torch.empty_like(x)
+        _need(out, "out", torch.bfloat16, (T, self.hidden))
+        if topk_idx is not None:
+            _need(topk_idx, "topk_idx", torch.int32, (T, self.top_k))
+        if topk_w is not None:
+            _need(topk_w, "topk_w", torch.float32, (T, self.top_k))
+        _check(lib().moe_forward(self._h, _ptr(x), T, _ptr(out), _ptr(topk_idx), _ptr(topk_w), _stream(stream)),
+               "moe_forward")
+        return out
+
+    __call__ = forward
+
+    def forward_with_routing(self, x: torch.Tensor, stream=None):
+        T = x.shape[0]
+        idx = torch.empty((T, self.top_k), dtype=torch.int32, device=x.device)
+        w = torch.empty((T, self.top_k), dtype=torch.float32, device=x.device)
+        y = self.forward(x, topk_idx=idx, topk_w=w, stream=stream)
+        return y, idx, w
+
+    def forward_host(self, x_host: torch.Tensor, y_host: torch.Tensor, topk_idx_host: Optional[torch.Tensor] = None,
+                     topk_w_host: Optional[torch.Tensor] = None, stream=None):
+        """Host buffers in, host buffers out (copies enqueued on the stream; sync before reading)."""
+        T = x_host.shape[0]
+        _need(x_host, "x_host", torch.bfloat16, (T, self.hidden), "cpu")
+        _need(y_host, "y_host", torch.bfloat16, (T, self.hidden), "cpu")
+        if topk_idx_host is not None:
+            _need(topk_idx_host, "topk_idx_host", torch.int32, (T, self.top_k), "cpu")
+        if topk_w_host is not None:
+            _need(topk_w_host, "topk_w_host", torch.float32, (T, self.top_k), "cpu")
+        _check(lib().moe_forward_host(self._h, _ptr(x_host), T, _ptr(y_host), _ptr(topk_idx_host),
+                                      _ptr(topk_w_host), _stream(stream)), "moe_forward_host")
+
+    # ------------------------------------------------------------------ inspection
+    def inspect(self, what: int, out: torch.Tensor, stream=None) -> torch.Tensor:
+        nbytes = out.numel() * out.element_size()
+        _check(lib().moe_inspect(self._h, what, _ptr(out), nbytes, _stream(stream)), "moe_inspect")
+        return out
+
+    def status(self) -> int:
+        return lib().moe_get_status(self._h)
+
+    def info(self) -> dict:
+        i = _Info()
+        _check(lib().moe_get_info(self._h, ctypes.byref(i)), "moe_get_info")
+        return dict(weight_bytes=i.weight_bytes, workspace_bytes=i.workspace_bytes, num_sms=i.num_sms,
+                    last_tokens=i.last_tokens)
+
+    def set_wait_timeout(self, ns: int):
+        _check(lib().moe_set_wait_timeout(self._h, int(ns)), "moe_set_wait_timeout")
+
+    def selftest_wait_timeout(self, ns: int, stream=None):
+        _check(lib().moe_selftest_wait_timeout(self._h, int(ns), _stream(stream)), "moe_selftest_wait_timeout")
+
+    def profile_begin(self, max_calls: int):
+        _check(lib().moe_profile_begin(self._h, max_calls), "moe_profile_begin")
+
+    def profile_end(self) -> dict:
+        L = lib()
+        n = L.moe_num_kernel_kinds()
+        ms = (ctypes.c_double * n)()
+        cnt = (ctypes.c_int64 * n)()
+        _check(L.moe_profile_end(self._h, ms, cnt, n), "moe_profile_end")
+        return {kernel_names()[i]: (ms[i], cnt[i]) for i in range(n) if cnt[i] > 0}
+
+    def close(self):
+        if self._h:
+            lib().moe_destroy(self._h)
+            self._h = ctypes.c_void_p(None)
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    @classmethod
+    def from_layer(cls, layer: dict, *, top_k: int, max_tokens: int, route_scale: float = 1.5,
+                   swiglu_limit: float = 10.0, mx: Optional[dict] = None, stream=None) -> "MoELayer":
+        """Build from a dict of tensors (x ignored): wg, bias, w1, w3, w2, sh_w1, sh_w3, sh_w2.
+
+        With ``mx`` = dict(w1, s1, w3, s3, w2, s2) of MXFP4 tensors the routed experts are MXFP4.
+        """
+        E, I, H = layer["w1"].shape
+        S = layer["sh_w1"].shape[0] if layer.get("sh_w1") is not None else 0
+        kw = dict(hidden=H, inter=I, n_routed=E, n_shared=S, top_k=top_k, max_tokens=max_tokens,
+                  router_w=layer["wg"], router_bias=layer.get("bias"), sh_w1=layer.get("sh_w1"),
+                  sh_w3=layer.get("sh_w3"), sh_w2=layer.get("sh_w2"), route_scale=route_scale,
+                  swiglu_limit=swiglu_limit, stream=stream)
+        if mx is None:
+            return cls(w1=layer["w1"], w3=layer["w3"], w2=layer["w2"], expert_dtype="bf16", **kw)
+        return cls(w1=mx["w1"], w3=mx["w3"], w2=mx["w2"], s1=mx["s1"], s3=mx["s3"], s2=mx["s2"],
+                   expert_dtype="mxfp4", **kw)

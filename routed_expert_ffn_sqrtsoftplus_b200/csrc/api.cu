@@ -1,0 +1,562 @@
+// Host runtime behind include/moe.h: argument validation, the handle (repacked
+// weights + workspace), TMA descriptors, and the launch sequence of one layer
+// invocation. Every step of the layer runs in this library's kernels.
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <new>
+#include <vector>
+
+#include "../../include/moe.h"
+#include "common.cuh"
+#include "kernels.h"
+
+using namespace moe;
+
+namespace {
+
+// Logit error of the approximate router is far below this (fp32 sums of exact
+// BF16 products, or tensor-core fp32 accumulation); every expert whose
+// approximate score lies within kRefineDelta of the k-th is re-scored exactly.
+constexpr float kRefineDelta = 2e-3f;
+// Token counts above this use the tensor-core router GEMM for the logits.
+constexpr int kTcRouterMinTokens = 256;
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (fn == nullptr) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// BF16 [rows, cols] row-major, 128-byte swizzled boxes of 64 columns x box_rows.
+bool make_tmap_bf16(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+  EncodeTiledFn enc = get_encode_fn();
+  if (enc == nullptr) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * 2};
+  cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+const char* kKernelNames[kKNumKinds] = {"router_logits", "router_gemm",  "topk_refine", "perm_count",
+                                        "perm_scan",     "perm_scatter", "gather_rows", "gemm_gateup",
+                                        "gemm_down",     "combine",      "quant_x"};
+
+}  // namespace
+
+struct moe_handle {
+  moe_config cfg{};
+  int device = 0;
+  int num_sms = 148;
+  int G = 0;       // routed + shared groups
+  int64_t R = 0;   // max rows of h / O
+  int nchunks_max = 0;
+  int m_tiles_gu = 0, m_tiles_dn = 0;
+  int64_t max_tiles_gu = 0, max_tiles_dn = 0;
+
+  void* wg = nullptr;
+  float* bias = nullptr;
+  void* w13 = nullptr;
+  void* w2 = nullptr;
+
+  float* z = nullptr;
+  int32_t* idx = nullptr;
+  float* wts = nullptr;
+  int32_t* chunk_cnt = nullptr;
+  int32_t* cnt = nullptr;
+  int32_t* off = nullptr;
+  int32_t* perm = nullptr;
+  int32_t* inv = nullptr;
+  int4* tiles_gu = nullptr;
+  int4* tiles_dn = nullptr;
+  int* ntiles = nullptr;
+  void* xp = nullptr;
+  void* h = nullptr;
+  float* o = nullptr;
+  int* status = nullptr;
+  void* x_stage = nullptr;
+  void* y_stage = nullptr;
+
+  CUtensorMap tm_w13, tm_w2, tm_xp, tm_h, tm_wg;
+  uint64_t timeout_ns = 2000000000ull;
+  std::vector<void*> allocs;
+  uint64_t weight_bytes = 0, workspace_bytes = 0;
+  int last_T = 0;
+
+  // profiling
+  bool prof_on = false;
+  std::vector<cudaEvent_t> ev;  // pairs
+  std::vector<int> ev_kind;
+  size_t ev_used = 0;
+
+  template <class T>
+  bool alloc(T** p, size_t bytes, uint64_t* counter) {
+    void* q = nullptr;
+    if (bytes == 0) bytes = 16;
+    if (cudaMalloc(&q, bytes) != cudaSuccess) {
+      cudaGetLastError();
+      return false;
+    }
+    allocs.push_back(q);
+    *p = static_cast<T*>(q);
+    *counter += bytes;
+    return true;
+  }
+
+  void release() {
+    for (void* p : allocs) cudaFree(p);
+    allocs.clear();
+    for (cudaEvent_t e : ev) cudaEventDestroy(e);
+    ev.clear();
+  }
+
+  void prof_mark(int kind, cudaStream_t s) {
+    if (!prof_on || ev_used + 2 > ev.size()) return;
+    cudaEventRecord(ev[ev_used], s);
+    ev_kind[ev_used / 2] = kind;
+  }
+  void prof_done(cudaStream_t s) {
+    if (!prof_on || ev_used + 2 > ev.size()) return;
+    cudaEventRecord(ev[ev_used + 1], s);
+    ev_used += 2;
+  }
+};
+
+namespace {
+
+moe_status validate_config(const moe_config* c) {
+  if (!(c->route_scale > 0.f) || !std::isfinite(c->route_scale)) return MOE_ERR_INVALID_ARG;
+  if (std::isnan(c->swiglu_limit) || c->swiglu_limit < 0.f) return MOE_ERR_INVALID_ARG;
+  if (c->hidden <= 0 || c->inter <= 0 || c->n_routed <= 0 || c->top_k <= 0 || c->max_tokens <= 0 ||
+      c->n_shared < 0)
+    return MOE_ERR_INVALID_ARG;
+  if (c->top_k > c->n_routed) return MOE_ERR_INVALID_ARG;
+  if (c->hidden % 128 != 0 || c->inter % 128 != 0) return MOE_ERR_UNSUPPORTED;
+  if (c->n_routed > 512 || c->top_k > 32 || c->n_shared > 4 || c->max_tokens > 65536) return MOE_ERR_UNSUPPORTED;
+  if (c->hidden > 16384 || c->inter > 16384) return MOE_ERR_UNSUPPORTED;
+  if (c->expert_dtype != MOE_DT_BF16 && c->expert_dtype != MOE_DT_MXFP4) return MOE_ERR_INVALID_ARG;
+  if (c->expert_dtype == MOE_DT_MXFP4) return MOE_ERR_UNSUPPORTED;
+  return MOE_OK;
+}
+
+#define MOE_TRY_CUDA(expr)                 \
+  do {                                     \
+    if ((expr) != cudaSuccess) {           \
+      cudaGetLastError();                  \
+      return MOE_ERR_CUDA;                 \
+    }                                      \
+  } while (0)
+
+}  // namespace
+
+extern "C" {
+
+int32_t moe_abi_version(void) { return MOE_ABI_VERSION; }
+
+const char* moe_status_string(moe_status s) {
+  switch (s) {
+    case MOE_OK: return "MOE_OK";
+    case MOE_ERR_INVALID_ARG: return "MOE_ERR_INVALID_ARG";
+    case MOE_ERR_UNSUPPORTED: return "MOE_ERR_UNSUPPORTED";
+    case MOE_ERR_OOM: return "MOE_ERR_OOM";
+    case MOE_ERR_CUDA: return "MOE_ERR_CUDA";
+    case MOE_ERR_TIMEOUT: return "MOE_ERR_TIMEOUT";
+    case MOE_ERR_DEVICE: return "MOE_ERR_DEVICE";
+  }
+  return "MOE_ERR_UNKNOWN";
+}
+
+int32_t moe_num_kernel_kinds(void) { return kKNumKinds; }
+
+const char* moe_kernel_name(int32_t kind) {
+  if (kind < 0 || kind >= kKNumKinds) return nullptr;
+  return kKernelNames[kind];
+}
+
+moe_status moe_create(const moe_config* cfg, const moe_weights* w, moe_stream_t stream, moe_handle** out) {
+  if (out == nullptr) return MOE_ERR_INVALID_ARG;
+  *out = nullptr;
+  if (cfg == nullptr || w == nullptr) return MOE_ERR_INVALID_ARG;
+  moe_status st = validate_config(cfg);
+  if (st != MOE_OK) return st;
+  const void* req[] = {w->router_w, w->w1, w->w3, w->w2};
+  for (const void* p : req)
+    if (p == nullptr || !aligned16(p)) return MOE_ERR_INVALID_ARG;
+  if (cfg->n_shared > 0) {
+    const void* sh[] = {w->sh_w1, w->sh_w3, w->sh_w2};
+    for (const void* p : sh)
+      if (p == nullptr || !aligned16(p)) return MOE_ERR_INVALID_ARG;
+  }
+  if (w->router_bias != nullptr && !aligned16(w->router_bias)) return MOE_ERR_INVALID_ARG;
+  if (get_encode_fn() == nullptr) return MOE_ERR_CUDA;
+
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  moe_handle* h = new (std::nothrow) moe_handle();
+  if (h == nullptr) return MOE_ERR_OOM;
+  h->cfg = *cfg;
+  if (cudaGetDevice(&h->device) != cudaSuccess ||
+      cudaDeviceGetAttribute(&h->num_sms, cudaDevAttrMultiProcessorCount, h->device) != cudaSuccess) {
+    cudaGetLastError();
+    delete h;
+    return MOE_ERR_CUDA;
+  }
+  if (gemm_set_attributes() != cudaSuccess) {
+    cudaGetLastError();
+    delete h;
+    return MOE_ERR_CUDA;
+  }
+  const int64_t H = cfg->hidden, I = cfg->inter, E = cfg->n_routed, S = cfg->n_shared, k = cfg->top_k,
+                Tm = cfg->max_tokens;
+  h->G = static_cast<int>(E + S);
+  h->R = Tm * k + S * Tm;
+  h->nchunks_max = static_cast<int>((Tm * k + kPermChunk - 1) / kPermChunk);
+  h->m_tiles_gu = static_cast<int>(I / 128);
+  h->m_tiles_dn = static_cast<int>(H / 128);
+  h->max_tiles_gu = h->m_tiles_gu * (h->G + (h->R + 31) / 32);
+  h->max_tiles_dn = h->m_tiles_dn * (h->G + (h->R + 31) / 32);
+
+  bool ok = true;
+  uint64_t* wb = &h->weight_bytes;
+  uint64_t* ws = &h->workspace_bytes;
+  ok = ok && h->alloc(&h->wg, E * H * 2, wb);
+  if (w->router_bias) ok = ok && h->alloc(&h->bias, E * 4, wb);
+  ok = ok && h->alloc(&h->w13, (E + S) * 2 * I * H * 2, wb);
+  ok = ok && h->alloc(&h->w2, (E + S) * H * I * 2, wb);
+  ok = ok && h->alloc(&h->z, Tm * E * 4, ws);
+  ok = ok && h->alloc(&h->idx, Tm * k * 4, ws);
+  ok = ok && h->alloc(&h->wts, Tm * k * 4, ws);
+  ok = ok && h->alloc(&h->chunk_cnt, static_cast<size_t>(h->nchunks_max) * E * 4, ws);
+  ok = ok && h->alloc(&h->cnt, (E + S) * 4, ws);
+  ok = ok && h->alloc(&h->off, (E + S + 1) * 4, ws);
+  ok = ok && h->alloc(&h->perm, Tm * k * 4, ws);
+  ok = ok && h->alloc(&h->inv, Tm * k * 4, ws);
+  ok = ok && h->alloc(&h->tiles_gu, h->max_tiles_gu * 16, ws);
+  ok = ok && h->alloc(&h->tiles_dn, h->max_tiles_dn * 16, ws);
+  ok = ok && h->alloc(&h->ntiles, 16, ws);
+  ok = ok && h->alloc(&h->xp, Tm * k * H * 2, ws);
+  ok = ok && h->alloc(&h->h, h->R * I * 2, ws);
+  ok = ok && h->alloc(&h->o, h->R * H * 4, ws);
+  ok = ok && h->alloc(&h->status, 16, ws);
+  ok = ok && h->alloc(&h->x_stage, Tm * H * 2, ws);
+  ok = ok && h->alloc(&h->y_stage, Tm * H * 2, ws);
+  if (!ok) {
+    h->release();
+    delete h;
+    return MOE_ERR_OOM;
+  }
+
+  bool err = false;
+  err |= cudaMemsetAsync(h->status, 0, 16, s) != cudaSuccess;
+  err |= cudaMemcpyAsync(h->wg, w->router_w, E * H * 2, cudaMemcpyDeviceToDevice, s) != cudaSuccess;
+  if (w->router_bias) err |= cudaMemcpyAsync(h->bias, w->router_bias, E * 4, cudaMemcpyDeviceToDevice, s) != cudaSuccess;
+  err |= launch_repack_w13(w->w1, w->w3, w->sh_w1, w->sh_w3, static_cast<int>(E), static_cast<int>(S),
+                           static_cast<int>(I), static_cast<int>(H), h->w13, s) != cudaSuccess;
+  err |= cudaMemcpyAsync(h->w2, w->w2, E * H * I * 2, cudaMemcpyDeviceToDevice, s) != cudaSuccess;
+  if (S > 0)
+    err |= cudaMemcpyAsync(static_cast<uint8_t*>(h->w2) + E * H * I * 2, w->sh_w2, S * H * I * 2,
+                           cudaMemcpyDeviceToDevice, s) != cudaSuccess;
+  // The tile lists are rewritten by every forward; zero them once so a stale
+  // read can never see uninitialised memory.
+  err |= cudaMemsetAsync(h->ntiles, 0, 16, s) != cudaSuccess;
+  err |= !make_tmap_bf16(&h->tm_w13, h->w13, (E + S) * 2 * I, H, 256);
+  err |= !make_tmap_bf16(&h->tm_w2, h->w2, (E + S) * H, I, 128);
+  err |= !make_tmap_bf16(&h->tm_xp, h->xp, Tm * k, H, 32);
+  err |= !make_tmap_bf16(&h->tm_h, h->h, h->R, I, 32);
+  err |= !make_tmap_bf16(&h->tm_wg, h->wg, E, H, 128);
+  if (err) {
+    cudaGetLastError();
+    cudaStreamSynchronize(s);
+    h->release();
+    delete h;
+    return MOE_ERR_CUDA;
+  }
+  *out = h;
+  return MOE_OK;
+}
+
+moe_status moe_forward(moe_handle* h, const void* x, int32_t T, void* y, int32_t* topk_idx, float* topk_w,
+                       moe_stream_t stream) {
+  if (h == nullptr) return MOE_ERR_INVALID_ARG;
+  if (T < 0 || T > h->cfg.max_tokens) return MOE_ERR_INVALID_ARG;
+  if (T == 0) {
+    h->last_T = 0;
+    return MOE_OK;
+  }
+  if (x == nullptr || y == nullptr || !aligned16(x) || !aligned16(y) || x == y) return MOE_ERR_INVALID_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const moe_config& c = h->cfg;
+  const int H = c.hidden, I = c.inter, E = c.n_routed, S = c.n_shared, k = c.top_k;
+  const int nslots = T * k;
+  const int nchunks = (nslots + kPermChunk - 1) / kPermChunk;
+  const bool small = T <= 32;
+  const int bn_gu = small ? 32 : 128;
+  const int bn_dn = small ? 32 : 256;
+
+  CUtensorMap tm_x;
+  if (!make_tmap_bf16(&tm_x, x, static_cast<uint64_t>(T), static_cast<uint64_t>(H), 32)) return MOE_ERR_CUDA;
+
+  // 1. router logits (+ bias)
+  if (T < kTcRouterMinTokens) {
+    h->prof_mark(kKRouterLogits, s);
+    MOE_TRY_CUDA(launch_router_logits(x, h->wg, h->bias, h->z, T, H, E, s));
+    h->prof_done(s);
+  } else {
+    GemmArgs a{};
+    a.tiles = nullptr;
+    a.ntiles = nullptr;
+    a.dense_m_tiles = (E + 127) / 128;
+    a.dense_rows = T;
+    a.num_kb = H / 64;
+    a.a_rows_per_group = 0;
+    a.n_routed = 0;
+    a.out = h->z;
+    a.out_ld = E;
+    a.out_rows = T;
+    a.m_limit = E;
+    a.limit = 0.f;
+    a.col_bias = h->bias;
+    a.status = h->status;
+    a.timeout_ns = h->timeout_ns;
+    const int nt = a.dense_m_tiles * ((T + 255) / 256);
+    h->prof_mark(kKRouterGemm, s);
+    MOE_TRY_CUDA(launch_gemm_down(h->tm_wg, tm_x, a, 256, nt < h->num_sms ? nt : h->num_sms, s));
+    h->prof_done(s);
+  }
+  // 2. scores, top-k with exact refinement, weights
+  h->prof_mark(kKTopk, s);
+  MOE_TRY_CUDA(launch_topk_refine(h->z, x, h->wg, h->bias, T, H, E, k, c.route_scale, kRefineDelta, h->idx, h->wts,
+                                  h->status, s));
+  h->prof_done(s);
+  // 3. permutation and tile lists
+  h->prof_mark(kKPermCount, s);
+  MOE_TRY_CUDA(launch_perm_count(h->idx, nslots, E, h->chunk_cnt, h->status, s));
+  h->prof_done(s);
+  ScanArgs sa;
+  sa.chunk_cnt = h->chunk_cnt;
+  sa.nchunks = nchunks;
+  sa.E = E;
+  sa.S = S;
+  sa.T = T;
+  sa.k = k;
+  sa.cnt = h->cnt;
+  sa.off = h->off;
+  sa.tiles_gu = h->tiles_gu;
+  sa.tiles_dn = h->tiles_dn;
+  sa.ntiles = h->ntiles;
+  sa.m_tiles_gu = h->m_tiles_gu;
+  sa.bn_gu = bn_gu;
+  sa.m_tiles_dn = h->m_tiles_dn;
+  sa.bn_dn = bn_dn;
+  h->prof_mark(kKPermScan, s);
+  MOE_TRY_CUDA(launch_perm_scan(sa, s));
+  h->prof_done(s);
+  h->prof_mark(kKPermScatter, s);
+  MOE_TRY_CUDA(launch_perm_scatter(h->idx, nslots, E, h->chunk_cnt, h->perm, h->inv, s));
+  h->prof_done(s);
+  h->prof_mark(kKGather, s);
+  MOE_TRY_CUDA(launch_gather_rows(x, h->perm, nslots, k, H, h->xp, s));
+  h->prof_done(s);
+  // 4. gate/up grouped GEMM with the clamped SwiGLU epilogue
+  {
+    GemmArgs a{};
+    a.tiles = h->tiles_gu;
+    a.ntiles = h->ntiles;
+    a.num_kb = H / 64;
+    a.a_rows_per_group = 2 * I;
+    a.n_routed = E;
+    a.out = h->h;
+    a.out_ld = I;
+    a.out_rows = static_cast<int>(h->R);
+    a.m_limit = I;
+    a.limit = c.swiglu_limit;
+    a.status = h->status;
+    a.timeout_ns = h->timeout_ns;
+    h->prof_mark(kKGateUp, s);
+    MOE_TRY_CUDA(launch_gemm_gateup(h->tm_w13, h->tm_xp, tm_x, a, bn_gu, h->num_sms, s));
+    h->prof_done(s);
+  }
+  // 5. down grouped GEMM
+  {
+    GemmArgs a{};
+    a.tiles = h->tiles_dn;
+    a.ntiles = h->ntiles + 1;
+    a.num_kb = I / 64;
+    a.a_rows_per_group = H;
+    a.n_routed = E;
+    a.out = h->o;
+    a.out_ld = H;
+    a.out_rows = static_cast<int>(h->R);
+    a.m_limit = H;
+    a.limit = 0.f;
+    a.status = h->status;
+    a.timeout_ns = h->timeout_ns;
+    h->prof_mark(kKDown, s);
+    MOE_TRY_CUDA(launch_gemm_down(h->tm_w2, h->tm_h, a, bn_dn, h->num_sms, s));
+    h->prof_done(s);
+  }
+  // 6. weighted combine with the shared experts
+  h->prof_mark(kKCombine, s);
+  MOE_TRY_CUDA(launch_combine(h->o, h->inv, h->wts, T, H, k, S, y, s));
+  h->prof_done(s);
+  if (topk_idx) MOE_TRY_CUDA(cudaMemcpyAsync(topk_idx, h->idx, static_cast<size_t>(nslots) * 4, cudaMemcpyDefault, s));
+  if (topk_w) MOE_TRY_CUDA(cudaMemcpyAsync(topk_w, h->wts, static_cast<size_t>(nslots) * 4, cudaMemcpyDefault, s));
+  h->last_T = T;
+  return MOE_OK;
+}
+
+moe_status moe_forward_host(moe_handle* h, const void* x_host, int32_t T, void* y_host, int32_t* topk_idx_host,
+                            float* topk_w_host, moe_stream_t stream) {
+  if (h == nullptr) return MOE_ERR_INVALID_ARG;
+  if (T < 0 || T > h->cfg.max_tokens) return MOE_ERR_INVALID_ARG;
+  if (T == 0) return MOE_OK;
+  if (x_host == nullptr || y_host == nullptr) return MOE_ERR_INVALID_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const size_t bytes = static_cast<size_t>(T) * h->cfg.hidden * 2;
+  MOE_TRY_CUDA(cudaMemcpyAsync(h->x_stage, x_host, bytes, cudaMemcpyHostToDevice, s));
+  moe_status st = moe_forward(h, h->x_stage, T, h->y_stage, nullptr, nullptr, stream);
+  if (st != MOE_OK) return st;
+  MOE_TRY_CUDA(cudaMemcpyAsync(y_host, h->y_stage, bytes, cudaMemcpyDeviceToHost, s));
+  const size_t kb = static_cast<size_t>(T) * h->cfg.top_k * 4;
+  if (topk_idx_host) MOE_TRY_CUDA(cudaMemcpyAsync(topk_idx_host, h->idx, kb, cudaMemcpyDeviceToHost, s));
+  if (topk_w_host) MOE_TRY_CUDA(cudaMemcpyAsync(topk_w_host, h->wts, kb, cudaMemcpyDeviceToHost, s));
+  return MOE_OK;
+}
+
+moe_status moe_get_status(moe_handle* h) {
+  if (h == nullptr) return MOE_ERR_INVALID_ARG;
+  if (cudaDeviceSynchronize() != cudaSuccess) {
+    cudaGetLastError();
+    return MOE_ERR_CUDA;
+  }
+  int v = 0;
+  if (cudaMemcpy(&v, h->status, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess ||
+      cudaMemset(h->status, 0, sizeof(int)) != cudaSuccess) {
+    cudaGetLastError();
+    return MOE_ERR_CUDA;
+  }
+  if (v & kStatusTimeout) return MOE_ERR_TIMEOUT;
+  if (v & kStatusDevice) return MOE_ERR_DEVICE;
+  return MOE_OK;
+}
+
+void moe_destroy(moe_handle* h) {
+  if (h == nullptr) return;
+  cudaDeviceSynchronize();
+  cudaGetLastError();
+  h->release();
+  delete h;
+}
+
+moe_status moe_quantize_mxfp4(const void* src_bf16, int64_t rows, int32_t cols, uint8_t* dst_packed,
+                              uint8_t* dst_scales, moe_stream_t stream) {
+  if (rows < 0 || cols <= 0 || cols % 32 != 0) return MOE_ERR_INVALID_ARG;
+  if (rows == 0) return MOE_OK;
+  if (src_bf16 == nullptr || dst_packed == nullptr || dst_scales == nullptr) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(src_bf16) || !aligned16(dst_packed)) return MOE_ERR_INVALID_ARG;
+  MOE_TRY_CUDA(launch_quantize_mxfp4(src_bf16, rows, cols, dst_packed, dst_scales,
+                                     reinterpret_cast<cudaStream_t>(stream)));
+  return MOE_OK;
+}
+
+moe_status moe_inspect(moe_handle* h, int32_t what, void* dst, size_t bytes, moe_stream_t stream) {
+  if (h == nullptr || dst == nullptr) return MOE_ERR_INVALID_ARG;
+  const int64_t Tm = h->cfg.max_tokens, k = h->cfg.top_k, E = h->cfg.n_routed, I = h->cfg.inter;
+  const void* src = nullptr;
+  size_t cap = 0;
+  switch (what) {
+    case MOE_BUF_LOGITS: src = h->z; cap = Tm * E * 4; break;
+    case MOE_BUF_TOPK_IDX: src = h->idx; cap = Tm * k * 4; break;
+    case MOE_BUF_TOPK_W: src = h->wts; cap = Tm * k * 4; break;
+    case MOE_BUF_COUNTS: src = h->cnt; cap = h->G * 4; break;
+    case MOE_BUF_OFFSETS: src = h->off; cap = (h->G + 1) * 4; break;
+    case MOE_BUF_PERM: src = h->perm; cap = Tm * k * 4; break;
+    case MOE_BUF_INV: src = h->inv; cap = Tm * k * 4; break;
+    case MOE_BUF_H: src = h->h; cap = h->R * I * 2; break;
+    default: return MOE_ERR_INVALID_ARG;
+  }
+  if (bytes > cap) return MOE_ERR_INVALID_ARG;
+  if (bytes == 0) return MOE_OK;
+  MOE_TRY_CUDA(cudaMemcpyAsync(dst, src, bytes, cudaMemcpyDefault, reinterpret_cast<cudaStream_t>(stream)));
+  return MOE_OK;
+}
+
+moe_status moe_set_wait_timeout(moe_handle* h, uint64_t timeout_ns) {
+  if (h == nullptr || timeout_ns == 0) return MOE_ERR_INVALID_ARG;
+  h->timeout_ns = timeout_ns;
+  return MOE_OK;
+}
+
+moe_status moe_selftest_wait_timeout(moe_handle* h, uint64_t timeout_ns, moe_stream_t stream) {
+  if (h == nullptr || timeout_ns == 0 || timeout_ns > 10000000000ull) return MOE_ERR_INVALID_ARG;
+  MOE_TRY_CUDA(launch_wait_timeout_probe(h->status, timeout_ns, reinterpret_cast<cudaStream_t>(stream)));
+  return MOE_OK;
+}
+
+moe_status moe_get_info(moe_handle* h, moe_info* out) {
+  if (h == nullptr || out == nullptr) return MOE_ERR_INVALID_ARG;
+  out->weight_bytes = h->weight_bytes;
+  out->workspace_bytes = h->workspace_bytes;
+  out->num_sms = h->num_sms;
+  out->last_tokens = h->last_T;
+  return MOE_OK;
+}
+
+moe_status moe_profile_begin(moe_handle* h, int32_t max_calls) {
+  if (h == nullptr || max_calls <= 0 || max_calls > 100000) return MOE_ERR_INVALID_ARG;
+  const size_t need = static_cast<size_t>(max_calls) * 2 * 12;
+  while (h->ev.size() < need) {
+    cudaEvent_t e;
+    if (cudaEventCreate(&e) != cudaSuccess) {
+      cudaGetLastError();
+      return MOE_ERR_CUDA;
+    }
+    h->ev.push_back(e);
+  }
+  h->ev_kind.assign(h->ev.size() / 2, -1);
+  h->ev_used = 0;
+  h->prof_on = true;
+  return MOE_OK;
+}
+
+moe_status moe_profile_end(moe_handle* h, double* ms, int64_t* launches, int32_t n) {
+  if (h == nullptr || ms == nullptr || launches == nullptr || n < 0) return MOE_ERR_INVALID_ARG;
+  h->prof_on = false;
+  for (int i = 0; i < n; ++i) {
+    ms[i] = 0.0;
+    launches[i] = 0;
+  }
+  if (cudaDeviceSynchronize() != cudaSuccess) {
+    cudaGetLastError();
+    return MOE_ERR_CUDA;
+  }
+  for (size_t p = 0; p + 1 < h->ev_used; p += 2) {
+    float t = 0.f;
+    const int kind = h->ev_kind[p / 2];
+    if (kind < 0 || kind >= n) continue;
+    if (cudaEventElapsedTime(&t, h->ev[p], h->ev[p + 1]) == cudaSuccess) {
+      ms[kind] += t;
+      launches[kind] += 1;
+    } else {
+      cudaGetLastError();
+    }
+  }
+  h->ev_used = 0;
+  return MOE_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,355 @@
+// Grouped expert GEMMs on the 5th-generation tensor cores (tcgen05 + TMEM + TMA).
+//
+// Swap-AB formulation: the expert weights are the M operand (128 rows of the
+// weight matrix per tile) and the tokens routed to the expert are the N
+// operand (16..BN tokens), so a decode step with 1-3 tokens per expert still
+// issues full-height MMAs while streaming every weight byte exactly once.
+//
+//   gate/up tile: D_G[128 x N] = W1[rows] . X^T,  D_U[128 x N] = W3[rows] . X^T
+//                 h[token, i] = silu(min(D_G, L)) * clamp(D_U, -L, L)   -> BF16
+//                 (the gated expert MLP with the swiglu_limit clamp of the
+//                 DeepSeek V4.1 config: "swiglu_limit": 10.0)
+//   down tile:    D[128 x N] = W2[rows] . h^T                            -> fp32 rows
+//
+// One persistent CTA per SM, warp-specialised:
+//   warp 0      TMA producer: A box (weights) + B boxes (token rows) per 64-wide K step
+//   warp 1      MMA issuer: tcgen05.mma kind::f16, accumulators in TMEM
+//   warps 2..5  epilogue: tcgen05.ld -> math -> global stores
+// A kStages-deep shared-memory ring (full/empty mbarriers) decouples TMA and
+// MMA; two TMEM accumulator buffers (tmem_full/tmem_empty) let the epilogue of
+// tile i overlap the MMAs of tile i+1. Every wait is bounded in time; a wait
+// that runs out records MOE_ERR_TIMEOUT, drains this CTA's in-flight copies and
+// MMAs, frees TMEM and returns.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace moe {
+
+namespace {
+
+constexpr int kThreads = 192;
+constexpr int kBK = 64;           // K elements per stage (128 bytes of BF16 = one swizzle row)
+constexpr int kBBoxRows = 32;     // token rows per B TMA box
+constexpr int kBBoxBytes = kBBoxRows * 128;
+
+constexpr int pow2_at_least(int v, int lo) {
+  int p = lo;
+  while (p < v) p *= 2;
+  return p;
+}
+
+template <bool kGateUp, int BN, int kStages>
+struct Cfg {
+  static constexpr int kARows = kGateUp ? 256 : 128;
+  static constexpr int kABytes = kARows * 128;
+  static constexpr int kBBytes = BN * 128;
+  static constexpr int kAccCols = kGateUp ? 2 * BN : BN;
+  static constexpr int kTmemCols = pow2_at_least(2 * kAccCols, 32);
+  static constexpr int kBarrierBytes = 256;
+  static constexpr int kSmemBytes = 1024 + kStages * (kABytes + kBBytes) + kBarrierBytes;
+  static_assert(kTmemCols <= 512, "TMEM holds 512 columns");
+  static_assert(BN % kBBoxRows == 0 && BN >= 32 && BN <= 256, "BN");
+  static_assert(kSmemBytes <= 227 * 1024, "shared memory");
+};
+
+struct Tile {
+  int group, m_tile, b_row0, out_row0, nrows;
+};
+
+template <int BN>
+__device__ __forceinline__ Tile load_tile(const GemmArgs& a, int t) {
+  Tile r;
+  if (a.tiles != nullptr) {
+    const int4 v = a.tiles[t];
+    r.group = v.x & 0xFFFF;
+    r.m_tile = v.x >> 16;
+    r.b_row0 = v.y;
+    r.out_row0 = v.z;
+    r.nrows = v.w;
+  } else {
+    r.group = 0;
+    r.m_tile = t % a.dense_m_tiles;
+    const int nt = t / a.dense_m_tiles;
+    r.b_row0 = r.out_row0 = nt * BN;
+    r.nrows = min(BN, a.dense_rows - nt * BN);
+  }
+  // A tile never holds more rows than the B ring has room for.
+  r.nrows = max(0, min(r.nrows, BN));
+  return r;
+}
+
+template <int BN>
+__device__ __forceinline__ int tile_count(const GemmArgs& a) {
+  if (a.tiles != nullptr) return *a.ntiles;
+  return a.dense_m_tiles * ((a.dense_rows + BN - 1) / BN);
+}
+
+// Wait that also gives up as soon as another role of this CTA has aborted.
+__device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, const GemmArgs& a,
+                                              volatile int* abort_flag) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
+#pragma unroll 1
+    for (int i = 0; i < 32; ++i)
+      if (mbar_try_wait(bar, parity)) return true;
+    if (*abort_flag) return false;
+    if (globaltimer_ns() - t0 > a.timeout_ns) {
+      *abort_flag = 1;
+      report_status(a.status, kStatusTimeout);
+      return false;
+    }
+  }
+}
+
+template <bool kGateUp, int BN, int kStages>
+__global__ void __launch_bounds__(kThreads, 1)
+    grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                        const __grid_constant__ CUtensorMap tmBsh, const GemmArgs args) {
+  using C = Cfg<kGateUp, BN, kStages>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + kStages * C::kABytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sB + kStages * C::kBBytes);
+  uint64_t* full = bars;
+  uint64_t* empty = bars + kStages;
+  uint64_t* tfull = bars + 2 * kStages;
+  uint64_t* tempty = bars + 2 * kStages + 2;
+  uint64_t* drain = bars + 2 * kStages + 4;
+  uint32_t* tmem_base_smem = reinterpret_cast<uint32_t*>(bars + 2 * kStages + 5);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_base_smem + 1);
+
+  const int warp = threadIdx.x / 32;
+  const int lane = threadIdx.x % 32;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kStages; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&tfull[i], 1);
+      mbar_init(&tempty[i], 4);  // one arrive per epilogue warp
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbarrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+    if (kGateUp) tma_prefetch_desc(&tmBsh);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_base_smem, C::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_base_smem;
+
+  const int ntiles = tile_count<BN>(args);
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      long issued = 0;
+      for (int t = blockIdx.x; t < ntiles && !*abort_flag; t += gridDim.x) {
+        const Tile tl = load_tile<BN>(args, t);
+        const CUtensorMap* mb = (kGateUp && tl.group >= args.n_routed) ? &tmBsh : &tmB;
+        const int a_row = tl.group * args.a_rows_per_group + tl.m_tile * C::kARows;
+        const int nb = (tl.nrows + kBBoxRows - 1) / kBBoxRows;
+        const uint32_t bytes = C::kABytes + nb * kBBoxBytes;
+        bool ok = true;
+        for (int kb = 0; kb < args.num_kb; ++kb) {
+          if (!wait_or_abort(&empty[stage], phase ^ 1, args, abort_flag)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&full[stage], bytes);
+          tma_load_2d(sA + stage * C::kABytes, &tmA, &full[stage], kb * kBK, a_row, kCacheEvictFirst);
+          for (int j = 0; j < nb; ++j)
+            tma_load_2d(sB + stage * C::kBBytes + j * kBBoxBytes, mb, &full[stage], kb * kBK,
+                        tl.b_row0 + j * kBBoxRows, kCacheEvictLast);
+          ++issued;
+          if (++stage == kStages) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+        if (!ok) break;
+      }
+      if (*abort_flag) {
+        // Let every copy this thread started land before the CTA goes away.
+        for (long i = issued - 1; i >= 0 && i >= issued - kStages; --i) {
+          const int s = static_cast<int>(i % kStages);
+          const uint32_t par = static_cast<uint32_t>((i / kStages) & 1);
+          const uint64_t t0 = globaltimer_ns();
+          while (!mbar_try_wait(&full[s], par) && globaltimer_ns() - t0 < args.timeout_ns) {
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      for (int t = blockIdx.x; t < ntiles && !*abort_flag; t += gridDim.x) {
+        const Tile tl = load_tile<BN>(args, t);
+        const uint32_t n_mma = max(16, (tl.nrows + 15) & ~15);
+        const uint32_t idesc = idesc_bf16_f32(128, n_mma);
+        if (!wait_or_abort(&tempty[acc], acc_phase ^ 1, args, abort_flag)) break;
+        tc_fence_after();
+        const uint32_t d = tmem_base + acc * C::kAccCols;
+        bool ok = true;
+        for (int kb = 0; kb < args.num_kb; ++kb) {
+          if (!wait_or_abort(&full[stage], phase, args, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_addr = smem_u32(sA + stage * C::kABytes);
+          const uint32_t b_addr = smem_u32(sB + stage * C::kBBytes);
+#pragma unroll
+          for (int k = 0; k < kBK / 16; ++k) {
+            const uint64_t bdesc = sdesc_sw128(b_addr + k * 32);
+            const uint32_t accum = (kb | k) != 0;
+            umma_f16(d, sdesc_sw128(a_addr + k * 32), bdesc, idesc, accum);
+            if (kGateUp) umma_f16(d + BN, sdesc_sw128(a_addr + 128 * 128 + k * 32), bdesc, idesc, accum);
+          }
+          umma_commit(&empty[stage]);
+          if (++stage == kStages) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+        if (!ok) break;
+        umma_commit(&tfull[acc]);
+        if (++acc == 2) {
+          acc = 0;
+          acc_phase ^= 1;
+        }
+      }
+      // Every MMA this thread issued has completed once `drain` flips.
+      umma_commit(drain);
+      const uint64_t t0 = globaltimer_ns();
+      while (!mbar_try_wait(drain, 0) && globaltimer_ns() - t0 < args.timeout_ns) {
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3;  // TMEM lane quarter this warp may access
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int t = blockIdx.x; t < ntiles; t += gridDim.x) {
+      const Tile tl = load_tile<BN>(args, t);
+      const int n_mma = max(16, (tl.nrows + 15) & ~15);
+      bool ok = true;
+      if (lane == 0) ok = wait_or_abort(&tfull[acc], acc_phase, args, abort_flag);
+      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+      if (!ok) break;
+      tc_fence_after();
+      const uint32_t tb = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * C::kAccCols;
+      const int m = tl.m_tile * 128 + q * 32 + lane;
+      const bool rows_ok = tl.out_row0 >= 0 && tl.out_row0 + tl.nrows <= args.out_rows;
+      if (!rows_ok && lane == 0 && q == 0) report_status(args.status, kStatusDevice);
+      const bool m_ok = m < args.m_limit && rows_ok;
+      for (int c0 = 0; c0 < n_mma; c0 += 16) {
+        uint32_t g[16];
+        tmem_ld16(tb + c0, g);
+        if constexpr (kGateUp) {
+          uint32_t u[16];
+          tmem_ld16(tb + BN + c0, u);
+          tmem_ld_wait();
+          __nv_bfloat16* out = static_cast<__nv_bfloat16*>(args.out);
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const int n = c0 + j;
+            if (n < tl.nrows && m_ok) {
+              const float hv = clamped_swiglu_f32(__uint_as_float(g[j]), __uint_as_float(u[j]), args.limit);
+              out[static_cast<size_t>(tl.out_row0 + n) * args.out_ld + m] = __float2bfloat16_rn(hv);
+            }
+          }
+        } else {
+          tmem_ld_wait();
+          float* out = static_cast<float*>(args.out);
+          const float cb = (args.col_bias != nullptr && m_ok) ? args.col_bias[m] : 0.0f;
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const int n = c0 + j;
+            if (n < tl.nrows && m_ok)
+              out[static_cast<size_t>(tl.out_row0 + n) * args.out_ld + m] = __uint_as_float(g[j]) + cb;
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty[acc]);
+      if (++acc == 2) {
+        acc = 0;
+        acc_phase ^= 1;
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, C::kTmemCols);
+  }
+}
+
+template <bool kGateUp, int BN, int kStages>
+cudaError_t set_attr() {
+  return cudaFuncSetAttribute(grouped_gemm_kernel<kGateUp, BN, kStages>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              Cfg<kGateUp, BN, kStages>::kSmemBytes);
+}
+
+template <bool kGateUp, int BN, int kStages>
+cudaError_t launch(const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap& tmBsh, const GemmArgs& a,
+                   int grid, cudaStream_t s) {
+  grouped_gemm_kernel<kGateUp, BN, kStages>
+      <<<grid, kThreads, Cfg<kGateUp, BN, kStages>::kSmemBytes, s>>>(tmA, tmB, tmBsh, a);
+  return cudaGetLastError();
+}
+
+// Stage counts: as many as fit in 227 KB with the barriers.
+constexpr int kGuSmallStages = 6;   // 6 * (32 KB + 4 KB)
+constexpr int kGuLargeStages = 4;   // 4 * (32 KB + 16 KB)
+constexpr int kDnSmallStages = 10;  // 10 * (16 KB + 4 KB)
+constexpr int kDnLargeStages = 4;   // 4 * (16 KB + 32 KB)
+
+}  // namespace
+
+cudaError_t gemm_set_attributes() {
+  cudaError_t e;
+  if ((e = set_attr<true, 32, kGuSmallStages>()) != cudaSuccess) return e;
+  if ((e = set_attr<true, 128, kGuLargeStages>()) != cudaSuccess) return e;
+  if ((e = set_attr<false, 32, kDnSmallStages>()) != cudaSuccess) return e;
+  if ((e = set_attr<false, 256, kDnLargeStages>()) != cudaSuccess) return e;
+  return cudaSuccess;
+}
+
+cudaError_t launch_gemm_gateup(const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap& tmBsh,
+                               const GemmArgs& a, int bn, int grid, cudaStream_t s) {
+  if (bn == 32) return launch<true, 32, kGuSmallStages>(tmA, tmB, tmBsh, a, grid, s);
+  if (bn == 128) return launch<true, 128, kGuLargeStages>(tmA, tmB, tmBsh, a, grid, s);
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_gemm_down(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmArgs& a, int bn, int grid,
+                             cudaStream_t s) {
+  if (bn == 32) return launch<false, 32, kDnSmallStages>(tmA, tmB, tmB, a, grid, s);
+  if (bn == 256) return launch<false, 256, kDnLargeStages>(tmA, tmB, tmB, a, grid, s);
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace moe

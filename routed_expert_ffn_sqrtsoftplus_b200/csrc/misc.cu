@@ -1,0 +1,160 @@
+// Weighted combine with the shared experts, weight repacking, the MXFP4 weight
+// quantiser utility, and the bounded-wait self test.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace moe {
+
+namespace {
+
+// y[t] = sum_shared O[T*k + j*T + t] + sum_j w[t, j] * O[inv[t*k + j]]
+// (shared experts have weight 1; the routed sum runs in slot order j = 0..k-1,
+// accumulated in fp32 and rounded once to BF16).
+__global__ void __launch_bounds__(128)
+    combine_kernel(const float4* __restrict__ O, const int32_t* __restrict__ inv, const float* __restrict__ w, int T,
+                   int H4, int k, int S, uint2* __restrict__ y) {
+  const int t = blockIdx.x;
+  const int c = blockIdx.y * blockDim.x + threadIdx.x;
+  if (c >= H4) return;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  const size_t routed_rows = static_cast<size_t>(T) * k;
+  for (int j = 0; j < S; ++j) {
+    const float4 v = __ldg(O + (routed_rows + static_cast<size_t>(j) * T + t) * H4 + c);
+    acc.x += v.x;
+    acc.y += v.y;
+    acc.z += v.z;
+    acc.w += v.w;
+  }
+  for (int j = 0; j < k; ++j) {
+    const int row = __ldg(inv + static_cast<size_t>(t) * k + j);
+    const float wj = __ldg(w + static_cast<size_t>(t) * k + j);
+    const float4 v = __ldg(O + static_cast<size_t>(row) * H4 + c);
+    acc.x = fmaf(wj, v.x, acc.x);
+    acc.y = fmaf(wj, v.y, acc.y);
+    acc.z = fmaf(wj, v.z, acc.z);
+    acc.w = fmaf(wj, v.w, acc.w);
+  }
+  __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y);
+  __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z, acc.w);
+  uint2 out;
+  out.x = *reinterpret_cast<uint32_t*>(&lo);
+  out.y = *reinterpret_cast<uint32_t*>(&hi);
+  y[static_cast<size_t>(t) * H4 + c] = out;
+}
+
+// W13 layout: for each group g and 128-row tile mt of the expert width, 256
+// consecutive rows = W1[g][mt*128 .. +128) followed by W3[g][mt*128 .. +128),
+// so one TMA box of 256 rows feeds both gate and up MMAs of a tile.
+__global__ void __launch_bounds__(256)
+    repack_w13_kernel(const uint4* __restrict__ w1, const uint4* __restrict__ w3, const uint4* __restrict__ sh1,
+                      const uint4* __restrict__ sh3, int E, int S, int I, int hv, uint4* __restrict__ dst) {
+  const size_t row = static_cast<size_t>(blockIdx.x) * 8 + threadIdx.x / 32;
+  const size_t total = static_cast<size_t>(E + S) * 2 * I;
+  if (row >= total) return;
+  const int g = static_cast<int>(row / (2 * I));
+  const int rr = static_cast<int>(row % (2 * I));
+  const int mt = rr / 256, within = rr % 256;
+  const int src_row = mt * 128 + (within & 127);
+  const bool up = within >= 128;
+  const uint4* base = g < E ? (up ? w3 : w1) + static_cast<size_t>(g) * I * hv
+                            : (up ? sh3 : sh1) + static_cast<size_t>(g - E) * I * hv;
+  const uint4* src = base + static_cast<size_t>(src_row) * hv;
+  uint4* d = dst + row * hv;
+  for (int c = threadIdx.x % 32; c < hv; c += 32) d[c] = __ldg(src + c);
+}
+
+// One thread per 32-element block: OCP MX rule with E2M1 elements.
+__global__ void __launch_bounds__(256)
+    quantize_mxfp4_kernel(const uint4* __restrict__ src, int64_t nblocks, uint4* __restrict__ packed,
+                          uint8_t* __restrict__ scales) {
+  const int64_t b = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (b >= nblocks) return;
+  float v[32];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const uint4 u = __ldg(src + b * 4 + q);
+    const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float2 f = __bfloat1622float2(p[i]);
+      v[q * 8 + 2 * i] = f.x;
+      v[q * 8 + 2 * i + 1] = f.y;
+    }
+  }
+  float amax = 0.f;
+#pragma unroll
+  for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(v[i]));
+  int code = 0;
+  float inv_scale = 0.f;
+  if (amax > 0.f) {
+    int ex;
+    frexpf(amax, &ex);                       // amax = f * 2^ex, f in [0.5, 1)
+    int shared = (ex - 1) - 2;               // floor(log2(amax)) - emax(E2M1)
+    shared = max(-127, min(127, shared));
+    code = shared + 127;
+    inv_scale = ldexpf(1.0f, -shared);       // exact power of two
+  }
+  uint32_t words[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    const float q = v[i] * inv_scale;
+    const float a = fabsf(q);
+    // nearest E2M1 magnitude, ties to the even code, saturating at 6
+    const uint32_t mag = (a > 0.25f) + (a >= 0.75f) + (a > 1.25f) + (a >= 1.75f) + (a > 2.5f) + (a >= 3.5f) + (a > 5.0f);
+    const uint32_t c = mag | (signbit(q) ? 8u : 0u);
+    words[i / 8] |= c << (4 * (i % 8));
+  }
+  packed[b] = make_uint4(words[0], words[1], words[2], words[3]);
+  scales[b] = static_cast<uint8_t>(code);
+}
+
+__global__ void wait_timeout_probe_kernel(int* status, unsigned long long timeout_ns) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_mbarrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    // Nothing ever arrives on `bar`: the wait must run out and report.
+    if (!mbar_wait(&bar, 0, timeout_ns)) report_status(status, kStatusTimeout);
+  }
+  __syncthreads();
+}
+
+}  // namespace
+
+cudaError_t launch_combine(const float* O, const int32_t* inv, const float* w, int T, int H, int k, int S, void* y,
+                           cudaStream_t s) {
+  if (T == 0) return cudaSuccess;
+  const int H4 = H / 4;
+  const dim3 grid(T, (H4 + 127) / 128);
+  combine_kernel<<<grid, 128, 0, s>>>(reinterpret_cast<const float4*>(O), inv, w, T, H4, k, S,
+                                      static_cast<uint2*>(y));
+  return cudaGetLastError();
+}
+
+cudaError_t launch_repack_w13(const void* w1, const void* w3, const void* sh1, const void* sh3, int E, int S, int I,
+                              int H, void* w13, cudaStream_t s) {
+  const size_t rows = static_cast<size_t>(E + S) * 2 * I;
+  repack_w13_kernel<<<static_cast<unsigned>((rows + 7) / 8), 256, 0, s>>>(
+      static_cast<const uint4*>(w1), static_cast<const uint4*>(w3), static_cast<const uint4*>(sh1),
+      static_cast<const uint4*>(sh3), E, S, I, H / 8, static_cast<uint4*>(w13));
+  return cudaGetLastError();
+}
+
+cudaError_t launch_quantize_mxfp4(const void* src, int64_t rows, int cols, uint8_t* packed, uint8_t* scales,
+                                  cudaStream_t s) {
+  const int64_t nblocks = rows * (cols / 32);
+  if (nblocks == 0) return cudaSuccess;
+  quantize_mxfp4_kernel<<<static_cast<unsigned>((nblocks + 255) / 256), 256, 0, s>>>(
+      static_cast<const uint4*>(src), nblocks, reinterpret_cast<uint4*>(packed), scales);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_wait_timeout_probe(int* status, unsigned long long timeout_ns, cudaStream_t s) {
+  wait_timeout_probe_kernel<<<1, 32, 0, s>>>(status, timeout_ns);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -1,0 +1,281 @@
+// Router: logits, sqrtsoftplus scores, top-k selection and weight normalisation.
+//
+// DeepSeek V4.1 inference/config.json: "score_func": "sqrtsoftplus",
+// "n_activated_experts": 6, "route_scale": 1.5. Computed as
+//   z_e = x . Wg_e + b_e,  s_e = sqrt(softplus(z_e)),
+//   top-k by s (ties: lower expert index), w_j = route_scale * s_j / sum_sel s.
+//
+// Two stages:
+//  1. approximate fp32 logits for all experts (CUDA cores here for small T, or
+//     the tcgen05 GEMM in dense mode for large T);
+//  2. one warp per token: fp32 scores from the approximate logits, the k-th
+//     largest score s_k, and a candidate set {e : s_e >= s_k - delta}. Every
+//     candidate's logit is recomputed exactly (BF16 x BF16 products are exact
+//     in fp32; they are summed in fp64) and the scores, the selection and the
+//     weights are taken from these fp64 values. With |approx error| < delta/2
+//     no expert outside the candidate set can belong to the true top-k, so the
+//     selection equals the exact one except on genuine fp64-level ties.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace moe {
+
+namespace {
+
+constexpr int kLogitWarps = 8;     // experts per CTA (one per warp)
+constexpr int kLogitTokens = 64;   // tokens per CTA
+constexpr int kTokPerPass = 4;     // tokens a warp accumulates at once
+
+__device__ __forceinline__ void bf16x8_to_f32(const uint4& v, float (&f)[8]) {
+  const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&v);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 t = __bfloat1622float2(p[i]);
+    f[2 * i] = t.x;
+    f[2 * i + 1] = t.y;
+  }
+}
+
+// z[t, e] = sum_h x[t, h] * wg[e, h] (+ bias[e]); fp32 accumulation per lane,
+// then a warp tree sum.
+__global__ void __launch_bounds__(kLogitWarps * 32)
+    router_logits_kernel(const uint4* __restrict__ x, const uint4* __restrict__ wg, const float* __restrict__ bias,
+                         float* __restrict__ z, int T, int H, int E) {
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int e = blockIdx.x * kLogitWarps + warp;
+  if (e >= E) return;
+  const int hv = H / 8;  // uint4 chunks per row
+  const uint4* wrow = wg + static_cast<size_t>(e) * hv;
+  const float b = bias ? bias[e] : 0.0f;
+  const int t_begin = blockIdx.y * kLogitTokens;
+  const int t_end = min(T, t_begin + kLogitTokens);
+  for (int t0 = t_begin; t0 < t_end; t0 += kTokPerPass) {
+    float acc[kTokPerPass] = {0.f, 0.f, 0.f, 0.f};
+    for (int c = lane; c < hv; c += 32) {
+      float wf[8];
+      bf16x8_to_f32(__ldg(wrow + c), wf);
+#pragma unroll
+      for (int tt = 0; tt < kTokPerPass; ++tt) {
+        if (t0 + tt < t_end) {
+          float xf[8];
+          bf16x8_to_f32(__ldg(x + static_cast<size_t>(t0 + tt) * hv + c), xf);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) acc[tt] = fmaf(xf[i], wf[i], acc[tt]);
+        }
+      }
+    }
+#pragma unroll
+    for (int tt = 0; tt < kTokPerPass; ++tt) {
+      float v = acc[tt];
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+      if (lane == 0 && t0 + tt < t_end) z[static_cast<size_t>(t0 + tt) * E + e] = v + b;
+    }
+  }
+}
+
+__device__ __forceinline__ float softplus_f32(float z) { return fmaxf(z, 0.0f) + log1pf(expf(-fabsf(z))); }
+__device__ __forceinline__ double softplus_f64(double z) { return fmax(z, 0.0) + log1p(exp(-fabs(z))); }
+
+// Warp-wide argmax over (value desc, index asc). Returns the winner on all lanes.
+__device__ __forceinline__ void warp_argmax(float& v, int& i) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const float ov = __shfl_xor_sync(0xffffffffu, v, o);
+    const int oi = __shfl_xor_sync(0xffffffffu, i, o);
+    if (ov > v || (ov == v && oi < i)) {
+      v = ov;
+      i = oi;
+    }
+  }
+}
+__device__ __forceinline__ void warp_argmax_d(double& v, int& i) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const double ov = __shfl_xor_sync(0xffffffffu, v, o);
+    const int oi = __shfl_xor_sync(0xffffffffu, i, o);
+    if (ov > v || (ov == v && oi < i)) {
+      v = ov;
+      i = oi;
+    }
+  }
+}
+
+constexpr int kTopkWarps = 8;
+constexpr int kMaxCand = 64;       // candidates refined per token
+constexpr int kMaxEPL = 16;        // experts per lane (E <= 512)
+constexpr int kMaxK = 32;
+
+template <int EPL>
+__global__ void __launch_bounds__(kTopkWarps * 32)
+    topk_refine_kernel(const float* __restrict__ z, const uint4* __restrict__ x, const uint4* __restrict__ wg,
+                       const float* __restrict__ bias, int T, int H, int E, int k, float route_scale, float delta,
+                       int32_t* __restrict__ idx_out, float* __restrict__ w_out, int* status) {
+  __shared__ int cand_s[kTopkWarps][kMaxCand];
+  __shared__ double cs_s[kTopkWarps][kMaxCand];
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int t = blockIdx.x * kTopkWarps + warp;
+  if (t >= T) return;
+  int* cand = cand_s[warp];
+  double* cs = cs_s[warp];
+
+  // 1. approximate scores
+  float s[EPL];
+#pragma unroll
+  for (int i = 0; i < EPL; ++i) {
+    const int e = lane + 32 * i;
+    s[i] = e < E ? sqrtf(softplus_f32(z[static_cast<size_t>(t) * E + e])) : -INFINITY;
+  }
+  // 2. k-th largest approximate score
+  float kth = 0.f;
+  {
+    float tmp[EPL];
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) tmp[i] = s[i];
+    for (int r = 0; r < k; ++r) {
+      float bv = -INFINITY;
+      int bi = 0x7fffffff;
+#pragma unroll
+      for (int i = 0; i < EPL; ++i) {
+        const int e = lane + 32 * i;
+        if (tmp[i] > bv || (tmp[i] == bv && e < bi)) {
+          bv = tmp[i];
+          bi = e;
+        }
+      }
+      warp_argmax(bv, bi);
+      kth = bv;
+#pragma unroll
+      for (int i = 0; i < EPL; ++i)
+        if (lane + 32 * i == bi) tmp[i] = -INFINITY;
+    }
+  }
+  // 3. candidates in ascending expert order
+  const float thr = kth - delta;
+  int ncand = 0;
+#pragma unroll
+  for (int i = 0; i < EPL; ++i) {
+    const bool f = s[i] >= thr;
+    const unsigned m = __ballot_sync(0xffffffffu, f);
+    const int pos = ncand + __popc(m & ((1u << lane) - 1u));
+    if (f && pos < kMaxCand) cand[pos] = lane + 32 * i;
+    ncand += __popc(m);
+  }
+  if (ncand > kMaxCand) {
+    // Degenerate router (more than kMaxCand experts within delta of the k-th
+    // score): keep the kMaxCand best by approximate score, lower index first.
+    float tmp[EPL];
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) tmp[i] = s[i];
+    for (int r = 0; r < kMaxCand; ++r) {
+      float bv = -INFINITY;
+      int bi = 0x7fffffff;
+#pragma unroll
+      for (int i = 0; i < EPL; ++i) {
+        const int e = lane + 32 * i;
+        if (tmp[i] > bv || (tmp[i] == bv && e < bi)) {
+          bv = tmp[i];
+          bi = e;
+        }
+      }
+      warp_argmax(bv, bi);
+      if (lane == 0) cand[r] = bi;
+#pragma unroll
+      for (int i = 0; i < EPL; ++i)
+        if (lane + 32 * i == bi) tmp[i] = -INFINITY;
+    }
+    ncand = kMaxCand;
+  }
+  __syncwarp();
+
+  // 4. exact logits of the candidates: fp32 products (exact), fp64 sums
+  const int hv = H / 8;
+  const uint4* xrow = x + static_cast<size_t>(t) * hv;
+  for (int c = 0; c < ncand; ++c) {
+    const int e = cand[c];
+    const uint4* wrow = wg + static_cast<size_t>(e) * hv;
+    double acc = 0.0;
+    for (int j = lane; j < hv; j += 32) {
+      float xf[8], wf[8];
+      bf16x8_to_f32(__ldg(xrow + j), xf);
+      bf16x8_to_f32(__ldg(wrow + j), wf);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) acc += static_cast<double>(xf[i] * wf[i]);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    if (lane == 0) {
+      const double zz = acc + (bias ? static_cast<double>(bias[e]) : 0.0);
+      cs[c] = sqrt(softplus_f64(zz));
+    }
+  }
+  __syncwarp();
+
+  // 5. exact top-k among the candidates, then the weights
+  double v0 = lane < ncand ? cs[lane] : -INFINITY;
+  double v1 = lane + 32 < ncand ? cs[lane + 32] : -INFINITY;
+  const int e0 = lane < ncand ? cand[lane] : 0x7fffffff;
+  const int e1 = lane + 32 < ncand ? cand[lane + 32] : 0x7fffffff;
+  double sel_s[kMaxK];
+  int sel_e[kMaxK];
+  double sum = 0.0;
+  for (int r = 0; r < k; ++r) {
+    double bv;
+    int bi;
+    if (v0 > v1 || (v0 == v1 && e0 < e1)) {
+      bv = v0;
+      bi = e0;
+    } else {
+      bv = v1;
+      bi = e1;
+    }
+    warp_argmax_d(bv, bi);
+    if (e0 == bi) v0 = -INFINITY;
+    if (e1 == bi) v1 = -INFINITY;
+    sel_s[r] = bv;
+    sel_e[r] = bi;
+    sum += bv;
+  }
+  if (lane == 0) {
+    for (int r = 0; r < k; ++r) {
+      const int e = sel_e[r];
+      if (e < 0 || e >= E) report_status(status, kStatusDevice);
+      idx_out[static_cast<size_t>(t) * k + r] = e;
+      w_out[static_cast<size_t>(t) * k + r] = static_cast<float>(route_scale * (sel_s[r] / sum));
+    }
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_router_logits(const void* x, const void* wg, const float* bias, float* z, int T, int H, int E,
+                                 cudaStream_t s) {
+  dim3 grid((E + kLogitWarps - 1) / kLogitWarps, (T + kLogitTokens - 1) / kLogitTokens);
+  router_logits_kernel<<<grid, kLogitWarps * 32, 0, s>>>(static_cast<const uint4*>(x), static_cast<const uint4*>(wg),
+                                                         bias, z, T, H, E);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_topk_refine(const float* z, const void* x, const void* wg, const float* bias, int T, int H,
+                               int E, int k, float route_scale, float delta, int32_t* idx, float* w, int* status,
+                               cudaStream_t s) {
+  if (k > kMaxK || E > 32 * kMaxEPL) return cudaErrorInvalidValue;
+  const dim3 grid((T + kTopkWarps - 1) / kTopkWarps);
+  const uint4* xv = static_cast<const uint4*>(x);
+  const uint4* wv = static_cast<const uint4*>(wg);
+  const int epl = (E + 31) / 32;
+#define MOE_TOPK_CASE(N)                                                                                 \
+  if (epl <= N) {                                                                                        \
+    topk_refine_kernel<N><<<grid, kTopkWarps * 32, 0, s>>>(z, xv, wv, bias, T, H, E, k, route_scale, delta, \
+                                                           idx, w, status);                              \
+    return cudaGetLastError();                                                                           \
+  }
+  MOE_TOPK_CASE(1)
+  MOE_TOPK_CASE(4)
+  MOE_TOPK_CASE(12)
+  MOE_TOPK_CASE(16)
+#undef MOE_TOPK_CASE
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace moe

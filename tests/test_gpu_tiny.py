@@ -1,0 +1,200 @@
+"""GPU parity of the whole layer and of each stage on the tiny workload
+(T=64, H=512, I=256, 32 routed + 1 shared, top-6), through the C ABI."""
+import numpy as np
+import pytest
+import torch
+
+import routed_expert_ffn_sqrtsoftplus_b200 as moe
+from routed_expert_ffn_sqrtsoftplus_b200 import synth
+from oracle import moe as om
+from oracle import mx as omx
+
+import parity
+
+pytestmark = pytest.mark.gpu
+
+WL = synth.WORKLOADS["tiny"]
+
+
+@pytest.fixture(scope="module")
+def tiny(cuda_device):
+    from routed_expert_ffn_sqrtsoftplus_b200 import build
+    build.build()
+    lay = synth.make_layer(WL.with_tokens(700), device="cpu")
+    lay = {k: (v.to(cuda_device) if isinstance(v, torch.Tensor) else v) for k, v in lay.items()}
+    layer = moe.MoELayer.from_layer(lay, top_k=WL.k, max_tokens=700)
+    yield lay, layer
+    layer.close()
+
+
+def _run(layer, x):
+    y, idx, w = layer.forward_with_routing(x)
+    torch.cuda.synchronize()
+    assert layer.status() == moe.MOE_OK
+    return y, idx, w
+
+
+@pytest.mark.parametrize("T", [64, 1, 3, 17, 63, 33, 129])
+def test_tiny_layer_parity(tiny, T):
+    lay, layer = tiny
+    x = lay["x"][:T].contiguous()
+    y, idx, w = _run(layer, x)
+    sub = dict(lay, x=x)
+    rep = parity.compare_layer(sub, np.arange(T), y.float().cpu().numpy(), idx.cpu().numpy(), w.cpu().numpy(),
+                               WL.k, WL.route_scale, WL.swiglu_limit)
+    assert rep["rel"] < parity.TOL_Y
+
+
+@pytest.mark.parametrize("T", [300, 700])
+def test_tiny_layer_parity_large_T(tiny, T):
+    """T >= 256 takes the tensor-core router and the 128/256-token GEMM tiles."""
+    lay, layer = tiny
+    x = lay["x"][:T].contiguous()
+    y, idx, w = _run(layer, x)
+    rep = parity.compare_layer(dict(lay, x=x), np.arange(T), y.float().cpu().numpy(), idx.cpu().numpy(),
+                               w.cpu().numpy(), WL.k, WL.route_scale, WL.swiglu_limit)
+    assert rep["rel"] < parity.TOL_Y
+
+
+@pytest.mark.parametrize("T", [64, 300])
+def test_permutation_is_exact(tiny, T):
+    lay, layer = tiny
+    x = lay["x"][:T].contiguous()
+    _, idx, _ = _run(layer, x)
+    G = WL.E + WL.n_shared
+    cnt = layer.inspect(moe.BUF_COUNTS, torch.empty(G, dtype=torch.int32, device=x.device)).cpu().numpy()
+    off = layer.inspect(moe.BUF_OFFSETS, torch.empty(G + 1, dtype=torch.int32, device=x.device)).cpu().numpy()
+    perm = layer.inspect(moe.BUF_PERM, torch.empty(T * WL.k, dtype=torch.int32, device=x.device)).cpu().numpy()
+    inv = layer.inspect(moe.BUF_INV, torch.empty(T * WL.k, dtype=torch.int32, device=x.device)).cpu().numpy()
+    torch.cuda.synchronize()
+    c_ref, o_ref, p_ref, i_ref = om.permutation_reference(idx.cpu().numpy(), WL.E)
+    assert np.array_equal(cnt[:WL.E], c_ref) and np.all(cnt[WL.E:] == T)
+    assert np.array_equal(off[:WL.E + 1], o_ref)
+    assert np.array_equal(off[WL.E + 1:], T * WL.k + T * np.arange(1, WL.n_shared + 1))
+    assert np.array_equal(perm, p_ref)
+    assert np.array_equal(inv, i_ref)
+
+
+def test_swiglu_rows_match_oracle(tiny):
+    """The gate/up GEMM's epilogue output h, row by row, against the oracle's h."""
+    lay, layer = tiny
+    T = 64
+    x = lay["x"][:T].contiguous()
+    _, idx, _ = _run(layer, x)
+    R = T * WL.k + WL.n_shared * T
+    h = layer.inspect(moe.BUF_H, torch.empty((R, WL.I), dtype=torch.bfloat16, device=x.device))
+    perm = layer.inspect(moe.BUF_PERM, torch.empty(T * WL.k, dtype=torch.int32, device=x.device))
+    torch.cuda.synchronize()
+    h = parity.f64(h)
+    perm = perm.cpu().numpy()
+    idx = idx.cpu().numpy()
+    xf = parity.f64(x)
+    ex = parity.LayerExperts(lay)
+    worst = 0.0
+    for e in range(WL.E):
+        rows = np.nonzero(idx.reshape(-1)[perm] == e)[0]
+        if len(rows) == 0:
+            continue
+        toks = perm[rows] // WL.k
+        _, h_or = om.expert_forward(xf[toks], *ex.routed(e), WL.swiglu_limit)
+        worst = max(worst, np.abs(h[rows] - h_or).max() / np.sqrt(np.mean(h_or ** 2)))
+    _, h_sh = om.expert_forward(xf, *ex.shared(0), WL.swiglu_limit)
+    worst = max(worst, np.abs(h[T * WL.k:] - h_sh).max() / np.sqrt(np.mean(h_sh ** 2)))
+    assert worst < parity.TOL_Y, worst
+
+
+def test_deterministic(tiny):
+    lay, layer = tiny
+    x = lay["x"][:300].contiguous()
+    y1, i1, w1 = _run(layer, x)
+    y2, i2, w2 = _run(layer, x)
+    assert torch.equal(y1, y2) and torch.equal(i1, i2) and torch.equal(w1, w2)
+
+
+def test_token_order_invariance(tiny):
+    lay, layer = tiny
+    T = 64
+    x = lay["x"][:T].contiguous()
+    p = torch.randperm(T, generator=torch.Generator().manual_seed(0)).to(x.device)
+    y, idx, w = _run(layer, x)
+    yp, idxp, wp = _run(layer, x[p].contiguous())
+    assert torch.equal(idxp, idx[p]) and torch.equal(wp, w[p])
+    assert torch.allclose(yp.float(), y[p].float(), rtol=0, atol=0)
+
+
+def test_zero_tokens(tiny):
+    lay, layer = tiny
+    x = lay["x"][:0]
+    y = layer.forward(x)
+    torch.cuda.synchronize()
+    assert y.shape == (0, WL.H)
+    assert layer.status() == moe.MOE_OK
+
+
+def test_rejects_too_many_tokens(tiny):
+    lay, layer = tiny
+    x = torch.zeros((701, WL.H), dtype=torch.bfloat16, device=lay["x"].device)
+    with pytest.raises(moe.MoEError) as ei:
+        layer.forward(x)
+    assert ei.value.status == moe.MOE_ERR_INVALID_ARG
+
+
+def test_forward_host_matches_device(tiny):
+    lay, layer = tiny
+    T = 17
+    x = lay["x"][:T].contiguous()
+    y, idx, w = _run(layer, x)
+    xh = x.cpu().pin_memory()
+    yh = torch.empty((T, WL.H), dtype=torch.bfloat16).pin_memory()
+    ih = torch.empty((T, WL.k), dtype=torch.int32).pin_memory()
+    layer.forward_host(xh, yh, ih)
+    torch.cuda.synchronize()
+    assert torch.equal(yh, y.cpu()) and torch.equal(ih, idx.cpu())
+
+
+def test_bounded_wait_reports_timeout(tiny):
+    _, layer = tiny
+    assert layer.status() == moe.MOE_OK
+    layer.selftest_wait_timeout(2_000_000)   # 2 ms wait that nothing completes
+    assert layer.status() == moe.MOE_ERR_TIMEOUT
+    assert layer.status() == moe.MOE_OK      # reading clears it
+
+
+def test_router_tie_break_lower_index(cuda_device):
+    """Identical router rows tie exactly: the lower expert index must win."""
+    H, I, E, S, k = 128, 128, 8, 1, 2
+    g = torch.Generator().manual_seed(4)
+    x = torch.randn((5, H), generator=g).to(torch.bfloat16)
+    wg = torch.randn((E, H), generator=g).to(torch.bfloat16) * 0.0
+    wg[3] = wg[6] = wg[1] = 0.5        # three identical best rows
+    w1 = (torch.randn((E, I, H), generator=g) / 11).to(torch.bfloat16)
+    w3 = (torch.randn((E, I, H), generator=g) / 11).to(torch.bfloat16)
+    w2 = (torch.randn((E, H, I), generator=g) / 11).to(torch.bfloat16)
+    sh = [(torch.randn(s, generator=g) / 11).to(torch.bfloat16) for s in ((S, I, H), (S, I, H), (S, H, I))]
+    d = {n: t.to(cuda_device) for n, t in dict(x=x, wg=wg, w1=w1, w3=w3, w2=w2, sh_w1=sh[0], sh_w3=sh[1],
+                                                sh_w2=sh[2]).items()}
+    layer = moe.MoELayer.from_layer(d, top_k=k, max_tokens=8)
+    y, idx, w = layer.forward_with_routing(d["x"])
+    torch.cuda.synchronize()
+    idx = idx.cpu().numpy()
+    # tokens whose x . row > 0 pick 1 then 3; otherwise all scores tie at sqrt(ln 2) -> 0, 1
+    for t in range(5):
+        z = float((x[t].double() * 0.5).sum())
+        assert list(idx[t]) == ([1, 3] if z > 0 else [0, 1] if z < 0 else [0, 1])
+    rep = parity.compare_layer(d, np.arange(5), y.float().cpu().numpy(), idx, w.cpu().numpy(), k, 1.5, 10.0)
+    layer.close()
+
+
+def test_quantize_mxfp4_bitexact(cuda_device):
+    g = torch.Generator().manual_seed(11)
+    w = (torch.randn((48, 512), generator=g) * 0.03).to(torch.bfloat16)
+    w[3, :32] = 0                                  # all-zero block
+    w[4, 32:64] = 7.0                              # saturating block
+    w[5, 64:96] = torch.tensor([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0, -0.25] * 4)   # E2M1 midpoints at scale 1
+    w[5, 64] = 4.0                                 # amax 4 -> scale code 127
+    w[6, :32] = torch.finfo(torch.bfloat16).tiny   # smallest normal BF16
+    q, s = moe.quantize_mxfp4(w.to(cuda_device))
+    torch.cuda.synchronize()
+    q_ref, s_ref = omx.quantize_mxfp4_packed(parity.f64(w))
+    assert np.array_equal(s.cpu().numpy(), s_ref)
+    assert np.array_equal(q.cpu().numpy(), q_ref)
