@@ -90,17 +90,20 @@ def test_swiglu_rows_match_oracle(tiny):
     idx = idx.cpu().numpy()
     xf = parity.f64(x)
     ex = parity.LayerExperts(lay)
-    worst = 0.0
+    # h is stored in BF16: each element carries at most 2^-9 relative rounding,
+    # plus fp32 accumulation error far below it
+    def check(h_gpu, h_or):
+        bound = 2.0 ** -8 * np.abs(h_or) + 1e-3 * np.sqrt(np.mean(h_or ** 2))
+        assert np.all(np.abs(h_gpu - h_or) <= bound), np.max(np.abs(h_gpu - h_or) / bound)
     for e in range(WL.E):
         rows = np.nonzero(idx.reshape(-1)[perm] == e)[0]
         if len(rows) == 0:
             continue
         toks = perm[rows] // WL.k
         _, h_or = om.expert_forward(xf[toks], *ex.routed(e), WL.swiglu_limit)
-        worst = max(worst, np.abs(h[rows] - h_or).max() / np.sqrt(np.mean(h_or ** 2)))
+        check(h[rows], h_or)
     _, h_sh = om.expert_forward(xf, *ex.shared(0), WL.swiglu_limit)
-    worst = max(worst, np.abs(h[T * WL.k:] - h_sh).max() / np.sqrt(np.mean(h_sh ** 2)))
-    assert worst < parity.TOL_Y, worst
+    check(h[T * WL.k:], h_sh)
 
 
 def test_deterministic(tiny):
@@ -177,10 +180,11 @@ def test_router_tie_break_lower_index(cuda_device):
     y, idx, w = layer.forward_with_routing(d["x"])
     torch.cuda.synchronize()
     idx = idx.cpu().numpy()
-    # tokens whose x . row > 0 pick 1 then 3; otherwise all scores tie at sqrt(ln 2) -> 0, 1
+    # z = x . row for rows 1, 3, 6 and 0 for the rest: z > 0 picks 1 then 3 (three-way
+    # tie, lowest indices win); z < 0 leaves the zero-logit experts 0, 2, 4, 5, 7 tied on top
     for t in range(5):
         z = float((x[t].double() * 0.5).sum())
-        assert list(idx[t]) == ([1, 3] if z > 0 else [0, 1] if z < 0 else [0, 1])
+        assert list(idx[t]) == ([1, 3] if z > 0 else [0, 2] if z < 0 else [0, 1])
     rep = parity.compare_layer(d, np.arange(5), y.float().cpu().numpy(), idx, w.cpu().numpy(), k, 1.5, 10.0)
     layer.close()
 
