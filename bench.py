@@ -51,6 +51,8 @@ def parse():
     p.add_argument("--workload", default="flash_decode", choices=sorted(synth.WORKLOADS))
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--tokens", type=int, default=None, help="override T of the workload")
+    p.add_argument("--experts", type=int, default=None,
+                   help="override the routed expert count (small instances for profiler captures)")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-seconds", type=float, default=15.0, help="budget of the CPU baseline sample")
     return p.parse_args()
@@ -140,6 +142,16 @@ class ClockSampler:
 
 
 # ----------------------------------------------------------------------------- workload
+def workload_from_args(args):
+    import dataclasses
+    wl = synth.WORKLOADS[args.workload]
+    if args.tokens:
+        wl = wl.with_tokens(args.tokens)
+    if args.experts:
+        wl = dataclasses.replace(wl, E=args.experts, name=f"{wl.name}_e{args.experts}")
+    return wl
+
+
 def build_layer(wl, device):
     d = synth.make_layer(wl, device=device)
     mxq = None
@@ -242,9 +254,7 @@ def run_ours(args, world, rank, local):
     if rank == 0:
         build.build()
     barrier(world)
-    wl = synth.WORKLOADS[args.workload]
-    if args.tokens:
-        wl = wl.with_tokens(args.tokens)
+    wl = workload_from_args(args)
     T = wl.T
     dev = torch.device("cuda", local)
     d, mxq = build_layer(wl, dev)
@@ -360,9 +370,7 @@ def run_ours(args, world, rank, local):
 
 def run_reference(args, world, rank, local):
     """The float64 CPU oracle as the reference arm, on rank 0 only."""
-    wl = synth.WORKLOADS[args.workload]
-    if args.tokens:
-        wl = wl.with_tokens(args.tokens)
+    wl = workload_from_args(args)
     if rank != 0:
         return None
     dev = torch.device("cuda", local)
