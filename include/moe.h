@@ -232,6 +232,44 @@ MOE_API moe_status moe_profile_end(moe_handle* h, double* ms, int64_t* launches,
 MOE_API int32_t moe_num_kernel_kinds(void);
 MOE_API const char* moe_kernel_name(int32_t kind);
 
+/* ------------------------------------------------------------------------
+ * Routing without device allocation
+ * ---------------------------------------------------------------------- */
+
+/*
+ * Routing alone (router logits, sqrtsoftplus scores, top-k and the
+ * route_scale-normalised weights) for callers that cannot allocate device
+ * memory: code whose device memory all belongs to a host framework's pool (a
+ * raw cudaMalloc there can fail or fragment that pool), loops that forbid any
+ * allocation once they have started, and callers that cannot accept the
+ * device-wide synchronisation cudaMalloc or cudaFree may cause. The pages have
+ * no counterpart of this entry point; it is an addition of this library.
+ *
+ *   x           BF16 [T, hidden], device, 16-byte aligned
+ *   router_w    BF16 [n_routed, hidden], device, 16-byte aligned
+ *   router_bias fp32 [n_routed] device, or NULL
+ *   topk_idx    int32 [T, top_k] device (output), descending score
+ *   topk_w      fp32  [T, top_k] device (output), sum = route_scale
+ * hidden % 8 == 0, 1 <= top_k <= min(n_routed, 32), n_routed <= 512. The
+ * results equal moe_forward's topk_idx / topk_w for the same inputs.
+ *
+ * The only scratch, the fp32 logits [T, n_routed], lives in a fixed array of
+ * MOE_NOALLOC_MAX_LOGITS floats (4 MiB) inside the library; every GPU that
+ * loads the library holds it until the process exits. T * n_routed above
+ * MOE_NOALLOC_MAX_LOGITS returns MOE_ERR_UNSUPPORTED and enqueues nothing.
+ * Nothing is allocated, by this call or by anything it calls. The first call
+ * on a device looks up the array's device address once for that device (with
+ * that device current); make that first call before any stream capture. All
+ * calls share the one array, and each call writes every entry it later reads,
+ * so nothing needs clearing between calls; calls that overlap on the GPU (on
+ * streams not ordered with each other) race on it.
+ */
+#define MOE_NOALLOC_MAX_LOGITS (1 << 20)
+
+MOE_API moe_status moe_route_noalloc(const void* x, const void* router_w, const float* router_bias, int32_t T,
+                                     int32_t hidden, int32_t n_routed, int32_t top_k, float route_scale,
+                                     int32_t* topk_idx, float* topk_w, moe_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -32,7 +32,7 @@ BUF_LOGITS, BUF_TOPK_IDX, BUF_TOPK_W, BUF_COUNTS, BUF_OFFSETS, BUF_PERM, BUF_INV
 EXPORTED = ("moe_create", "moe_forward", "moe_forward_host", "moe_get_status", "moe_status_string",
             "moe_destroy", "moe_abi_version", "moe_quantize_mxfp4", "moe_inspect", "moe_set_wait_timeout",
             "moe_selftest_wait_timeout", "moe_get_info", "moe_profile_begin", "moe_profile_end",
-            "moe_num_kernel_kinds", "moe_kernel_name")
+            "moe_num_kernel_kinds", "moe_kernel_name", "moe_route_noalloc")
 
 
 class MoEError(RuntimeError):
@@ -88,6 +88,7 @@ def lib() -> ctypes.CDLL:
             "moe_profile_end": (I32, [P, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(I64), I32]),
             "moe_num_kernel_kinds": (I32, []),
             "moe_kernel_name": (ctypes.c_char_p, [I32]),
+            "moe_route_noalloc": (I32, [P, P, P, I32, I32, I32, I32, ctypes.c_float, P, P, P]),
         }
         for name, (res, args) in sig.items():
             f = getattr(L, name)
