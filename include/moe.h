@@ -187,8 +187,8 @@ typedef enum {
   MOE_BUF_PERM = 5,     /* int32 [T*k] flat slot t*k+j of each routed row (expert-major) */
   MOE_BUF_INV = 6,      /* int32 [T*k] row of each flat slot */
   MOE_BUF_H = 7,        /* BF16 [T*k + n_shared*T, I] SwiGLU output rows (group order) */
-  MOE_BUF_XQ = 8,       /* MXFP4 layers: uint8 E4M3 [T, H] MXFP8 codes of x */
-  MOE_BUF_XQ_SCALES = 9 /* MXFP4 layers: uint8 E8M0 [T, H/32] */
+  MOE_BUF_XQ = 8,       /* MXFP4 layers: uint8 E4M3 [T*k, H], MXFP8 codes of the routed rows (perm order) */
+  MOE_BUF_XQ_SCALES = 9 /* MXFP4 layers: their E8M0 scales, packed in 512-byte atoms per token tile */
 } moe_buffer;
 
 /*

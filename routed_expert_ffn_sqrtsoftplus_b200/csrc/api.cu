@@ -55,7 +55,22 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 
 const char* kKernelNames[kKNumKinds] = {"router_logits", "router_gemm",  "topk_refine", "perm_count",
                                         "perm_scan",     "perm_scatter", "gather_rows", "gemm_gateup",
-                                        "gemm_down",     "combine",      "quant_x"};
+                                        "gemm_down",     "combine",      "quant_x",     "gemm_gateup_mx",
+                                        "gemm_down_mx"};
+
+// 2-D tensor map, 128-byte swizzle, box of box_cols x box_rows elements.
+bool make_tmap(CUtensorMap* m, const void* ptr, CUtensorMapDataType dt, uint64_t rows, uint64_t cols,
+               uint64_t row_bytes, uint32_t box_cols, uint32_t box_rows) {
+  EncodeTiledFn enc = get_encode_fn();
+  if (enc == nullptr) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {row_bytes};
+  cuuint32_t box[2] = {box_cols, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(m, dt, 2, const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
 
 }  // namespace
 
@@ -93,6 +108,24 @@ struct moe_handle {
   void* y_stage = nullptr;
 
   CUtensorMap tm_w13, tm_w2, tm_xp, tm_h, tm_wg;
+
+  // MXFP4 routed experts (expert_dtype == MOE_DT_MXFP4)
+  bool mx = false;
+  uint8_t* w13q = nullptr;      // packed E2M1, gate/up tile order
+  uint8_t* w2q = nullptr;       // packed E2M1
+  uint8_t* sfa13 = nullptr;     // scale atoms of W1|W3
+  uint8_t* sfa2 = nullptr;      // scale atoms of W2
+  void* w13sh = nullptr;        // shared experts, BF16
+  void* w2sh = nullptr;
+  uint8_t* xq = nullptr;        // MXFP8 routed token rows
+  uint8_t* hq = nullptr;        // MXFP8 routed h rows
+  uint8_t* sfb_gu = nullptr;    // activation scale atoms, gate/up token tiles
+  uint8_t* sfb_dn = nullptr;    // h scale atoms, down token tiles
+  int32_t* ntile_base_gu = nullptr;
+  int32_t* ntile_base_dn = nullptr;
+  int* bad = nullptr;
+  int64_t max_ntiles_r = 0;
+  CUtensorMap tm_w13q, tm_w2q, tm_xq, tm_hq, tm_w13sh, tm_w2sh;
   uint64_t timeout_ns = 2000000000ull;
   std::vector<void*> allocs;
   uint64_t weight_bytes = 0, workspace_bytes = 0;
@@ -150,7 +183,6 @@ moe_status validate_config(const moe_config* c) {
   if (c->n_routed > 512 || c->top_k > 32 || c->n_shared > 4 || c->max_tokens > 65536) return MOE_ERR_UNSUPPORTED;
   if (c->hidden > 16384 || c->inter > 16384) return MOE_ERR_UNSUPPORTED;
   if (c->expert_dtype != MOE_DT_BF16 && c->expert_dtype != MOE_DT_MXFP4) return MOE_ERR_INVALID_ARG;
-  if (c->expert_dtype == MOE_DT_MXFP4) return MOE_ERR_UNSUPPORTED;
   return MOE_OK;
 }
 
@@ -194,9 +226,11 @@ moe_status moe_create(const moe_config* cfg, const moe_weights* w, moe_stream_t 
   if (cfg == nullptr || w == nullptr) return MOE_ERR_INVALID_ARG;
   moe_status st = validate_config(cfg);
   if (st != MOE_OK) return st;
+  const bool mx = cfg->expert_dtype == MOE_DT_MXFP4;
   const void* req[] = {w->router_w, w->w1, w->w3, w->w2};
   for (const void* p : req)
     if (p == nullptr || !aligned16(p)) return MOE_ERR_INVALID_ARG;
+  if (mx && (w->s1 == nullptr || w->s3 == nullptr || w->s2 == nullptr)) return MOE_ERR_INVALID_ARG;
   if (cfg->n_shared > 0) {
     const void* sh[] = {w->sh_w1, w->sh_w3, w->sh_w2};
     for (const void* p : sh)
@@ -209,13 +243,10 @@ moe_status moe_create(const moe_config* cfg, const moe_weights* w, moe_stream_t 
   moe_handle* h = new (std::nothrow) moe_handle();
   if (h == nullptr) return MOE_ERR_OOM;
   h->cfg = *cfg;
+  h->mx = mx;
   if (cudaGetDevice(&h->device) != cudaSuccess ||
-      cudaDeviceGetAttribute(&h->num_sms, cudaDevAttrMultiProcessorCount, h->device) != cudaSuccess) {
-    cudaGetLastError();
-    delete h;
-    return MOE_ERR_CUDA;
-  }
-  if (gemm_set_attributes() != cudaSuccess) {
+      cudaDeviceGetAttribute(&h->num_sms, cudaDevAttrMultiProcessorCount, h->device) != cudaSuccess ||
+      gemm_set_attributes() != cudaSuccess || gemm_mx_set_attributes() != cudaSuccess) {
     cudaGetLastError();
     delete h;
     return MOE_ERR_CUDA;
@@ -229,14 +260,34 @@ moe_status moe_create(const moe_config* cfg, const moe_weights* w, moe_stream_t 
   h->m_tiles_dn = static_cast<int>(H / 128);
   h->max_tiles_gu = h->m_tiles_gu * (h->G + (h->R + 31) / 32);
   h->max_tiles_dn = h->m_tiles_dn * (h->G + (h->R + 31) / 32);
+  h->max_ntiles_r = E + (Tm * k + 31) / 32;
 
   bool ok = true;
   uint64_t* wb = &h->weight_bytes;
   uint64_t* ws = &h->workspace_bytes;
   ok = ok && h->alloc(&h->wg, E * H * 2, wb);
   if (w->router_bias) ok = ok && h->alloc(&h->bias, E * 4, wb);
-  ok = ok && h->alloc(&h->w13, (E + S) * 2 * I * H * 2, wb);
-  ok = ok && h->alloc(&h->w2, (E + S) * H * I * 2, wb);
+  if (!mx) {
+    ok = ok && h->alloc(&h->w13, (E + S) * 2 * I * H * 2, wb);
+    ok = ok && h->alloc(&h->w2, (E + S) * H * I * 2, wb);
+    ok = ok && h->alloc(&h->xp, Tm * k * H * 2, ws);
+  } else {
+    ok = ok && h->alloc(&h->w13q, E * 2 * I * H / 2, wb);
+    ok = ok && h->alloc(&h->w2q, E * H * I / 2, wb);
+    ok = ok && h->alloc(&h->sfa13, E * (I / 128) * (H / 128) * 1024, wb);
+    ok = ok && h->alloc(&h->sfa2, E * (H / 128) * (I / 128) * 512, wb);
+    if (S > 0) {
+      ok = ok && h->alloc(&h->w13sh, S * 2 * I * H * 2, wb);
+      ok = ok && h->alloc(&h->w2sh, S * H * I * 2, wb);
+    }
+    ok = ok && h->alloc(&h->xq, Tm * k * H, ws);
+    ok = ok && h->alloc(&h->hq, Tm * k * I, ws);
+    ok = ok && h->alloc(&h->sfb_gu, h->max_ntiles_r * (H / 128) * 512, ws);
+    ok = ok && h->alloc(&h->sfb_dn, h->max_ntiles_r * (I / 128) * 512, ws);
+    ok = ok && h->alloc(&h->ntile_base_gu, (E + 1) * 4, ws);
+    ok = ok && h->alloc(&h->ntile_base_dn, (E + 1) * 4, ws);
+    ok = ok && h->alloc(&h->bad, 16, ws);
+  }
   ok = ok && h->alloc(&h->z, Tm * E * 4, ws);
   ok = ok && h->alloc(&h->idx, Tm * k * 4, ws);
   ok = ok && h->alloc(&h->wts, Tm * k * 4, ws);
@@ -248,7 +299,6 @@ moe_status moe_create(const moe_config* cfg, const moe_weights* w, moe_stream_t 
   ok = ok && h->alloc(&h->tiles_gu, h->max_tiles_gu * 16, ws);
   ok = ok && h->alloc(&h->tiles_dn, h->max_tiles_dn * 16, ws);
   ok = ok && h->alloc(&h->ntiles, 16, ws);
-  ok = ok && h->alloc(&h->xp, Tm * k * H * 2, ws);
   ok = ok && h->alloc(&h->h, h->R * I * 2, ws);
   ok = ok && h->alloc(&h->o, h->R * H * 4, ws);
   ok = ok && h->alloc(&h->status, 16, ws);
@@ -262,22 +312,53 @@ moe_status moe_create(const moe_config* cfg, const moe_weights* w, moe_stream_t 
 
   bool err = false;
   err |= cudaMemsetAsync(h->status, 0, 16, s) != cudaSuccess;
+  err |= cudaMemsetAsync(h->ntiles, 0, 16, s) != cudaSuccess;
   err |= cudaMemcpyAsync(h->wg, w->router_w, E * H * 2, cudaMemcpyDeviceToDevice, s) != cudaSuccess;
   if (w->router_bias) err |= cudaMemcpyAsync(h->bias, w->router_bias, E * 4, cudaMemcpyDeviceToDevice, s) != cudaSuccess;
-  err |= launch_repack_w13(w->w1, w->w3, w->sh_w1, w->sh_w3, static_cast<int>(E), static_cast<int>(S),
-                           static_cast<int>(I), static_cast<int>(H), h->w13, s) != cudaSuccess;
-  err |= cudaMemcpyAsync(h->w2, w->w2, E * H * I * 2, cudaMemcpyDeviceToDevice, s) != cudaSuccess;
-  if (S > 0)
-    err |= cudaMemcpyAsync(static_cast<uint8_t*>(h->w2) + E * H * I * 2, w->sh_w2, S * H * I * 2,
-                           cudaMemcpyDeviceToDevice, s) != cudaSuccess;
-  // The tile lists are rewritten by every forward; zero them once so a stale
-  // read can never see uninitialised memory.
-  err |= cudaMemsetAsync(h->ntiles, 0, 16, s) != cudaSuccess;
-  err |= !make_tmap_bf16(&h->tm_w13, h->w13, (E + S) * 2 * I, H, 256);
-  err |= !make_tmap_bf16(&h->tm_w2, h->w2, (E + S) * H, I, 128);
-  err |= !make_tmap_bf16(&h->tm_xp, h->xp, Tm * k, H, 32);
+  if (!mx) {
+    err |= launch_repack_w13(w->w1, w->w3, w->sh_w1, w->sh_w3, static_cast<int>(E), static_cast<int>(S),
+                             static_cast<int>(I), static_cast<int>(H), h->w13, s) != cudaSuccess;
+    err |= cudaMemcpyAsync(h->w2, w->w2, E * H * I * 2, cudaMemcpyDeviceToDevice, s) != cudaSuccess;
+    if (S > 0)
+      err |= cudaMemcpyAsync(static_cast<uint8_t*>(h->w2) + E * H * I * 2, w->sh_w2, S * H * I * 2,
+                             cudaMemcpyDeviceToDevice, s) != cudaSuccess;
+    err |= !make_tmap_bf16(&h->tm_w13, h->w13, (E + S) * 2 * I, H, 256);
+    err |= !make_tmap_bf16(&h->tm_w2, h->w2, (E + S) * H, I, 128);
+    err |= !make_tmap_bf16(&h->tm_xp, h->xp, Tm * k, H, 32);
+  } else {
+    err |= cudaMemsetAsync(h->bad, 0, 16, s) != cudaSuccess;
+    err |= launch_repack_w13_bytes(w->w1, w->w3, nullptr, nullptr, static_cast<int>(E), 0, static_cast<int>(I),
+                                   static_cast<int>(H / 2), h->w13q, s) != cudaSuccess;
+    err |= cudaMemcpyAsync(h->w2q, w->w2, E * H * I / 2, cudaMemcpyDeviceToDevice, s) != cudaSuccess;
+    err |= launch_sf_atoms(w->s1, w->s3, static_cast<int>(E), static_cast<int>(I), static_cast<int>(H), h->sfa13,
+                           h->bad, s) != cudaSuccess;
+    err |= launch_sf_atoms(w->s2, nullptr, static_cast<int>(E), static_cast<int>(H), static_cast<int>(I), h->sfa2,
+                           h->bad, s) != cudaSuccess;
+    if (S > 0) {
+      err |= launch_repack_w13(nullptr, nullptr, w->sh_w1, w->sh_w3, 0, static_cast<int>(S), static_cast<int>(I),
+                               static_cast<int>(H), h->w13sh, s) != cudaSuccess;
+      err |= cudaMemcpyAsync(h->w2sh, w->sh_w2, S * H * I * 2, cudaMemcpyDeviceToDevice, s) != cudaSuccess;
+      err |= !make_tmap_bf16(&h->tm_w13sh, h->w13sh, S * 2 * I, H, 256);
+      err |= !make_tmap_bf16(&h->tm_w2sh, h->w2sh, S * H, I, 128);
+    }
+    err |= !make_tmap(&h->tm_w13q, h->w13q, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, E * 2 * I, H, H / 2, 128, 256);
+    err |= !make_tmap(&h->tm_w2q, h->w2q, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, E * H, I, I / 2, 128, 128);
+    err |= !make_tmap(&h->tm_xq, h->xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, Tm * k, H, H, 128, 32);
+    err |= !make_tmap(&h->tm_hq, h->hq, CU_TENSOR_MAP_DATA_TYPE_UINT8, Tm * k, I, I, 128, 32);
+  }
   err |= !make_tmap_bf16(&h->tm_h, h->h, h->R, I, 32);
   err |= !make_tmap_bf16(&h->tm_wg, h->wg, E, H, 128);
+  if (!err && mx) {
+    // NaN scale codes (0xFF) are rejected: check what the atom packer saw.
+    int bad = 0;
+    err |= cudaMemcpyAsync(&bad, h->bad, sizeof(int), cudaMemcpyDeviceToHost, s) != cudaSuccess;
+    err |= cudaStreamSynchronize(s) != cudaSuccess;
+    if (!err && bad) {
+      h->release();
+      delete h;
+      return MOE_ERR_INVALID_ARG;
+    }
+  }
   if (err) {
     cudaGetLastError();
     cudaStreamSynchronize(s);
@@ -304,8 +385,9 @@ moe_status moe_forward(moe_handle* h, const void* x, int32_t T, void* y, int32_t
   const int nslots = T * k;
   const int nchunks = (nslots + kPermChunk - 1) / kPermChunk;
   const bool small = T <= 32;
-  const int bn_gu = small ? 32 : 128;
+  const int bn_gu = small ? 32 : 128;   // BF16 token tiles
   const int bn_dn = small ? 32 : 256;
+  const int bn_mx = small ? 32 : 64;    // MXFP4 token tiles (gate/up and down)
 
   CUtensorMap tm_x;
   if (!make_tmap_bf16(&tm_x, x, static_cast<uint64_t>(T), static_cast<uint64_t>(H), 32)) return MOE_ERR_CUDA;
@@ -317,18 +399,13 @@ moe_status moe_forward(moe_handle* h, const void* x, int32_t T, void* y, int32_t
     h->prof_done(s);
   } else {
     GemmArgs a{};
-    a.tiles = nullptr;
-    a.ntiles = nullptr;
     a.dense_m_tiles = (E + 127) / 128;
     a.dense_rows = T;
     a.num_kb = H / 64;
-    a.a_rows_per_group = 0;
-    a.n_routed = 0;
     a.out = h->z;
     a.out_ld = E;
     a.out_rows = T;
     a.m_limit = E;
-    a.limit = 0.f;
     a.col_bias = h->bias;
     a.status = h->status;
     a.timeout_ns = h->timeout_ns;
@@ -346,7 +423,7 @@ moe_status moe_forward(moe_handle* h, const void* x, int32_t T, void* y, int32_t
   h->prof_mark(kKPermCount, s);
   MOE_TRY_CUDA(launch_perm_count(h->idx, nslots, E, h->chunk_cnt, h->status, s));
   h->prof_done(s);
-  ScanArgs sa;
+  ScanArgs sa{};
   sa.chunk_cnt = h->chunk_cnt;
   sa.nchunks = nchunks;
   sa.E = E;
@@ -359,20 +436,26 @@ moe_status moe_forward(moe_handle* h, const void* x, int32_t T, void* y, int32_t
   sa.tiles_dn = h->tiles_dn;
   sa.ntiles = h->ntiles;
   sa.m_tiles_gu = h->m_tiles_gu;
-  sa.bn_gu = bn_gu;
   sa.m_tiles_dn = h->m_tiles_dn;
-  sa.bn_dn = bn_dn;
+  sa.bn_gu_r = h->mx ? bn_mx : bn_gu;
+  sa.bn_dn_r = h->mx ? bn_mx : bn_dn;
+  sa.bn_gu_s = bn_gu;
+  sa.bn_dn_s = bn_dn;
+  sa.mx = h->mx ? 1 : 0;
+  sa.ntile_base_gu = h->ntile_base_gu;
+  sa.ntile_base_dn = h->ntile_base_dn;
   h->prof_mark(kKPermScan, s);
   MOE_TRY_CUDA(launch_perm_scan(sa, s));
   h->prof_done(s);
   h->prof_mark(kKPermScatter, s);
   MOE_TRY_CUDA(launch_perm_scatter(h->idx, nslots, E, h->chunk_cnt, h->perm, h->inv, s));
   h->prof_done(s);
-  h->prof_mark(kKGather, s);
-  MOE_TRY_CUDA(launch_gather_rows(x, h->perm, nslots, k, H, h->xp, s));
-  h->prof_done(s);
-  // 4. gate/up grouped GEMM with the clamped SwiGLU epilogue
-  {
+
+  if (!h->mx) {
+    h->prof_mark(kKGather, s);
+    MOE_TRY_CUDA(launch_gather_rows(x, h->perm, nslots, k, H, h->xp, s));
+    h->prof_done(s);
+    // 4. gate/up grouped GEMM with the clamped SwiGLU epilogue (routed and shared groups)
     GemmArgs a{};
     a.tiles = h->tiles_gu;
     a.ntiles = h->ntiles;
@@ -389,25 +472,111 @@ moe_status moe_forward(moe_handle* h, const void* x, int32_t T, void* y, int32_t
     h->prof_mark(kKGateUp, s);
     MOE_TRY_CUDA(launch_gemm_gateup(h->tm_w13, h->tm_xp, tm_x, a, bn_gu, h->num_sms, s));
     h->prof_done(s);
-  }
-  // 5. down grouped GEMM
-  {
-    GemmArgs a{};
-    a.tiles = h->tiles_dn;
-    a.ntiles = h->ntiles + 1;
-    a.num_kb = I / 64;
-    a.a_rows_per_group = H;
-    a.n_routed = E;
-    a.out = h->o;
-    a.out_ld = H;
-    a.out_rows = static_cast<int>(h->R);
-    a.m_limit = H;
-    a.limit = 0.f;
-    a.status = h->status;
-    a.timeout_ns = h->timeout_ns;
+    // 5. down grouped GEMM
+    GemmArgs d{};
+    d.tiles = h->tiles_dn;
+    d.ntiles = h->ntiles + 1;
+    d.num_kb = I / 64;
+    d.a_rows_per_group = H;
+    d.n_routed = E;
+    d.out = h->o;
+    d.out_ld = H;
+    d.out_rows = static_cast<int>(h->R);
+    d.m_limit = H;
+    d.status = h->status;
+    d.timeout_ns = h->timeout_ns;
     h->prof_mark(kKDown, s);
-    MOE_TRY_CUDA(launch_gemm_down(h->tm_w2, h->tm_h, a, bn_dn, h->num_sms, s));
+    MOE_TRY_CUDA(launch_gemm_down(h->tm_w2, h->tm_h, d, bn_dn, h->num_sms, s));
     h->prof_done(s);
+  } else {
+    // MXFP8 token rows of the routed slots
+    h->prof_mark(kKQuantX, s);
+    MOE_TRY_CUDA(launch_quant_gather_mx(x, h->perm, h->idx, h->off, h->ntile_base_gu, nslots, k, H, bn_mx, h->xq,
+                                        h->sfb_gu, s));
+    h->prof_done(s);
+    // 4a. routed gate/up on block-scaled MMAs (tiles after the shared ones)
+    MxGemmArgs g{};
+    g.tiles = h->tiles_gu;
+    g.ntiles = h->ntiles;
+    g.tile_begin = h->ntiles + 2;
+    g.num_kb = H / 128;
+    g.a_rows_per_group = 2 * I;
+    g.m_tiles = I / 128;
+    g.sfa = h->sfa13;
+    g.sfb = h->sfb_gu;
+    g.out = h->hq;
+    g.out_ld = I;
+    g.out_rows = T * k;
+    g.m_limit = I;
+    g.limit = c.swiglu_limit;
+    g.sf_out = h->sfb_dn;
+    g.sf_out_kb4 = I / 128;
+    g.bn_dn = bn_mx;
+    g.group_off = h->off;
+    g.dn_ntile_base = h->ntile_base_dn;
+    g.status = h->status;
+    g.timeout_ns = h->timeout_ns;
+    h->prof_mark(kKGateUpMx, s);
+    MOE_TRY_CUDA(launch_gemm_mx_gateup(h->tm_w13q, h->tm_xq, g, bn_mx, h->num_sms, s));
+    h->prof_done(s);
+    // 4b. shared experts' gate/up in BF16 (the first tiles of the list)
+    if (S > 0) {
+      GemmArgs a{};
+      a.tiles = h->tiles_gu;
+      a.ntiles = h->ntiles + 2;
+      a.group_base = E;
+      a.num_kb = H / 64;
+      a.a_rows_per_group = 2 * I;
+      a.n_routed = E;
+      a.out = h->h;
+      a.out_ld = I;
+      a.out_rows = static_cast<int>(h->R);
+      a.m_limit = I;
+      a.limit = c.swiglu_limit;
+      a.status = h->status;
+      a.timeout_ns = h->timeout_ns;
+      h->prof_mark(kKGateUp, s);
+      MOE_TRY_CUDA(launch_gemm_gateup(h->tm_w13sh, tm_x, tm_x, a, bn_gu, h->num_sms, s));
+      h->prof_done(s);
+    }
+    // 5a. routed down on block-scaled MMAs
+    MxGemmArgs d{};
+    d.tiles = h->tiles_dn;
+    d.ntiles = h->ntiles + 1;
+    d.tile_begin = h->ntiles + 3;
+    d.num_kb = I / 128;
+    d.a_rows_per_group = H;
+    d.m_tiles = H / 128;
+    d.sfa = h->sfa2;
+    d.sfb = h->sfb_dn;
+    d.out = h->o;
+    d.out_ld = H;
+    d.out_rows = static_cast<int>(h->R);
+    d.m_limit = H;
+    d.status = h->status;
+    d.timeout_ns = h->timeout_ns;
+    h->prof_mark(kKDownMx, s);
+    MOE_TRY_CUDA(launch_gemm_mx_down(h->tm_w2q, h->tm_hq, d, bn_mx, h->num_sms, s));
+    h->prof_done(s);
+    // 5b. shared experts' down in BF16
+    if (S > 0) {
+      GemmArgs a{};
+      a.tiles = h->tiles_dn;
+      a.ntiles = h->ntiles + 3;
+      a.group_base = E;
+      a.num_kb = I / 64;
+      a.a_rows_per_group = H;
+      a.n_routed = E;
+      a.out = h->o;
+      a.out_ld = H;
+      a.out_rows = static_cast<int>(h->R);
+      a.m_limit = H;
+      a.status = h->status;
+      a.timeout_ns = h->timeout_ns;
+      h->prof_mark(kKDown, s);
+      MOE_TRY_CUDA(launch_gemm_down(h->tm_w2sh, h->tm_h, a, bn_dn, h->num_sms, s));
+      h->prof_done(s);
+    }
   }
   // 6. weighted combine with the shared experts
   h->prof_mark(kKCombine, s);
@@ -487,6 +656,16 @@ moe_status moe_inspect(moe_handle* h, int32_t what, void* dst, size_t bytes, moe
     case MOE_BUF_PERM: src = h->perm; cap = Tm * k * 4; break;
     case MOE_BUF_INV: src = h->inv; cap = Tm * k * 4; break;
     case MOE_BUF_H: src = h->h; cap = h->R * I * 2; break;
+    case MOE_BUF_XQ:
+      if (!h->mx) return MOE_ERR_INVALID_ARG;
+      src = h->xq;
+      cap = Tm * k * h->cfg.hidden;
+      break;
+    case MOE_BUF_XQ_SCALES:
+      if (!h->mx) return MOE_ERR_INVALID_ARG;
+      src = h->sfb_gu;
+      cap = h->max_ntiles_r * (h->cfg.hidden / 128) * 512;
+      break;
     default: return MOE_ERR_INVALID_ARG;
   }
   if (bytes > cap) return MOE_ERR_INVALID_ARG;
@@ -518,7 +697,7 @@ moe_status moe_get_info(moe_handle* h, moe_info* out) {
 
 moe_status moe_profile_begin(moe_handle* h, int32_t max_calls) {
   if (h == nullptr || max_calls <= 0 || max_calls > 100000) return MOE_ERR_INVALID_ARG;
-  const size_t need = static_cast<size_t>(max_calls) * 2 * 12;
+  const size_t need = static_cast<size_t>(max_calls) * 2 * 16;
   while (h->ev.size() < need) {
     cudaEvent_t e;
     if (cudaEventCreate(&e) != cudaSuccess) {

@@ -5,6 +5,7 @@
 
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp8.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -165,6 +166,69 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr) {
 // N >> 3 in bits 17-22, M >> 4 in bits 24-28.
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(uint32_t M, uint32_t N) {
   return (1u << 4) | (1u << 7) | (1u << 10) | ((N >> 3) << 17) | ((M >> 4) << 24);
+}
+
+// ---------------------------------------------------------------- MX (block-scaled) helpers
+// 1-D bulk copy global -> shared, completing `bytes` on `bar` (16-byte aligned, size % 16 == 0).
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar,
+                                          uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;" ::"r"(
+          smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar)), "l"(policy)
+      : "memory");
+}
+
+// Copy 32 rows x 128 bits from shared memory into TMEM lanes 0-31 and replicate
+// them to the other three lane quarters (scale-factor layout of the block-scaled MMA).
+__device__ __forceinline__ void tmem_cp_32x128b_x4(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+
+// Shared-memory descriptor of a contiguous block of 16-byte rows without swizzle
+// (8-row core matrices 128 bytes apart): the source of tcgen05.cp.
+__device__ __forceinline__ uint64_t sdesc_plain(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4);
+  d |= static_cast<uint64_t>(16u >> 4) << 16;
+  d |= static_cast<uint64_t>(128u >> 4) << 32;
+  d |= static_cast<uint64_t>(1) << 46;
+  return d;  // layout type 0 = no swizzle
+}
+
+// D[tmem] (+)= (A * 2^sfa) (B * 2^sfb)^T, kind::mxf8f6f4 with one E8M0 scale per 32 K.
+__device__ __forceinline__ void umma_mx(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                        uint32_t tsfa, uint32_t tsfb, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}\n" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(tsfa), "r"(tsfb)
+      : "memory");
+}
+
+// Block-scaled instruction descriptor: A E2M1 (format 5, bits 7-9), B E4M3
+// (format 0, bits 10-12), both K-major, N >> 3 in bits 17-22, scale format E8M0
+// (bit 23), M >> 4 in bits 24-28, scale-factor byte ids in bits 4-5 (B) and
+// 29-30 (A), K = 32 (bit 31 = 0).
+__host__ __device__ constexpr uint32_t idesc_mx_e2m1_e4m3(uint32_t M, uint32_t N, uint32_t sfa_id, uint32_t sfb_id) {
+  return (sfb_id << 4) | (5u << 7) | (0u << 10) | ((N >> 3) << 17) | (1u << 23) | ((M >> 4) << 24) |
+         (sfa_id << 29);
+}
+
+// E8M0 scale code and the exact reciprocal scale for an MX block with the given
+// amax (OCP MX v1.0: shared exponent floor(log2 amax) - emax, clamped; code 0 for
+// an all-zero block).
+__device__ __forceinline__ void mx_scale(float amax, int emax, int& code, float& inv_scale) {
+  code = 0;
+  inv_scale = 0.f;
+  if (amax > 0.f) {
+    int ex;
+    frexpf(amax, &ex);
+    int sh = max(-127, min(127, (ex - 1) - emax));
+    code = sh + 127;
+    inv_scale = ldexpf(1.0f, -sh);
+  }
 }
 
 // ---------------------------------------------------------------- math

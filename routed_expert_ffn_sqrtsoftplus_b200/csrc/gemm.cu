@@ -84,6 +84,10 @@ __device__ __forceinline__ int tile_count(const GemmArgs& a) {
   return a.dense_m_tiles * ((a.dense_rows + BN - 1) / BN);
 }
 
+__device__ __forceinline__ int tile_first(const GemmArgs& a) {
+  return (a.tiles != nullptr && a.tile_begin != nullptr) ? *a.tile_begin : 0;
+}
+
 // Wait that also gives up as soon as another role of this CTA has aborted.
 __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, const GemmArgs& a,
                                               volatile int* abort_flag) {
@@ -151,6 +155,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem_base = *tmem_base_smem;
 
   const int ntiles = tile_count<BN>(args);
+  const int tfirst = tile_first(args) + static_cast<int>(blockIdx.x);
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
@@ -158,10 +163,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       int stage = 0;
       uint32_t phase = 0;
       long issued = 0;
-      for (int t = blockIdx.x; t < ntiles && !*abort_flag; t += gridDim.x) {
+      for (int t = tfirst; t < ntiles && !*abort_flag; t += gridDim.x) {
         const Tile tl = load_tile<BN>(args, t);
         const CUtensorMap* mb = (kGateUp && tl.group >= args.n_routed) ? &tmBsh : &tmB;
-        const int a_row = tl.group * args.a_rows_per_group + tl.m_tile * C::kARows;
+        const int a_row = (tl.group - args.group_base) * args.a_rows_per_group + tl.m_tile * C::kARows;
         const int nb = (tl.nrows + kBBoxRows - 1) / kBBoxRows;
         const uint32_t bytes = C::kABytes + nb * kBBoxBytes;
         bool ok = true;
@@ -201,7 +206,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t phase = 0;
       int acc = 0;
       uint32_t acc_phase = 0;
-      for (int t = blockIdx.x; t < ntiles && !*abort_flag; t += gridDim.x) {
+      for (int t = tfirst; t < ntiles && !*abort_flag; t += gridDim.x) {
         const Tile tl = load_tile<BN>(args, t);
         const uint32_t n_mma = max(16, (tl.nrows + 15) & ~15);
         const uint32_t idesc = idesc_bf16_f32(128, n_mma);
@@ -248,7 +253,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int q = warp & 3;  // TMEM lane quarter this warp may access
     int acc = 0;
     uint32_t acc_phase = 0;
-    for (int t = blockIdx.x; t < ntiles; t += gridDim.x) {
+    for (int t = tfirst; t < ntiles; t += gridDim.x) {
       const Tile tl = load_tile<BN>(args, t);
       const int n_mma = max(16, (tl.nrows + 15) & ~15);
       bool ok = true;

@@ -13,7 +13,9 @@ using TileEntry = int4;
 
 struct GemmArgs {
   const int4* tiles;            // grouped mode: tile list; nullptr = dense mode
-  const int* ntiles;            // grouped mode: device tile count
+  const int* ntiles;            // grouped mode: device index one past the last tile to run
+  const int* tile_begin;        // grouped mode: device index of the first tile to run (nullptr = 0)
+  int group_base;               // A rows of group g start at (g - group_base) * a_rows_per_group
   int dense_m_tiles;            // dense mode: 128-row tiles of A
   int dense_rows;               // dense mode: rows of B (tokens)
   int num_kb;                   // K / 64
@@ -42,6 +44,8 @@ enum KernelKind {
   kKDown,
   kKCombine,
   kKQuantX,
+  kKGateUpMx,
+  kKDownMx,
   kKNumKinds
 };
 
@@ -63,8 +67,13 @@ struct ScanArgs {
   int32_t* off;
   int4* tiles_gu;
   int4* tiles_dn;
-  int* ntiles;
-  int m_tiles_gu, bn_gu, m_tiles_dn, bn_dn;
+  int* ntiles;                  // [gu_end, dn_end, gu_shared_end, dn_shared_end]
+  int m_tiles_gu, m_tiles_dn;
+  int bn_gu_r, bn_dn_r;         // token tile of routed groups (gate/up, down)
+  int bn_gu_s, bn_dn_s;         // token tile of shared groups
+  int mx;                       // routed tiles carry their token-tile id in .y
+  int32_t* ntile_base_gu;       // [E + 1] first token tile of each routed group (gate/up)
+  int32_t* ntile_base_dn;       // [E + 1] same for the down GEMM
 };
 cudaError_t launch_perm_scan(const ScanArgs& a, cudaStream_t s);
 cudaError_t launch_perm_scatter(const int32_t* idx, int nslots, int E, const int32_t* chunk_base, int32_t* perm,
@@ -79,6 +88,48 @@ cudaError_t launch_gemm_gateup(const CUtensorMap& tmA, const CUtensorMap& tmB, c
 cudaError_t launch_gemm_down(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmArgs& a, int bn, int grid,
                              cudaStream_t s);
 cudaError_t gemm_set_attributes();
+
+// ---- MX (MXFP4 routed experts)
+struct MxGemmArgs {
+  const int4* tiles;            // {group | m_tile << 16, token tile id, first row, rows}
+  const int* ntiles;            // device index one past the last tile
+  const int* tile_begin;        // device index of the first tile (nullptr = 0)
+  int num_kb;                   // K / 128
+  int a_rows_per_group;
+  int m_tiles;                  // weight tiles per group
+  const uint8_t* sfa;           // weight scale atoms [groups][m_tiles][num_kb][atoms of this GEMM]
+  const uint8_t* sfb;           // activation scale atoms [token tiles][num_kb][512]
+  void* out;                    // gate/up: E4M3 h rows; down: fp32 rows
+  int out_ld;
+  int out_rows;
+  int m_limit;
+  float limit;
+  uint8_t* sf_out;              // gate/up: scale atoms of h for the down GEMM
+  int sf_out_kb4;               // I / 128
+  int bn_dn;                    // token tile of the down GEMM
+  const int32_t* group_off;     // first row of each group
+  const int32_t* dn_ntile_base; // first down token tile of each group
+  int* status;
+  unsigned long long timeout_ns;
+};
+cudaError_t gemm_mx_set_attributes();
+cudaError_t launch_gemm_mx_gateup(const CUtensorMap& tmA, const CUtensorMap& tmB, const MxGemmArgs& a, int bn,
+                                  int grid, cudaStream_t s);
+cudaError_t launch_gemm_mx_down(const CUtensorMap& tmA, const CUtensorMap& tmB, const MxGemmArgs& a, int bn,
+                                int grid, cudaStream_t s);
+// x rows of the routed slots -> MXFP8: xq[row] = E4M3 codes of x[perm[row] / k], scale
+// atoms by gate/up token tile.
+cudaError_t launch_quant_gather_mx(const void* x, const int32_t* perm, const int32_t* idx, const int32_t* off,
+                                   const int32_t* ntile_base_gu, int nrows, int k, int H, int bn_gu, uint8_t* xq,
+                                   uint8_t* sfb, cudaStream_t s);
+// Weight scales [groups, rows, K/32] -> atoms [groups][rows/128][K/128][parts * 512]; for
+// gate/up the two parts are W1 and W3 of the same 128 rows. Codes 0xFF raise *bad.
+cudaError_t launch_sf_atoms(const uint8_t* s_a, const uint8_t* s_b, int groups, int rows, int K, uint8_t* dst,
+                            int* bad, cudaStream_t s);
+// Row permutation of the W1/W3 rows into 256-row gate/up tiles for any row width
+// (bytes per row a multiple of 16); groups >= E come from the shared pointers.
+cudaError_t launch_repack_w13_bytes(const void* w1, const void* w3, const void* sh1, const void* sh3, int E, int S,
+                                    int I, int row_bytes, void* w13, cudaStream_t s);
 
 // ---- combine
 cudaError_t launch_combine(const float* O, const int32_t* inv, const float* w, int T, int H, int k, int S,

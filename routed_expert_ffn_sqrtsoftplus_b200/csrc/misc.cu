@@ -63,6 +63,35 @@ __global__ void __launch_bounds__(256)
   for (int c = threadIdx.x % 32; c < hv; c += 32) d[c] = __ldg(src + c);
 }
 
+// Scale atoms of the block-scaled MMA: for each group, 128-row weight tile and
+// 128-wide K block, 512 bytes holding row m, block kb at (m % 32) * 16 +
+// (m / 32) * 4 + kb (rows interleaved by 32 so that a 32-lane x 16-byte copy
+// to TMEM puts every row's four scales in one 32-bit word). With two sources
+// (W1, W3) the two atoms of the same rows are adjacent.
+__global__ void __launch_bounds__(256)
+    sf_atoms_kernel(const uint8_t* __restrict__ sa, const uint8_t* __restrict__ sb, int groups, int rows, int K,
+                    uint8_t* __restrict__ dst, int* bad) {
+  const int parts = sb ? 2 : 1;
+  const int mtiles = rows / 128, kb4s = K / 128;
+  const size_t total = static_cast<size_t>(groups) * mtiles * kb4s * parts * 512;
+  const size_t i = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i >= total) return;
+  const int within = static_cast<int>(i % 512);
+  size_t rest = i / 512;
+  const int p = static_cast<int>(rest % parts);
+  rest /= parts;
+  const int kb4 = static_cast<int>(rest % kb4s);
+  rest /= kb4s;
+  const int mt = static_cast<int>(rest % mtiles);
+  const size_t g = rest / mtiles;
+  const int rem = within % 16;
+  const int m = mt * 128 + (rem / 4) * 32 + within / 16;
+  const int kblk = kb4 * 4 + rem % 4;
+  const uint8_t v = (p ? sb : sa)[(g * rows + m) * (K / 32) + kblk];
+  if (v == 0xFF) atomicOr(bad, 1);
+  dst[i] = v;
+}
+
 // One thread per 32-element block: OCP MX rule with E2M1 elements.
 __global__ void __launch_bounds__(256)
     quantize_mxfp4_kernel(const uint4* __restrict__ src, int64_t nblocks, uint4* __restrict__ packed,
@@ -134,12 +163,26 @@ cudaError_t launch_combine(const float* O, const int32_t* inv, const float* w, i
   return cudaGetLastError();
 }
 
-cudaError_t launch_repack_w13(const void* w1, const void* w3, const void* sh1, const void* sh3, int E, int S, int I,
-                              int H, void* w13, cudaStream_t s) {
+cudaError_t launch_repack_w13_bytes(const void* w1, const void* w3, const void* sh1, const void* sh3, int E, int S,
+                                    int I, int row_bytes, void* w13, cudaStream_t s) {
   const size_t rows = static_cast<size_t>(E + S) * 2 * I;
+  if (rows == 0) return cudaSuccess;
   repack_w13_kernel<<<static_cast<unsigned>((rows + 7) / 8), 256, 0, s>>>(
       static_cast<const uint4*>(w1), static_cast<const uint4*>(w3), static_cast<const uint4*>(sh1),
-      static_cast<const uint4*>(sh3), E, S, I, H / 8, static_cast<uint4*>(w13));
+      static_cast<const uint4*>(sh3), E, S, I, row_bytes / 16, static_cast<uint4*>(w13));
+  return cudaGetLastError();
+}
+
+cudaError_t launch_repack_w13(const void* w1, const void* w3, const void* sh1, const void* sh3, int E, int S, int I,
+                              int H, void* w13, cudaStream_t s) {
+  return launch_repack_w13_bytes(w1, w3, sh1, sh3, E, S, I, H * 2, w13, s);
+}
+
+cudaError_t launch_sf_atoms(const uint8_t* s_a, const uint8_t* s_b, int groups, int rows, int K, uint8_t* dst,
+                            int* bad, cudaStream_t s) {
+  const size_t total = static_cast<size_t>(groups) * (rows / 128) * (K / 128) * (s_b ? 2 : 1) * 512;
+  if (total == 0) return cudaSuccess;
+  sf_atoms_kernel<<<static_cast<unsigned>((total + 255) / 256), 256, 0, s>>>(s_a, s_b, groups, rows, K, dst, bad);
   return cudaGetLastError();
 }
 

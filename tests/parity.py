@@ -30,10 +30,16 @@ def f64(t: torch.Tensor) -> np.ndarray:
 class LayerExperts(om.ExpertSource):
     """Oracle expert source reading one expert at a time from the generator's tensors."""
 
-    def __init__(self, layer: dict, mx_q: dict | None = None):
+    def __init__(self, layer: dict, mx_q: dict | None = None, mx_from_bf16: bool = False):
         S = layer["sh_w1"].shape[0]
         E = layer["w1"].shape[0]
-        if mx_q is None:
+        if mx_from_bf16:
+            # quantise each routed expert with the oracle's own MXFP4 codec
+            from oracle import mx as omx
+            rt = lambda w: omx.mx_roundtrip(f64(w), "e2m1")
+            routed = lambda e: (rt(layer["w1"][e]), rt(layer["w3"][e]), rt(layer["w2"][e]))
+            is_mx = True
+        elif mx_q is None:
             routed = lambda e: (f64(layer["w1"][e]), f64(layer["w3"][e]), f64(layer["w2"][e]))
             is_mx = False
         else:
@@ -52,13 +58,16 @@ def oracle_route(layer, k, rs, tokens=None):
     return om.route(f64(x), f64(layer["wg"]), k, rs, bias=bias)
 
 
-def compare_layer(layer, tokens, y_gpu, idx_gpu, w_gpu, k, rs, limit, mx_q=None):
-    """Compare GPU rows (for `tokens`) with the oracle; returns a report dict, asserts the bars."""
+def compare_layer(layer, tokens, y_gpu, idx_gpu, w_gpu, k, rs, limit, mx_q=None, mx_from_bf16=False):
+    """Compare GPU rows (for `tokens`) with the oracle; returns a report dict, asserts the bars.
+
+    With mx_q (packed MXFP4 tensors) or mx_from_bf16 the routed experts are MXFP4 and
+    the oracle mirrors the MXFP8 activation quantisation."""
     tokens = np.asarray(tokens)
     x = f64(layer["x"][torch.as_tensor(tokens, device=layer["x"].device)])
     wg = f64(layer["wg"])
     bias = None if layer.get("bias") is None else f64(layer["bias"])
-    ex = LayerExperts(layer, mx_q)
+    ex = LayerExperts(layer, mx_q, mx_from_bf16)
     r = om.route(x, wg, k, rs, bias=bias)
     idx_g = np.asarray(idx_gpu, dtype=np.int64)
     sure = r.gap > GAP_EXACT
