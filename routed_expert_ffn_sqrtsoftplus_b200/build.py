@@ -6,7 +6,8 @@ Each csrc/*.cu is compiled by nvcc for sm_100a only (``-gencode
 arch=compute_100a,code=sm_100a``) and linked, with the CUDA runtime linked
 statically, into routed_expert_ffn_sqrtsoftplus_b200/_lib/libmoe_b200.so. The
 library exposes exactly the C ABI of include/moe.h. Rebuilds only when a
-source or header is newer than the library (or with --force).
+source or header is newer than the library (or with --force). Extra nvcc flags
+(for example -D overrides of the GEMM ring depths) can be given in MOE_NVCC_EXTRA.
 """
 from __future__ import annotations
 
@@ -55,7 +56,8 @@ def up_to_date() -> bool:
 
 def _compile(src: str, log_dir: str) -> str:
     obj = os.path.join(BUILD, os.path.basename(src)[:-3] + ".o")
-    cmd = [nvcc(), *ARCH, *NVCC_FLAGS, "-I", INCLUDE, "-c", src, "-o", obj]
+    extra = os.environ.get("MOE_NVCC_EXTRA", "").split()
+    cmd = [nvcc(), *ARCH, *NVCC_FLAGS, *extra, "-I", INCLUDE, "-c", src, "-o", obj]
     r = subprocess.run(cmd, capture_output=True, text=True)
     with open(os.path.join(log_dir, os.path.basename(src) + ".log"), "w") as f:
         f.write(" ".join(cmd) + "\n" + r.stdout + r.stderr)

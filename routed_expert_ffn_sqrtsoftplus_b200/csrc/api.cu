@@ -3,6 +3,7 @@
 // invocation. Every step of the layer runs in this library's kernels.
 #include <cmath>
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <new>
 #include <vector>
@@ -21,6 +22,8 @@ namespace {
 constexpr float kRefineDelta = 2e-3f;
 // Token counts above this use the tensor-core router GEMM for the logits.
 constexpr int kTcRouterMinTokens = 256;
+// Token counts up to this use the sliced CUDA-core router and the per-token top-k.
+constexpr int kSmallRouterMaxTokens = 32;
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
@@ -90,6 +93,7 @@ struct moe_handle {
   void* w2 = nullptr;
 
   float* z = nullptr;
+  float* zpart = nullptr;       // logit slices for T <= kSmallRouterMaxTokens
   int32_t* idx = nullptr;
   float* wts = nullptr;
   int32_t* chunk_cnt = nullptr;
@@ -108,6 +112,8 @@ struct moe_handle {
   void* y_stage = nullptr;
 
   CUtensorMap tm_w13, tm_w2, tm_xp, tm_h, tm_wg;
+  CUtensorMap tm_w2w;           // W2 with 256-row boxes (wide down tiles)
+  bool wide_ok = false;         // H % 256 == 0
 
   // MXFP4 routed experts (expert_dtype == MOE_DT_MXFP4)
   bool mx = false;
@@ -126,6 +132,11 @@ struct moe_handle {
   int* bad = nullptr;
   int64_t max_ntiles_r = 0;
   CUtensorMap tm_w13q, tm_w2q, tm_xq, tm_hq, tm_w13sh, tm_w2sh;
+  // shared experts alone (MXFP4 layers, few tokens): split-K partial sums
+  float* sh_parts_gu = nullptr;  // [S][ks_gu][T][2I]
+  float* sh_parts_dn = nullptr;  // [S][ks_dn][T][H]
+  int ks_gu = 1, ks_dn = 1;
+
   uint64_t timeout_ns = 2000000000ull;
   std::vector<void*> allocs;
   uint64_t weight_bytes = 0, workspace_bytes = 0;
@@ -171,6 +182,13 @@ struct moe_handle {
 };
 
 namespace {
+
+// Largest divisor of n that is <= cap.
+int divisor_at_most(int n, int cap) {
+  for (int d = cap; d > 1; --d)
+    if (n % d == 0) return d;
+  return 1;
+}
 
 moe_status validate_config(const moe_config* c) {
   if (!(c->route_scale > 0.f) || !std::isfinite(c->route_scale)) return MOE_ERR_INVALID_ARG;
@@ -246,7 +264,8 @@ moe_status moe_create(const moe_config* cfg, const moe_weights* w, moe_stream_t 
   h->mx = mx;
   if (cudaGetDevice(&h->device) != cudaSuccess ||
       cudaDeviceGetAttribute(&h->num_sms, cudaDevAttrMultiProcessorCount, h->device) != cudaSuccess ||
-      gemm_set_attributes() != cudaSuccess || gemm_mx_set_attributes() != cudaSuccess) {
+      gemm_set_attributes() != cudaSuccess || gemm_mx_set_attributes() != cudaSuccess ||
+      router_set_attributes() != cudaSuccess) {
     cudaGetLastError();
     delete h;
     return MOE_ERR_CUDA;
@@ -287,8 +306,16 @@ moe_status moe_create(const moe_config* cfg, const moe_weights* w, moe_stream_t 
     ok = ok && h->alloc(&h->ntile_base_gu, (E + 1) * 4, ws);
     ok = ok && h->alloc(&h->ntile_base_dn, (E + 1) * 4, ws);
     ok = ok && h->alloc(&h->bad, 16, ws);
+    if (S > 0) {
+      const int64_t tsmall = Tm < kSmallRouterMaxTokens ? Tm : kSmallRouterMaxTokens;
+      h->ks_gu = divisor_at_most(static_cast<int>(H / 64), 8);
+      h->ks_dn = divisor_at_most(static_cast<int>(I / 64), 4);
+      ok = ok && h->alloc(&h->sh_parts_gu, S * h->ks_gu * tsmall * 2 * I * 4, ws);
+      ok = ok && h->alloc(&h->sh_parts_dn, S * h->ks_dn * tsmall * H * 4, ws);
+    }
   }
   ok = ok && h->alloc(&h->z, Tm * E * 4, ws);
+  ok = ok && h->alloc(&h->zpart, (H / 128) * (Tm < kSmallRouterMaxTokens ? Tm : kSmallRouterMaxTokens) * E * 4, ws);
   ok = ok && h->alloc(&h->idx, Tm * k * 4, ws);
   ok = ok && h->alloc(&h->wts, Tm * k * 4, ws);
   ok = ok && h->alloc(&h->chunk_cnt, static_cast<size_t>(h->nchunks_max) * E * 4, ws);
@@ -324,6 +351,8 @@ moe_status moe_create(const moe_config* cfg, const moe_weights* w, moe_stream_t 
                              cudaMemcpyDeviceToDevice, s) != cudaSuccess;
     err |= !make_tmap_bf16(&h->tm_w13, h->w13, (E + S) * 2 * I, H, 256);
     err |= !make_tmap_bf16(&h->tm_w2, h->w2, (E + S) * H, I, 128);
+    h->wide_ok = H % 256 == 0;
+    if (h->wide_ok) err |= !make_tmap_bf16(&h->tm_w2w, h->w2, (E + S) * H, I, 256);
     err |= !make_tmap_bf16(&h->tm_xp, h->xp, Tm * k, H, 32);
   } else {
     err |= cudaMemsetAsync(h->bad, 0, 16, s) != cudaSuccess;
@@ -384,16 +413,29 @@ moe_status moe_forward(moe_handle* h, const void* x, int32_t T, void* y, int32_t
   const int H = c.hidden, I = c.inter, E = c.n_routed, S = c.n_shared, k = c.top_k;
   const int nslots = T * k;
   const int nchunks = (nslots + kPermChunk - 1) / kPermChunk;
+  // Token tiles. Few tokens: 32-row tiles and deep smem rings (weight streaming).
+  // Many tokens per expert: 256-row tiles so each weight tile is read once and
+  // every staged byte feeds twice the MMA work (one TMEM accumulator).
   const bool small = T <= 32;
-  const int bn_gu = small ? 32 : 128;   // BF16 token tiles
+  const bool large = !small && static_cast<int64_t>(T) * k >= 24LL * E;
+  const int bn_gu = small ? 32 : (large ? 256 : 128);   // BF16 token tiles
   const int bn_dn = small ? 32 : 256;
-  const int bn_mx = small ? 32 : 64;    // MXFP4 token tiles (gate/up and down)
+  const bool wide = large && h->wide_ok && !h->mx;      // 256-row W2 tiles
+  const int bn_mx = small ? 32 : 64;                    // MXFP4 token tiles (gate/up and down)
 
   CUtensorMap tm_x;
   if (!make_tmap_bf16(&tm_x, x, static_cast<uint64_t>(T), static_cast<uint64_t>(H), 32)) return MOE_ERR_CUDA;
 
-  // 1. router logits (+ bias)
-  if (T < kTcRouterMinTokens) {
+  // 1-2. router logits (+ bias), scores, top-k, weights
+  if (T <= kSmallRouterMaxTokens) {
+    h->prof_mark(kKRouterLogits, s);
+    MOE_TRY_CUDA(launch_router_small(x, h->wg, h->zpart, T, H, E, s));
+    h->prof_done(s);
+    h->prof_mark(kKTopk, s);
+    MOE_TRY_CUDA(launch_topk_small(h->zpart, H / router_small_slice(H), x, h->wg, h->bias, T, H, E, k, c.route_scale,
+                                   kRefineDelta, h->idx, h->wts, h->z, h->status, s, h->bias));
+    h->prof_done(s);
+  } else if (T < kTcRouterMinTokens) {
     h->prof_mark(kKRouterLogits, s);
     MOE_TRY_CUDA(launch_router_logits(x, h->wg, h->bias, h->z, T, H, E, s));
     h->prof_done(s);
@@ -414,15 +456,20 @@ moe_status moe_forward(moe_handle* h, const void* x, int32_t T, void* y, int32_t
     MOE_TRY_CUDA(launch_gemm_down(h->tm_wg, tm_x, a, 256, nt < h->num_sms ? nt : h->num_sms, s));
     h->prof_done(s);
   }
-  // 2. scores, top-k with exact refinement, weights
-  h->prof_mark(kKTopk, s);
-  MOE_TRY_CUDA(launch_topk_refine(h->z, x, h->wg, h->bias, T, H, E, k, c.route_scale, kRefineDelta, h->idx, h->wts,
-                                  h->status, s));
-  h->prof_done(s);
+  if (T > kSmallRouterMaxTokens) {
+    // scores, top-k with exact refinement of the near-tie candidates, weights (one
+    // warp per token: with thousands of tokens the warps keep every SM busy)
+    h->prof_mark(kKTopk, s);
+    MOE_TRY_CUDA(launch_topk_refine(h->z, x, h->wg, h->bias, T, H, E, k, c.route_scale, kRefineDelta, h->idx,
+                                    h->wts, h->status, s));
+    h->prof_done(s);
+  }
   // 3. permutation and tile lists
-  h->prof_mark(kKPermCount, s);
-  MOE_TRY_CUDA(launch_perm_count(h->idx, nslots, E, h->chunk_cnt, h->status, s));
-  h->prof_done(s);
+  if (nchunks > 1) {
+    h->prof_mark(kKPermCount, s);
+    MOE_TRY_CUDA(launch_perm_count(h->idx, nslots, E, h->chunk_cnt, h->status, s));
+    h->prof_done(s);
+  }
   ScanArgs sa{};
   sa.chunk_cnt = h->chunk_cnt;
   sa.nchunks = nchunks;
@@ -436,7 +483,7 @@ moe_status moe_forward(moe_handle* h, const void* x, int32_t T, void* y, int32_t
   sa.tiles_dn = h->tiles_dn;
   sa.ntiles = h->ntiles;
   sa.m_tiles_gu = h->m_tiles_gu;
-  sa.m_tiles_dn = h->m_tiles_dn;
+  sa.m_tiles_dn = wide ? H / 256 : h->m_tiles_dn;
   sa.bn_gu_r = h->mx ? bn_mx : bn_gu;
   sa.bn_dn_r = h->mx ? bn_mx : bn_dn;
   sa.bn_gu_s = bn_gu;
@@ -444,12 +491,18 @@ moe_status moe_forward(moe_handle* h, const void* x, int32_t T, void* y, int32_t
   sa.mx = h->mx ? 1 : 0;
   sa.ntile_base_gu = h->ntile_base_gu;
   sa.ntile_base_dn = h->ntile_base_dn;
-  h->prof_mark(kKPermScan, s);
-  MOE_TRY_CUDA(launch_perm_scan(sa, s));
-  h->prof_done(s);
-  h->prof_mark(kKPermScatter, s);
-  MOE_TRY_CUDA(launch_perm_scatter(h->idx, nslots, E, h->chunk_cnt, h->perm, h->inv, s));
-  h->prof_done(s);
+  if (nchunks == 1) {
+    h->prof_mark(kKPermScan, s);
+    MOE_TRY_CUDA(launch_perm_fused(sa, h->idx, nslots, h->perm, h->inv, h->status, s));
+    h->prof_done(s);
+  } else {
+    h->prof_mark(kKPermScan, s);
+    MOE_TRY_CUDA(launch_perm_scan(sa, s));
+    h->prof_done(s);
+    h->prof_mark(kKPermScatter, s);
+    MOE_TRY_CUDA(launch_perm_scatter(h->idx, nslots, E, h->chunk_cnt, h->perm, h->inv, s));
+    h->prof_done(s);
+  }
 
   if (!h->mx) {
     h->prof_mark(kKGather, s);
@@ -486,7 +539,7 @@ moe_status moe_forward(moe_handle* h, const void* x, int32_t T, void* y, int32_t
     d.status = h->status;
     d.timeout_ns = h->timeout_ns;
     h->prof_mark(kKDown, s);
-    MOE_TRY_CUDA(launch_gemm_down(h->tm_w2, h->tm_h, d, bn_dn, h->num_sms, s));
+    MOE_TRY_CUDA(launch_gemm_down(wide ? h->tm_w2w : h->tm_w2, h->tm_h, d, bn_dn, h->num_sms, s, wide));
     h->prof_done(s);
   } else {
     // MXFP8 token rows of the routed slots
@@ -519,8 +572,39 @@ moe_status moe_forward(moe_handle* h, const void* x, int32_t T, void* y, int32_t
     h->prof_mark(kKGateUpMx, s);
     MOE_TRY_CUDA(launch_gemm_mx_gateup(h->tm_w13q, h->tm_xq, g, bn_mx, h->num_sms, s));
     h->prof_done(s);
-    // 4b. shared experts' gate/up in BF16 (the first tiles of the list)
-    if (S > 0) {
+    // 4b. shared experts' gate/up in BF16. With few tokens the shared expert has
+    // only I/128 weight tiles: split K so every SM streams part of it, then sum
+    // the slices and apply the SwiGLU.
+    const bool sh_split = S > 0 && T <= kSmallRouterMaxTokens;
+    if (sh_split) {
+      for (int j = 0; j < S; ++j) {
+        GemmArgs a{};
+        a.dense_m_tiles = I / 128;
+        a.dense_rows = T;
+        a.dense_k_splits = h->ks_gu;
+        a.num_kb = H / 64;
+        a.a_rows_per_group = 2 * I;
+        a.group_base = -j;
+        a.out = h->sh_parts_gu + static_cast<size_t>(j) * h->ks_gu * T * 2 * I;
+        a.out_ld = 2 * I;
+        a.out_rows = T;
+        a.m_limit = I;
+        a.raw_gateup = 1;
+        a.split_stride = static_cast<size_t>(T) * 2 * I;
+        a.limit = c.swiglu_limit;
+        a.status = h->status;
+        a.timeout_ns = h->timeout_ns;
+        const int nt = a.dense_m_tiles * a.dense_k_splits;
+        h->prof_mark(kKGateUp, s);
+        MOE_TRY_CUDA(launch_gemm_gateup(h->tm_w13sh, tm_x, tm_x, a, 32, nt < h->num_sms ? nt : h->num_sms, s));
+        MOE_TRY_CUDA(launch_swiglu_reduce(a.out ? static_cast<float*>(a.out) : nullptr, h->ks_gu, T, I,
+                                          c.swiglu_limit,
+                                          static_cast<__nv_bfloat16*>(h->h) + (static_cast<size_t>(T) * k +
+                                                                               static_cast<size_t>(j) * T) * I,
+                                          s));
+        h->prof_done(s);
+      }
+    } else if (S > 0) {
       GemmArgs a{};
       a.tiles = h->tiles_gu;
       a.ntiles = h->ntiles + 2;
@@ -558,8 +642,30 @@ moe_status moe_forward(moe_handle* h, const void* x, int32_t T, void* y, int32_t
     h->prof_mark(kKDownMx, s);
     MOE_TRY_CUDA(launch_gemm_mx_down(h->tm_w2q, h->tm_hq, d, bn_mx, h->num_sms, s));
     h->prof_done(s);
-    // 5b. shared experts' down in BF16
-    if (S > 0) {
+    // 5b. shared experts' down in BF16 (split K for few tokens; the combine sums the slices)
+    if (sh_split) {
+      for (int j = 0; j < S; ++j) {
+        GemmArgs a{};
+        a.dense_m_tiles = H / 128;
+        a.dense_rows = T;
+        a.dense_b_row0 = T * k + j * T;
+        a.dense_k_splits = h->ks_dn;
+        a.num_kb = I / 64;
+        a.a_rows_per_group = H;
+        a.group_base = -j;
+        a.out = h->sh_parts_dn + static_cast<size_t>(j) * h->ks_dn * T * H;
+        a.out_ld = H;
+        a.out_rows = T;
+        a.m_limit = H;
+        a.split_stride = static_cast<size_t>(T) * H;
+        a.status = h->status;
+        a.timeout_ns = h->timeout_ns;
+        const int nt = a.dense_m_tiles * a.dense_k_splits;
+        h->prof_mark(kKDown, s);
+        MOE_TRY_CUDA(launch_gemm_down(h->tm_w2sh, h->tm_h, a, 32, nt < h->num_sms ? nt : h->num_sms, s));
+        h->prof_done(s);
+      }
+    } else if (S > 0) {
       GemmArgs a{};
       a.tiles = h->tiles_dn;
       a.ntiles = h->ntiles + 3;
@@ -580,7 +686,9 @@ moe_status moe_forward(moe_handle* h, const void* x, int32_t T, void* y, int32_t
   }
   // 6. weighted combine with the shared experts
   h->prof_mark(kKCombine, s);
-  MOE_TRY_CUDA(launch_combine(h->o, h->inv, h->wts, T, H, k, S, y, s));
+  const bool parts = h->mx && S > 0 && T <= kSmallRouterMaxTokens;
+  MOE_TRY_CUDA(launch_combine(h->o, h->inv, h->wts, T, H, k, S, y, parts ? h->sh_parts_dn : nullptr,
+                              parts ? h->ks_dn : 0, s));
   h->prof_done(s);
   if (topk_idx) MOE_TRY_CUDA(cudaMemcpyAsync(topk_idx, h->idx, static_cast<size_t>(nslots) * 4, cudaMemcpyDefault, s));
   if (topk_w) MOE_TRY_CUDA(cudaMemcpyAsync(topk_w, h->wts, static_cast<size_t>(nslots) * 4, cudaMemcpyDefault, s));

@@ -1,25 +1,27 @@
 // Grouped expert GEMMs on the 5th-generation tensor cores (tcgen05 + TMEM + TMA).
 //
 // Swap-AB formulation: the expert weights are the M operand (128 rows of the
-// weight matrix per tile) and the tokens routed to the expert are the N
-// operand (16..BN tokens), so a decode step with 1-3 tokens per expert still
-// issues full-height MMAs while streaming every weight byte exactly once.
+// weight matrix per MMA) and the tokens routed to the expert are the N operand
+// (16..BN tokens), so a decode step with 1-3 tokens per expert still issues
+// full-height MMAs while streaming every weight byte exactly once.
 //
 //   gate/up tile: D_G[128 x N] = W1[rows] . X^T,  D_U[128 x N] = W3[rows] . X^T
 //                 h[token, i] = silu(min(D_G, L)) * clamp(D_U, -L, L)   -> BF16
 //                 (the gated expert MLP with the swiglu_limit clamp of the
 //                 DeepSeek V4.1 config: "swiglu_limit": 10.0)
-//   down tile:    D[128 x N] = W2[rows] . h^T                            -> fp32 rows
+//   down tile:    D[128 x N] = W2[rows] . h^T (one or two 128-row MMAs) -> fp32 rows
 //
 // One persistent CTA per SM, warp-specialised:
-//   warp 0      TMA producer: A box (weights) + B boxes (token rows) per 64-wide K step
+//   warp 0      TMA producer: per 64-wide K step one A box (weights) and the B
+//               boxes (token rows) into one stage of the shared-memory ring
 //   warp 1      MMA issuer: tcgen05.mma kind::f16, accumulators in TMEM
 //   warps 2..5  epilogue: tcgen05.ld -> math -> global stores
-// A kStages-deep shared-memory ring (full/empty mbarriers) decouples TMA and
-// MMA; two TMEM accumulator buffers (tmem_full/tmem_empty) let the epilogue of
-// tile i overlap the MMAs of tile i+1. Every wait is bounded in time; a wait
-// that runs out records MOE_ERR_TIMEOUT, drains this CTA's in-flight copies and
-// MMAs, frees TMEM and returns.
+// A ring of full/empty mbarriers decouples TMA and MMA (weights and tokens of a
+// stage travel together: separate, differently deep rings for the two measured
+// slower on B200). One or two TMEM accumulator buffers (tmem_full/tmem_empty)
+// let the epilogue of tile i overlap the MMAs of tile i+1 when they fit. Every wait is bounded in time; a wait that runs out
+// records MOE_ERR_TIMEOUT, drains this CTA's in-flight copies and MMAs, frees
+// TMEM and returns.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -31,6 +33,7 @@ constexpr int kThreads = 192;
 constexpr int kBK = 64;           // K elements per stage (128 bytes of BF16 = one swizzle row)
 constexpr int kBBoxRows = 32;     // token rows per B TMA box
 constexpr int kBBoxBytes = kBBoxRows * 128;
+constexpr int kWarpTma = 0, kWarpMma = 1;
 
 constexpr int pow2_at_least(int v, int lo) {
   int p = lo;
@@ -38,27 +41,38 @@ constexpr int pow2_at_least(int v, int lo) {
   return p;
 }
 
-template <bool kGateUp, int BN, int kStages>
+// kAMmas 128-row MMAs per K step share one B tile: gate/up always has two (W1
+// and W3 rows of the same 128 expert-width rows); the down GEMM has one, or two
+// consecutive 128-row tiles of W2 ("wide") to double the work per B byte.
+template <bool kGateUp, int kAMmas, int BN, int kStages>
 struct Cfg {
-  static constexpr int kARows = kGateUp ? 256 : 128;
+  static constexpr int kARows = 128 * kAMmas;
   static constexpr int kABytes = kARows * 128;
   static constexpr int kBBytes = BN * 128;
-  static constexpr int kAccCols = kGateUp ? 2 * BN : BN;
-  static constexpr int kTmemCols = pow2_at_least(2 * kAccCols, 32);
-  static constexpr int kBarrierBytes = 256;
+  static constexpr int kAccCols = kAMmas * BN;
+  // two accumulator buffers when they fit in TMEM, otherwise one
+  static constexpr int kAccBufs = 2 * kAccCols <= 512 ? 2 : 1;
+  static constexpr int kTmemCols = pow2_at_least(kAccBufs * kAccCols, 32);
+  static constexpr int kBarrierBytes = 512;
   static constexpr int kSmemBytes = 1024 + kStages * (kABytes + kBBytes) + kBarrierBytes;
+  static_assert(!kGateUp || kAMmas == 2, "gate/up tiles pair W1 and W3 rows");
   static_assert(kTmemCols <= 512, "TMEM holds 512 columns");
   static_assert(BN % kBBoxRows == 0 && BN >= 32 && BN <= 256, "BN");
+  static_assert((2 * kStages + 5) * 8 + 8 <= kBarrierBytes, "barriers");
   static_assert(kSmemBytes <= 227 * 1024, "shared memory");
 };
 
 struct Tile {
   int group, m_tile, b_row0, out_row0, nrows;
+  int kb0, nkb, split;  // K blocks [kb0, kb0 + nkb) of slice `split`
 };
 
 template <int BN>
 __device__ __forceinline__ Tile load_tile(const GemmArgs& a, int t) {
   Tile r;
+  r.kb0 = 0;
+  r.nkb = a.num_kb;
+  r.split = 0;
   if (a.tiles != nullptr) {
     const int4 v = a.tiles[t];
     r.group = v.x & 0xFFFF;
@@ -67,10 +81,17 @@ __device__ __forceinline__ Tile load_tile(const GemmArgs& a, int t) {
     r.out_row0 = v.z;
     r.nrows = v.w;
   } else {
+    // dense: m fastest, then K slice, then token tile
+    const int ks = max(1, a.dense_k_splits);
     r.group = 0;
     r.m_tile = t % a.dense_m_tiles;
-    const int nt = t / a.dense_m_tiles;
-    r.b_row0 = r.out_row0 = nt * BN;
+    const int rest = t / a.dense_m_tiles;
+    r.split = rest % ks;
+    const int nt = rest / ks;
+    r.nkb = a.num_kb / ks;
+    r.kb0 = r.split * r.nkb;
+    r.out_row0 = nt * BN;
+    r.b_row0 = a.dense_b_row0 + nt * BN;
     r.nrows = min(BN, a.dense_rows - nt * BN);
   }
   // A tile never holds more rows than the B ring has room for.
@@ -81,7 +102,7 @@ __device__ __forceinline__ Tile load_tile(const GemmArgs& a, int t) {
 template <int BN>
 __device__ __forceinline__ int tile_count(const GemmArgs& a) {
   if (a.tiles != nullptr) return *a.ntiles;
-  return a.dense_m_tiles * ((a.dense_rows + BN - 1) / BN);
+  return a.dense_m_tiles * max(1, a.dense_k_splits) * ((a.dense_rows + BN - 1) / BN);
 }
 
 __device__ __forceinline__ int tile_first(const GemmArgs& a) {
@@ -106,22 +127,34 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, co
   }
 }
 
-template <bool kGateUp, int BN, int kStages>
+// After an abort: wait (bounded) until the last `depth` copies this thread
+// issued into a ring have landed, so no copy writes into a CTA that is gone.
+__device__ __forceinline__ void drain_ring(uint64_t* full, int depth, long issued, uint64_t timeout_ns) {
+  for (long i = issued - 1; i >= 0 && i >= issued - depth; --i) {
+    const int s = static_cast<int>(i % depth);
+    const uint32_t par = static_cast<uint32_t>((i / depth) & 1);
+    const uint64_t t0 = globaltimer_ns();
+    while (!mbar_try_wait(&full[s], par) && globaltimer_ns() - t0 < timeout_ns) {
+    }
+  }
+}
+
+template <bool kGateUp, int kAMmas, int BN, int kStages>
 __global__ void __launch_bounds__(kThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                         const __grid_constant__ CUtensorMap tmBsh, const GemmArgs args) {
-  using C = Cfg<kGateUp, BN, kStages>;
+  using C = Cfg<kGateUp, kAMmas, BN, kStages>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
   uint8_t* sB = smem + kStages * C::kABytes;
   uint64_t* bars = reinterpret_cast<uint64_t*>(sB + kStages * C::kBBytes);
   uint64_t* full = bars;
-  uint64_t* empty = bars + kStages;
-  uint64_t* tfull = bars + 2 * kStages;
-  uint64_t* tempty = bars + 2 * kStages + 2;
-  uint64_t* drain = bars + 2 * kStages + 4;
-  uint32_t* tmem_base_smem = reinterpret_cast<uint32_t*>(bars + 2 * kStages + 5);
+  uint64_t* empty = full + kStages;
+  uint64_t* tfull = empty + kStages;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_base_smem = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_base_smem + 1);
 
   const int warp = threadIdx.x / 32;
@@ -140,12 +173,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     *abort_flag = 0;
     fence_mbarrier_init();
   }
-  if (warp == 0 && lane == 0) {
+  if (warp == kWarpTma && lane == 0) {
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
     if (kGateUp) tma_prefetch_desc(&tmBsh);
   }
-  if (warp == 1) {
+  if (warp == kWarpMma) {
     tmem_alloc(tmem_base_smem, C::kTmemCols);
     tmem_relinquish();
   }
@@ -157,64 +190,55 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int ntiles = tile_count<BN>(args);
   const int tfirst = tile_first(args) + static_cast<int>(blockIdx.x);
 
-  if (warp == 0) {
+  if (warp == kWarpTma) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
       long issued = 0;
-      for (int t = tfirst; t < ntiles && !*abort_flag; t += gridDim.x) {
+      bool ok = true;
+      for (int t = tfirst; ok && t < ntiles && !*abort_flag; t += gridDim.x) {
         const Tile tl = load_tile<BN>(args, t);
         const CUtensorMap* mb = (kGateUp && tl.group >= args.n_routed) ? &tmBsh : &tmB;
         const int a_row = (tl.group - args.group_base) * args.a_rows_per_group + tl.m_tile * C::kARows;
         const int nb = (tl.nrows + kBBoxRows - 1) / kBBoxRows;
         const uint32_t bytes = C::kABytes + nb * kBBoxBytes;
-        bool ok = true;
-        for (int kb = 0; kb < args.num_kb; ++kb) {
+        for (int kb = 0; kb < tl.nkb; ++kb) {
           if (!wait_or_abort(&empty[stage], phase ^ 1, args, abort_flag)) {
             ok = false;
             break;
           }
           mbar_arrive_expect_tx(&full[stage], bytes);
-          tma_load_2d(sA + stage * C::kABytes, &tmA, &full[stage], kb * kBK, a_row, kCacheEvictFirst);
+          const int kx = (tl.kb0 + kb) * kBK;
+          tma_load_2d(sA + stage * C::kABytes, &tmA, &full[stage], kx, a_row, kCacheEvictFirst);
           for (int j = 0; j < nb; ++j)
-            tma_load_2d(sB + stage * C::kBBytes + j * kBBoxBytes, mb, &full[stage], kb * kBK,
-                        tl.b_row0 + j * kBBoxRows, kCacheEvictLast);
+            tma_load_2d(sB + stage * C::kBBytes + j * kBBoxBytes, mb, &full[stage], kx, tl.b_row0 + j * kBBoxRows,
+                        kCacheEvictLast);
           ++issued;
           if (++stage == kStages) {
             stage = 0;
             phase ^= 1;
           }
         }
-        if (!ok) break;
       }
-      if (*abort_flag) {
-        // Let every copy this thread started land before the CTA goes away.
-        for (long i = issued - 1; i >= 0 && i >= issued - kStages; --i) {
-          const int s = static_cast<int>(i % kStages);
-          const uint32_t par = static_cast<uint32_t>((i / kStages) & 1);
-          const uint64_t t0 = globaltimer_ns();
-          while (!mbar_try_wait(&full[s], par) && globaltimer_ns() - t0 < args.timeout_ns) {
-          }
-        }
-      }
+      if (*abort_flag) drain_ring(full, kStages, issued, args.timeout_ns);
     }
-  } else if (warp == 1) {
+  } else if (warp == kWarpMma) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
       uint32_t acc_phase = 0;
-      for (int t = tfirst; t < ntiles && !*abort_flag; t += gridDim.x) {
+      bool ok = true;
+      for (int t = tfirst; ok && t < ntiles && !*abort_flag; t += gridDim.x) {
         const Tile tl = load_tile<BN>(args, t);
         const uint32_t n_mma = max(16, (tl.nrows + 15) & ~15);
         const uint32_t idesc = idesc_bf16_f32(128, n_mma);
         if (!wait_or_abort(&tempty[acc], acc_phase ^ 1, args, abort_flag)) break;
         tc_fence_after();
         const uint32_t d = tmem_base + acc * C::kAccCols;
-        bool ok = true;
-        for (int kb = 0; kb < args.num_kb; ++kb) {
+        for (int kb = 0; kb < tl.nkb; ++kb) {
           if (!wait_or_abort(&full[stage], phase, args, abort_flag)) {
             ok = false;
             break;
@@ -226,8 +250,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int k = 0; k < kBK / 16; ++k) {
             const uint64_t bdesc = sdesc_sw128(b_addr + k * 32);
             const uint32_t accum = (kb | k) != 0;
-            umma_f16(d, sdesc_sw128(a_addr + k * 32), bdesc, idesc, accum);
-            if (kGateUp) umma_f16(d + BN, sdesc_sw128(a_addr + 128 * 128 + k * 32), bdesc, idesc, accum);
+#pragma unroll
+            for (int i = 0; i < kAMmas; ++i)
+              umma_f16(d + i * BN, sdesc_sw128(a_addr + i * 128 * 128 + k * 32), bdesc, idesc, accum);
           }
           umma_commit(&empty[stage]);
           if (++stage == kStages) {
@@ -237,7 +262,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (!ok) break;
         umma_commit(&tfull[acc]);
-        if (++acc == 2) {
+        if (++acc == C::kAccBufs) {
           acc = 0;
           acc_phase ^= 1;
         }
@@ -249,7 +274,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   } else {
-    // ------------------------------------------------------------ epilogue
+    // ------------------------------------------------------------ epilogue (warps 2..5)
     const int q = warp & 3;  // TMEM lane quarter this warp may access
     int acc = 0;
     uint32_t acc_phase = 0;
@@ -262,7 +287,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok) break;
       tc_fence_after();
       const uint32_t tb = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * C::kAccCols;
-      const int m = tl.m_tile * 128 + q * 32 + lane;
+      const int m = tl.m_tile * (kGateUp ? 128 : C::kARows) + q * 32 + lane;
       const bool rows_ok = tl.out_row0 >= 0 && tl.out_row0 + tl.nrows <= args.out_rows;
       if (!rows_ok && lane == 0 && q == 0) report_status(args.status, kStatusDevice);
       const bool m_ok = m < args.m_limit && rows_ok;
@@ -273,31 +298,58 @@ __global__ void __launch_bounds__(kThreads, 1)
           uint32_t u[16];
           tmem_ld16(tb + BN + c0, u);
           tmem_ld_wait();
-          __nv_bfloat16* out = static_cast<__nv_bfloat16*>(args.out);
+          if (args.raw_gateup) {
+            // split-K partial sums: fp32 G at column m, U at column m_limit + m
+            float* out = static_cast<float*>(args.out) + static_cast<size_t>(tl.split) * args.split_stride;
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            const int n = c0 + j;
-            if (n < tl.nrows && m_ok) {
-              const float hv = clamped_swiglu_f32(__uint_as_float(g[j]), __uint_as_float(u[j]), args.limit);
-              out[static_cast<size_t>(tl.out_row0 + n) * args.out_ld + m] = __float2bfloat16_rn(hv);
+            for (int j = 0; j < 16; ++j) {
+              const int n = c0 + j;
+              if (n < tl.nrows && m_ok) {
+                const size_t o = static_cast<size_t>(tl.out_row0 + n) * args.out_ld + m;
+                out[o] = __uint_as_float(g[j]);
+                out[o + args.m_limit] = __uint_as_float(u[j]);
+              }
+            }
+          } else {
+            __nv_bfloat16* out = static_cast<__nv_bfloat16*>(args.out);
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+              const int n = c0 + j;
+              if (n < tl.nrows && m_ok) {
+                const float hv = clamped_swiglu_f32(__uint_as_float(g[j]), __uint_as_float(u[j]), args.limit);
+                out[static_cast<size_t>(tl.out_row0 + n) * args.out_ld + m] = __float2bfloat16_rn(hv);
+              }
             }
           }
         } else {
           tmem_ld_wait();
-          float* out = static_cast<float*>(args.out);
-          const float cb = (args.col_bias != nullptr && m_ok) ? args.col_bias[m] : 0.0f;
+          float* out = static_cast<float*>(args.out) + static_cast<size_t>(tl.split) * args.split_stride;
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            const int n = c0 + j;
-            if (n < tl.nrows && m_ok)
-              out[static_cast<size_t>(tl.out_row0 + n) * args.out_ld + m] = __uint_as_float(g[j]) + cb;
+          for (int i = 0; i < kAMmas; ++i) {
+            uint32_t v[16];
+            if (i == 0) {
+#pragma unroll
+              for (int j = 0; j < 16; ++j) v[j] = g[j];
+            } else {
+              tmem_ld16(tb + i * BN + c0, v);
+              tmem_ld_wait();
+            }
+            const int mi = m + i * 128;
+            const bool ok_i = mi < args.m_limit && rows_ok;
+            const float cb = (args.col_bias != nullptr && ok_i) ? args.col_bias[mi] : 0.0f;
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+              const int n = c0 + j;
+              if (n < tl.nrows && ok_i)
+                out[static_cast<size_t>(tl.out_row0 + n) * args.out_ld + mi] = __uint_as_float(v[j]) + cb;
+            }
           }
         }
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&tempty[acc]);
-      if (++acc == 2) {
+      if (++acc == C::kAccBufs) {
         acc = 0;
         acc_phase ^= 1;
       }
@@ -306,54 +358,84 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 1) {
+  if (warp == kWarpMma) {
     tc_fence_after();
     tmem_dealloc(tmem_base, C::kTmemCols);
   }
 }
 
-template <bool kGateUp, int BN, int kStages>
+template <bool kGateUp, int kAMmas, int BN, int kStages>
 cudaError_t set_attr() {
-  return cudaFuncSetAttribute(grouped_gemm_kernel<kGateUp, BN, kStages>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              Cfg<kGateUp, BN, kStages>::kSmemBytes);
+  return cudaFuncSetAttribute(grouped_gemm_kernel<kGateUp, kAMmas, BN, kStages>,
+                              cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              Cfg<kGateUp, kAMmas, BN, kStages>::kSmemBytes);
 }
 
-template <bool kGateUp, int BN, int kStages>
+template <bool kGateUp, int kAMmas, int BN, int kStages>
 cudaError_t launch(const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap& tmBsh, const GemmArgs& a,
                    int grid, cudaStream_t s) {
-  grouped_gemm_kernel<kGateUp, BN, kStages>
-      <<<grid, kThreads, Cfg<kGateUp, BN, kStages>::kSmemBytes, s>>>(tmA, tmB, tmBsh, a);
+  grouped_gemm_kernel<kGateUp, kAMmas, BN, kStages>
+      <<<grid, kThreads, Cfg<kGateUp, kAMmas, BN, kStages>::kSmemBytes, s>>>(tmA, tmB, tmBsh, a);
   return cudaGetLastError();
 }
 
-// Stage counts: as many as fit in 227 KB with the barriers.
-constexpr int kGuSmallStages = 6;   // 6 * (32 KB + 4 KB)
-constexpr int kGuLargeStages = 4;   // 4 * (32 KB + 16 KB)
-constexpr int kDnSmallStages = 10;  // 10 * (16 KB + 4 KB)
-constexpr int kDnLargeStages = 4;   // 4 * (16 KB + 32 KB)
+// Ring depths: as many stages of (A box + B boxes) as fit in 227 KB.
+//   gate/up  BN 32: 6 x (32 + 4) KB   BN 128: 4 x (32 + 16) KB   BN 256: 3 x (32 + 32) KB
+//   down     BN 32: 10 x (16 + 4) KB  BN 256: 4 x (16 + 32) KB   wide: 3 x (32 + 32) KB
+#ifndef MOE_STAGES_GU_SMALL
+#define MOE_STAGES_GU_SMALL 6
+#endif
+#ifndef MOE_STAGES_GU_MID
+#define MOE_STAGES_GU_MID 4
+#endif
+#ifndef MOE_STAGES_GU_LARGE
+#define MOE_STAGES_GU_LARGE 3
+#endif
+#ifndef MOE_STAGES_DN_SMALL
+#define MOE_STAGES_DN_SMALL 10
+#endif
+#ifndef MOE_STAGES_DN_LARGE
+#define MOE_STAGES_DN_LARGE 4
+#endif
+#ifndef MOE_STAGES_DN_WIDE
+#define MOE_STAGES_DN_WIDE 3
+#endif
+#define MOE_GU_SMALL true, 2, 32, MOE_STAGES_GU_SMALL
+#define MOE_GU_MID true, 2, 128, MOE_STAGES_GU_MID
+#define MOE_GU_LARGE true, 2, 256, MOE_STAGES_GU_LARGE
+#define MOE_DN_SMALL false, 1, 32, MOE_STAGES_DN_SMALL
+#define MOE_DN_LARGE false, 1, 256, MOE_STAGES_DN_LARGE
+#define MOE_DN_WIDE false, 2, 256, MOE_STAGES_DN_WIDE
 
 }  // namespace
 
 cudaError_t gemm_set_attributes() {
   cudaError_t e;
-  if ((e = set_attr<true, 32, kGuSmallStages>()) != cudaSuccess) return e;
-  if ((e = set_attr<true, 128, kGuLargeStages>()) != cudaSuccess) return e;
-  if ((e = set_attr<false, 32, kDnSmallStages>()) != cudaSuccess) return e;
-  if ((e = set_attr<false, 256, kDnLargeStages>()) != cudaSuccess) return e;
+  if ((e = set_attr<MOE_GU_SMALL>()) != cudaSuccess) return e;
+  if ((e = set_attr<MOE_GU_MID>()) != cudaSuccess) return e;
+  if ((e = set_attr<MOE_GU_LARGE>()) != cudaSuccess) return e;
+  if ((e = set_attr<MOE_DN_SMALL>()) != cudaSuccess) return e;
+  if ((e = set_attr<MOE_DN_LARGE>()) != cudaSuccess) return e;
+  if ((e = set_attr<MOE_DN_WIDE>()) != cudaSuccess) return e;
   return cudaSuccess;
 }
 
 cudaError_t launch_gemm_gateup(const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap& tmBsh,
                                const GemmArgs& a, int bn, int grid, cudaStream_t s) {
-  if (bn == 32) return launch<true, 32, kGuSmallStages>(tmA, tmB, tmBsh, a, grid, s);
-  if (bn == 128) return launch<true, 128, kGuLargeStages>(tmA, tmB, tmBsh, a, grid, s);
+  if (bn == 32) return launch<MOE_GU_SMALL>(tmA, tmB, tmBsh, a, grid, s);
+  if (bn == 128) return launch<MOE_GU_MID>(tmA, tmB, tmBsh, a, grid, s);
+  if (bn == 256) return launch<MOE_GU_LARGE>(tmA, tmB, tmBsh, a, grid, s);
   return cudaErrorInvalidValue;
 }
 
 cudaError_t launch_gemm_down(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmArgs& a, int bn, int grid,
-                             cudaStream_t s) {
-  if (bn == 32) return launch<false, 32, kDnSmallStages>(tmA, tmB, tmB, a, grid, s);
-  if (bn == 256) return launch<false, 256, kDnLargeStages>(tmA, tmB, tmB, a, grid, s);
+                             cudaStream_t s, bool wide) {
+  if (wide) {
+    if (bn == 256) return launch<MOE_DN_WIDE>(tmA, tmB, tmB, a, grid, s);
+    return cudaErrorInvalidValue;
+  }
+  if (bn == 32) return launch<MOE_DN_SMALL>(tmA, tmB, tmB, a, grid, s);
+  if (bn == 256) return launch<MOE_DN_LARGE>(tmA, tmB, tmB, a, grid, s);
   return cudaErrorInvalidValue;
 }
 

@@ -18,6 +18,7 @@ struct GemmArgs {
   int group_base;               // A rows of group g start at (g - group_base) * a_rows_per_group
   int dense_m_tiles;            // dense mode: 128-row tiles of A
   int dense_rows;               // dense mode: rows of B (tokens)
+  int dense_b_row0;             // dense mode: first B row
   int num_kb;                   // K / 64
   int a_rows_per_group;         // rows of A per group
   int n_routed;                 // gate/up: groups >= n_routed read B through the shared-token map
@@ -27,6 +28,9 @@ struct GemmArgs {
   int m_limit;                  // output columns >= m_limit are not stored
   float limit;                  // swiglu limit (gate/up)
   const float* col_bias;        // down / dense: added to output column m (nullptr = none)
+  int dense_k_splits;           // dense mode: K split into this many slices (partial sums)
+  size_t split_stride;          // dense mode with k splits: elements between the slices' outputs
+  int raw_gateup;               // gate/up: store fp32 G | U (ld = out_ld, U at + I) instead of h
   int* status;                  // device status word
   unsigned long long timeout_ns;
 };
@@ -52,6 +56,15 @@ enum KernelKind {
 // ---- router
 cudaError_t launch_router_logits(const void* x, const void* wg, const float* bias, float* z, int T, int H, int E,
                                  cudaStream_t s);
+// Few tokens (T <= 32): fp32 logit slices [H / router_small_slice(H)][T][E] over
+// CTAs of 8 experts x one hidden slice, then one CTA per token sums the slices,
+// picks the candidates and re-scores them exactly in parallel.
+int router_small_slice(int H);
+cudaError_t router_set_attributes();
+cudaError_t launch_router_small(const void* x, const void* wg, float* part, int T, int H, int E, cudaStream_t s);
+cudaError_t launch_topk_small(const float* part, int nparts, const void* x, const void* wg, const float* bias, int T,
+                              int H, int E, int k, float route_scale, float delta, int32_t* idx, float* w, float* z,
+                              int* status, cudaStream_t s, const float* exact_bias);
 cudaError_t launch_topk_refine(const float* z, const void* x, const void* wg, const float* bias, int T, int H,
                                int E, int k, float route_scale, float delta, int32_t* idx, float* w, int* status,
                                cudaStream_t s);
@@ -76,17 +89,23 @@ struct ScanArgs {
   int32_t* ntile_base_dn;       // [E + 1] same for the down GEMM
 };
 cudaError_t launch_perm_scan(const ScanArgs& a, cudaStream_t s);
+// count + scan + scatter in one launch when all slots fit one chunk
+cudaError_t launch_perm_fused(const ScanArgs& a, const int32_t* idx, int nslots, int32_t* perm, int32_t* inv,
+                              int* status, cudaStream_t s);
 cudaError_t launch_perm_scatter(const int32_t* idx, int nslots, int E, const int32_t* chunk_base, int32_t* perm,
                                 int32_t* inv, cudaStream_t s);
 cudaError_t launch_gather_rows(const void* x, const int32_t* perm, int nrows, int k, int H, void* xp,
                                cudaStream_t s);
 
 // ---- grouped GEMMs (tcgen05)
-// bn: 32 (few tokens per group) or the large-tile variant (gate/up 128, down 256).
+// bn: 32 (few tokens per group), 128 or 256 (gate/up; 256 keeps one TMEM
+// accumulator) and 32 or 256 (down).
 cudaError_t launch_gemm_gateup(const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap& tmBsh,
                                const GemmArgs& a, int bn, int grid, cudaStream_t s);
+// wide: each tile covers 256 rows of W2 (two 128-row MMAs sharing the token tile);
+// the tile list's m tiles are then H / 256.
 cudaError_t launch_gemm_down(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmArgs& a, int bn, int grid,
-                             cudaStream_t s);
+                             cudaStream_t s, bool wide = false);
 cudaError_t gemm_set_attributes();
 
 // ---- MX (MXFP4 routed experts)
@@ -132,8 +151,13 @@ cudaError_t launch_repack_w13_bytes(const void* w1, const void* w3, const void* 
                                     int I, int row_bytes, void* w13, cudaStream_t s);
 
 // ---- combine
+// sh_parts: when not null, the shared experts' outputs are the sum of n_parts fp32
+// slices [n_parts][S][T][H] (split-K partial sums) instead of O's shared rows.
 cudaError_t launch_combine(const float* O, const int32_t* inv, const float* w, int T, int H, int k, int S,
-                           void* y, cudaStream_t s);
+                           void* y, const float* sh_parts, int n_parts, cudaStream_t s);
+// h[row0 + t] = clamped SwiGLU of the sum over n_parts slices of fp32 G | U rows [n_parts][T][2I].
+cudaError_t launch_swiglu_reduce(const float* parts, int n_parts, int T, int I, float limit, void* h,
+                                 cudaStream_t s);
 
 // ---- MX utilities
 cudaError_t launch_quantize_mxfp4(const void* src, int64_t rows, int cols, uint8_t* packed, uint8_t* scales,

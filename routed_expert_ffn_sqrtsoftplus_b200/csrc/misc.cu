@@ -12,18 +12,34 @@ namespace {
 // accumulated in fp32 and rounded once to BF16).
 __global__ void __launch_bounds__(128)
     combine_kernel(const float4* __restrict__ O, const int32_t* __restrict__ inv, const float* __restrict__ w, int T,
-                   int H4, int k, int S, uint2* __restrict__ y) {
+                   int H4, int k, int S, uint2* __restrict__ y, const float4* __restrict__ sh_parts, int n_parts) {
   const int t = blockIdx.x;
   const int c = blockIdx.y * blockDim.x + threadIdx.x;
   if (c >= H4) return;
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
   const size_t routed_rows = static_cast<size_t>(T) * k;
   for (int j = 0; j < S; ++j) {
-    const float4 v = __ldg(O + (routed_rows + static_cast<size_t>(j) * T + t) * H4 + c);
-    acc.x += v.x;
-    acc.y += v.y;
-    acc.z += v.z;
-    acc.w += v.w;
+    if (sh_parts == nullptr) {
+      const float4 v = __ldg(O + (routed_rows + static_cast<size_t>(j) * T + t) * H4 + c);
+      acc.x += v.x;
+      acc.y += v.y;
+      acc.z += v.z;
+      acc.w += v.w;
+    } else {
+      // split-K slices of shared expert j, summed in slice order
+      float4 sj = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int p = 0; p < n_parts; ++p) {
+        const float4 v = __ldg(sh_parts + ((static_cast<size_t>(j) * n_parts + p) * T + t) * H4 + c);
+        sj.x += v.x;
+        sj.y += v.y;
+        sj.z += v.z;
+        sj.w += v.w;
+      }
+      acc.x += sj.x;
+      acc.y += sj.y;
+      acc.z += sj.z;
+      acc.w += sj.w;
+    }
   }
   for (int j = 0; j < k; ++j) {
     const int row = __ldg(inv + static_cast<size_t>(t) * k + j);
@@ -40,6 +56,23 @@ __global__ void __launch_bounds__(128)
   out.x = *reinterpret_cast<uint32_t*>(&lo);
   out.y = *reinterpret_cast<uint32_t*>(&hi);
   y[static_cast<size_t>(t) * H4 + c] = out;
+}
+
+// h[t, i] = silu(min(G, L)) * clamp(U, -L, L) with G, U the sums of the split-K
+// slices parts[p][t][i] and parts[p][t][I + i] (slice order), rounded to BF16.
+__global__ void __launch_bounds__(256)
+    swiglu_reduce_kernel(const float* __restrict__ parts, int n_parts, int T, int I, float limit,
+                         __nv_bfloat16* __restrict__ h) {
+  const size_t i = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i >= static_cast<size_t>(T) * I) return;
+  const size_t t = i / I, c = i % I;
+  float g = 0.f, u = 0.f;
+  for (int p = 0; p < n_parts; ++p) {
+    const float* row = parts + (static_cast<size_t>(p) * T + t) * 2 * I;
+    g += __ldg(row + c);
+    u += __ldg(row + I + c);
+  }
+  h[i] = __float2bfloat16_rn(clamped_swiglu_f32(g, u, limit));
 }
 
 // W13 layout: for each group g and 128-row tile mt of the expert width, 256
@@ -154,12 +187,21 @@ __global__ void wait_timeout_probe_kernel(int* status, unsigned long long timeou
 }  // namespace
 
 cudaError_t launch_combine(const float* O, const int32_t* inv, const float* w, int T, int H, int k, int S, void* y,
-                           cudaStream_t s) {
+                           const float* sh_parts, int n_parts, cudaStream_t s) {
   if (T == 0) return cudaSuccess;
   const int H4 = H / 4;
   const dim3 grid(T, (H4 + 127) / 128);
   combine_kernel<<<grid, 128, 0, s>>>(reinterpret_cast<const float4*>(O), inv, w, T, H4, k, S,
-                                      static_cast<uint2*>(y));
+                                      static_cast<uint2*>(y), reinterpret_cast<const float4*>(sh_parts), n_parts);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_swiglu_reduce(const float* parts, int n_parts, int T, int I, float limit, void* h,
+                                 cudaStream_t s) {
+  const size_t n = static_cast<size_t>(T) * I;
+  if (n == 0) return cudaSuccess;
+  swiglu_reduce_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, s>>>(parts, n_parts, T, I, limit,
+                                                                             static_cast<__nv_bfloat16*>(h));
   return cudaGetLastError();
 }
 

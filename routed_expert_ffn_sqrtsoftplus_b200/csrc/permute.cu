@@ -17,7 +17,7 @@ namespace moe {
 
 namespace {
 
-constexpr int kMaxGroups = 1024;
+constexpr int kMaxGroups = 1024;  // routed + shared groups (one scan thread each)
 
 __global__ void __launch_bounds__(256)
     perm_count_kernel(const int32_t* __restrict__ idx, int nslots, int E, int32_t* __restrict__ chunk_cnt,
@@ -38,105 +38,183 @@ __global__ void __launch_bounds__(256)
   for (int e = threadIdx.x; e < E; e += blockDim.x) chunk_cnt[static_cast<size_t>(blockIdx.x) * E + e] = hist[e];
 }
 
-__global__ void __launch_bounds__(1024) perm_scan_kernel(ScanArgs a) {
+// Exclusive scan of one int per thread over a 1024-thread block; returns the
+// thread's exclusive prefix, *total gets the block sum. Uses warp shuffles and
+// one shared array of 32 warp totals.
+__device__ __forceinline__ int block_exclusive_scan(int v, int* warp_tot, int* total) {
+  const int lane = threadIdx.x % 32, warp = threadIdx.x / 32;
+  int inc = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int n = __shfl_up_sync(0xffffffffu, inc, o);
+    if (lane >= o) inc += n;
+  }
+  if (lane == 31) warp_tot[warp] = inc;
+  __syncthreads();
+  if (warp == 0) {
+    int w = lane < static_cast<int>(blockDim.x / 32) ? warp_tot[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int n = __shfl_up_sync(0xffffffffu, w, o);
+      if (lane >= o) w += n;
+    }
+    warp_tot[lane] = w;  // inclusive over warps
+  }
+  __syncthreads();
+  const int before = warp > 0 ? warp_tot[warp - 1] : 0;
+  *total = warp_tot[blockDim.x / 32 - 1];
+  __syncthreads();
+  return before + inc - v;
+}
+
+// Counts, offsets, token-tile bases and both tile lists, one thread per group.
+// With `fused` (all slots in one chunk) the kernel also builds the histogram
+// and scatters the slots itself, so one launch replaces three.
+__global__ void __launch_bounds__(1024) perm_scan_kernel(ScanArgs a, int fused, const int32_t* idx, int nslots,
+                                                        int32_t* perm, int32_t* inv, int* status) {
   __shared__ int cnt_s[kMaxGroups];
   __shared__ int off_s[kMaxGroups + 1];
-  __shared__ int tgu_s[kMaxGroups + 1];
+  __shared__ int tgu_s[kMaxGroups + 1];   // first gate/up tile of each group (tile order)
   __shared__ int tdn_s[kMaxGroups + 1];
-  __shared__ int ngu_s[kMaxGroups + 1];
+  __shared__ int ngu_s[kMaxGroups + 1];   // first token tile of each routed group
   __shared__ int ndn_s[kMaxGroups + 1];
+  __shared__ int ord_g[kMaxGroups + 1];   // group at tile-order position r
+  __shared__ int warp_tot[32];
+  __shared__ int tot;
   const int G = a.E + a.S;
-  // 1. per-expert totals and per-chunk running counts (relative bases)
-  for (int g = threadIdx.x; g < G; g += blockDim.x) {
-    if (g < a.E) {
-      int run = 0;
-      for (int c = 0; c < a.nchunks; ++c) {
-        const size_t i = static_cast<size_t>(c) * a.E + g;
-        const int v = a.chunk_cnt[i];
-        a.chunk_cnt[i] = run;
-        run += v;
+  const int tid = threadIdx.x;
+  // 1. per-group row counts
+  if (fused) {
+    for (int g = tid; g < a.E; g += blockDim.x) cnt_s[g] = 0;
+    __syncthreads();
+    for (int s = tid; s < nslots; s += blockDim.x) {
+      const int e = idx[s];
+      if (e >= 0 && e < a.E)
+        atomicAdd(&cnt_s[e], 1);
+      else
+        report_status(status, kStatusDevice);
+    }
+    __syncthreads();
+    for (int g = a.E + tid; g < G; g += blockDim.x) cnt_s[g] = a.T;
+  } else {
+    for (int g = tid; g < G; g += blockDim.x) {
+      if (g < a.E) {
+        int run = 0;
+        for (int c = 0; c < a.nchunks; ++c) {
+          const size_t i = static_cast<size_t>(c) * a.E + g;
+          const int v = a.chunk_cnt[i];
+          a.chunk_cnt[i] = run;
+          run += v;
+        }
+        cnt_s[g] = run;
+      } else {
+        cnt_s[g] = a.T;
       }
-      cnt_s[g] = run;
-    } else {
-      cnt_s[g] = a.T;
     }
   }
   __syncthreads();
-  // 2. exclusive scans over groups (serial: G <= 1024)
-  if (threadIdx.x == 0) {
-    int o = 0, tg = 0, td = 0, ng = 0, nd = 0;
-    // tile lists visit the shared experts first, then the routed experts
-    for (int r = 0; r < G; ++r) {
-      const int g = r < a.S ? a.E + r : r - a.S;
-      const int n = cnt_s[g];
-      const bool sh = g >= a.E;
-      const int bgu = sh ? a.bn_gu_s : a.bn_gu_r, bdn = sh ? a.bn_dn_s : a.bn_dn_r;
-      const int ntg = (n + bgu - 1) / bgu, ntd = (n + bdn - 1) / bdn;
-      tgu_s[g] = tg;
-      tdn_s[g] = td;
-      tg += a.m_tiles_gu * ntg;
-      td += a.m_tiles_dn * ntd;
-      if (r == a.S - 1) {
-        a.ntiles[2] = tg;
-        a.ntiles[3] = td;
-      }
-      if (!sh) {
-        ngu_s[g] = ng;
-        ndn_s[g] = nd;
-        ng += ntg;
-        nd += ntd;
-      }
+  // 2. scans (G <= 1024: one group per thread)
+  {
+    const int g = tid;
+    const int n = g < G ? cnt_s[g] : 0;
+    int o = block_exclusive_scan(n, warp_tot, &tot);
+    if (g < G) off_s[g] = o;
+    if (tid == 0) off_s[G] = tot;
+    // tile order: shared groups first, then routed
+    const int r = tid;
+    const int gr = r < G ? (r < a.S ? a.E + r : r - a.S) : -1;
+    const int nr = gr >= 0 ? cnt_s[gr] : 0;
+    const bool sh = gr >= a.E;
+    const int bgu = sh ? a.bn_gu_s : a.bn_gu_r, bdn = sh ? a.bn_dn_s : a.bn_dn_r;
+    const int ntg = (nr + bgu - 1) / bgu, ntd = (nr + bdn - 1) / bdn;
+    int tg = block_exclusive_scan(gr >= 0 ? a.m_tiles_gu * ntg : 0, warp_tot, &tot);
+    if (gr >= 0) tgu_s[r] = tg;
+    if (tid == 0) {
+      tgu_s[G] = tot;
+      a.ntiles[0] = tot;
     }
-    if (a.S == 0) {
-      a.ntiles[2] = 0;
-      a.ntiles[3] = 0;
+    int td = block_exclusive_scan(gr >= 0 ? a.m_tiles_dn * ntd : 0, warp_tot, &tot);
+    if (gr >= 0) tdn_s[r] = td;
+    if (tid == 0) {
+      tdn_s[G] = tot;
+      a.ntiles[1] = tot;
     }
-    ngu_s[a.E] = ng;
-    ndn_s[a.E] = nd;
-    for (int g = 0; g < G; ++g) {
-      off_s[g] = o;
-      o += cnt_s[g];
-    }
-    off_s[G] = o;
-    a.ntiles[0] = tg;
-    a.ntiles[1] = td;
+    int ng = block_exclusive_scan(gr >= 0 && !sh ? ntg : 0, warp_tot, &tot);
+    if (gr >= 0 && !sh) ngu_s[gr] = ng;
+    if (tid == 0) ngu_s[a.E] = tot;
+    int nd = block_exclusive_scan(gr >= 0 && !sh ? ntd : 0, warp_tot, &tot);
+    if (gr >= 0 && !sh) ndn_s[gr] = nd;
+    if (tid == 0) ndn_s[a.E] = tot;
+    if (gr >= 0) ord_g[r] = gr;
   }
   __syncthreads();
+  if (tid == 0) {
+    a.ntiles[2] = a.S > 0 ? tgu_s[a.S] : 0;
+    a.ntiles[3] = a.S > 0 ? tdn_s[a.S] : 0;
+  }
   // 3. outputs
-  for (int g = threadIdx.x; g <= G; g += blockDim.x) {
+  for (int g = tid; g <= G; g += blockDim.x) {
     a.off[g] = off_s[g];
     if (g < G) a.cnt[g] = cnt_s[g];
   }
   if (a.ntile_base_gu != nullptr)
-    for (int g = threadIdx.x; g <= a.E; g += blockDim.x) {
+    for (int g = tid; g <= a.E; g += blockDim.x) {
       a.ntile_base_gu[g] = ngu_s[g];
       a.ntile_base_dn[g] = ndn_s[g];
     }
-  for (int g = threadIdx.x; g < a.E; g += blockDim.x)
-    for (int c = 0; c < a.nchunks; ++c) a.chunk_cnt[static_cast<size_t>(c) * a.E + g] += off_s[g];
-  for (int g = threadIdx.x; g < G; g += blockDim.x) {
-    const int n = cnt_s[g];
-    const bool shared = g >= a.E;
-    const bool mx = a.mx && !shared;
-    // gate/up tiles: m-major, token tiles of one weight tile adjacent
-    int bn = shared ? a.bn_gu_s : a.bn_gu_r;
-    int ntn = (n + bn - 1) / bn;
-    int pos = tgu_s[g];
-    for (int mt = 0; mt < a.m_tiles_gu; ++mt)
-      for (int nt = 0; nt < ntn; ++nt) {
-        const int r0 = nt * bn;
-        const int y = mx ? ngu_s[g] + nt : (shared ? r0 : off_s[g] + r0);
-        a.tiles_gu[pos++] = make_int4(g | (mt << 16), y, off_s[g] + r0, min(bn, n - r0));
+  if (!fused)
+    for (int g = tid; g < a.E; g += blockDim.x)
+      for (int c = 0; c < a.nchunks; ++c) a.chunk_cnt[static_cast<size_t>(c) * a.E + g] += off_s[g];
+  // tile lists, spread over all threads: tile -> group by binary search over the
+  // tile-order prefix, then (m tile, token tile) inside the group
+  for (int list = 0; list < 2; ++list) {
+    const int* pre = list == 0 ? tgu_s : tdn_s;
+    int4* out = list == 0 ? a.tiles_gu : a.tiles_dn;
+    const int total = pre[G];
+    for (int t = tid; t < total; t += blockDim.x) {
+      int lo = 0, hi = G - 1;
+      while (lo < hi) {  // last r with pre[r] <= t
+        const int mid = (lo + hi + 1) >> 1;
+        if (pre[mid] <= t) lo = mid; else hi = mid - 1;
       }
-    bn = shared ? a.bn_dn_s : a.bn_dn_r;
-    ntn = (n + bn - 1) / bn;
-    pos = tdn_s[g];
-    for (int mt = 0; mt < a.m_tiles_dn; ++mt)
-      for (int nt = 0; nt < ntn; ++nt) {
-        const int r0 = nt * bn;
-        const int y = mx ? ndn_s[g] + nt : off_s[g] + r0;
-        a.tiles_dn[pos++] = make_int4(g | (mt << 16), y, off_s[g] + r0, min(bn, n - r0));
+      const int g = ord_g[lo];
+      const bool shared = g >= a.E;
+      const bool mx = a.mx && !shared;
+      const int bn = list == 0 ? (shared ? a.bn_gu_s : a.bn_gu_r) : (shared ? a.bn_dn_s : a.bn_dn_r);
+      const int n = cnt_s[g];
+      const int ntn = (n + bn - 1) / bn;
+      const int local = t - pre[lo];
+      const int mt = local / ntn, nt = local % ntn;
+      const int r0 = nt * bn;
+      int y;
+      if (list == 0)
+        y = mx ? ngu_s[g] + nt : (shared ? r0 : off_s[g] + r0);
+      else
+        y = mx ? ndn_s[g] + nt : off_s[g] + r0;
+      out[t] = make_int4(g | (mt << 16), y, off_s[g] + r0, min(bn, n - r0));
+    }
+  }
+  // 4. fused small case: scatter the slots (one warp, 32 slots at a time, in order)
+  __syncthreads();
+  if (fused && tid < 32) {
+    const int lane = tid;
+    for (int e = lane; e < a.E; e += 32) cnt_s[e] = off_s[e];  // reuse as running position
+    __syncwarp();
+    for (int b = 0; b < nslots; b += 32) {
+      const int s = b + lane;
+      const int e = s < nslots ? idx[s] : -1;
+      const bool valid = e >= 0 && e < a.E;
+      const unsigned peers = __match_any_sync(0xffffffffu, valid ? e : -1);
+      const int rank = __popc(peers & ((1u << lane) - 1u));
+      if (valid) {
+        const int pos = cnt_s[e] + rank;
+        perm[pos] = s;
+        inv[s] = pos;
       }
+      __syncwarp();
+      if (valid && rank == 0) cnt_s[e] += __popc(peers);
+      __syncwarp();
+    }
   }
 }
 
@@ -259,7 +337,14 @@ cudaError_t launch_perm_count(const int32_t* idx, int nslots, int E, int32_t* ch
 
 cudaError_t launch_perm_scan(const ScanArgs& a, cudaStream_t s) {
   if (a.E + a.S > kMaxGroups) return cudaErrorInvalidValue;
-  perm_scan_kernel<<<1, 1024, 0, s>>>(a);
+  perm_scan_kernel<<<1, 1024, 0, s>>>(a, 0, nullptr, 0, nullptr, nullptr, nullptr);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_perm_fused(const ScanArgs& a, const int32_t* idx, int nslots, int32_t* perm, int32_t* inv,
+                              int* status, cudaStream_t s) {
+  if (a.E + a.S > kMaxGroups || nslots > kPermChunk) return cudaErrorInvalidValue;
+  perm_scan_kernel<<<1, 1024, 0, s>>>(a, 1, idx, nslots, perm, inv, status);
   return cudaGetLastError();
 }
 

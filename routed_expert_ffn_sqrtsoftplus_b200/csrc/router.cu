@@ -74,6 +74,57 @@ __global__ void __launch_bounds__(kLogitWarps * 32)
   }
 }
 
+// Approximate logits for up to 32 tokens: CTA = 8 experts x one slice of P
+// hidden values (the tokens' slice staged in shared memory), one warp per
+// expert, 32 fp32 partial sums per lane reduced with a halving butterfly
+// (31 shuffles leave token l's sum in lane l). Slices are written separately
+// ([slice][T][E]) and summed in slice order by the top-k kernel.
+constexpr int kSmallTok = 32;
+
+__global__ void __launch_bounds__(256)
+    router_small_kernel(const uint4* __restrict__ x, const uint4* __restrict__ wg, float* __restrict__ part, int T,
+                        int H, int E, int P) {
+  extern __shared__ uint4 xs[];  // [T][P / 8]
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int slice = blockIdx.y;
+  const int pv = P / 8, hv = H / 8;
+  for (int i = threadIdx.x; i < T * pv; i += blockDim.x) {
+    const int t = i / pv, c = i % pv;
+    xs[i] = __ldg(x + static_cast<size_t>(t) * hv + slice * pv + c);
+  }
+  __syncthreads();
+  const int e = blockIdx.x * 8 + warp;
+  if (e >= E) return;
+  const uint4* wrow = wg + static_cast<size_t>(e) * hv + slice * pv;
+  float v[kSmallTok];
+#pragma unroll
+  for (int i = 0; i < kSmallTok; ++i) v[i] = 0.f;
+  for (int c = lane; c < pv; c += 32) {
+    float wf[8];
+    bf16x8_to_f32(__ldg(wrow + c), wf);
+#pragma unroll
+    for (int tt = 0; tt < kSmallTok; ++tt) {
+      if (tt < T) {
+        float xf[8];
+        bf16x8_to_f32(xs[tt * pv + c], xf);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) v[tt] = fmaf(xf[i], wf[i], v[tt]);
+      }
+    }
+  }
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) {
+    const bool upper = (lane & o) != 0;
+#pragma unroll
+    for (int i = 0; i < o; ++i) {
+      const float send = upper ? v[i] : v[i + o];
+      const float keep = upper ? v[i + o] : v[i];
+      v[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+    }
+  }
+  if (lane < T) part[(static_cast<size_t>(slice) * T + lane) * E + e] = v[0];
+}
+
 __device__ __forceinline__ float softplus_f32(float z) { return fmaxf(z, 0.0f) + log1pf(expf(-fabsf(z))); }
 __device__ __forceinline__ double softplus_f64(double z) { return fmax(z, 0.0) + log1p(exp(-fabs(z))); }
 
@@ -246,7 +297,205 @@ __global__ void __launch_bounds__(kTopkWarps * 32)
   }
 }
 
+// Top-k for few tokens, one CTA per token: warp 0 forms the approximate scores
+// (sum of the logit slices + bias), the k-th score and the candidate set
+// {s >= s_k - delta}; the 8 warps then re-score the candidates exactly (fp32
+// products, fp64 sums, four independent accumulators per lane) in parallel,
+// and warp 0 takes the top-k of the exact scores and the weights.
+// `bias` is added to the summed slices (pass nullptr when the logits already hold
+// it); `exact_bias` is the bias of the exact re-scoring.
+template <int EPL>
+__global__ void __launch_bounds__(256)
+    topk_cta_kernel(const float* __restrict__ part, int nparts, const uint4* __restrict__ x,
+                    const uint4* __restrict__ wg, const float* __restrict__ bias, int T, int H, int E, int k,
+                    float route_scale, float delta, int32_t* __restrict__ idx_out, float* __restrict__ w_out,
+                    float* __restrict__ z_out, int* status, const float* __restrict__ exact_bias) {
+  __shared__ int cand[kMaxCand];
+  __shared__ double cs[kMaxCand];
+  __shared__ int ncand_s;
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int t = blockIdx.x;
+  if (warp == 0) {
+    float s[EPL];
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) {
+      const int e = lane + 32 * i;
+      if (e < E) {
+        float z = bias ? bias[e] : 0.f;
+        for (int p = 0; p < nparts; ++p) z += part[(static_cast<size_t>(p) * T + t) * E + e];
+        if (z_out) z_out[static_cast<size_t>(t) * E + e] = z;
+        s[i] = sqrtf(softplus_f32(z));
+      } else {
+        s[i] = -INFINITY;
+      }
+    }
+    float kth = 0.f;
+    {
+      float tmp[EPL];
+#pragma unroll
+      for (int i = 0; i < EPL; ++i) tmp[i] = s[i];
+      for (int r = 0; r < k; ++r) {
+        float bv = -INFINITY;
+        int bi = 0x7fffffff;
+#pragma unroll
+        for (int i = 0; i < EPL; ++i) {
+          const int e = lane + 32 * i;
+          if (tmp[i] > bv || (tmp[i] == bv && e < bi)) {
+            bv = tmp[i];
+            bi = e;
+          }
+        }
+        warp_argmax(bv, bi);
+        kth = bv;
+#pragma unroll
+        for (int i = 0; i < EPL; ++i)
+          if (lane + 32 * i == bi) tmp[i] = -INFINITY;
+      }
+    }
+    const float thr = kth - delta;
+    int n = 0;
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) {
+      const bool f = s[i] >= thr;
+      const unsigned m = __ballot_sync(0xffffffffu, f);
+      const int pos = n + __popc(m & ((1u << lane) - 1u));
+      if (f && pos < kMaxCand) cand[pos] = lane + 32 * i;
+      n += __popc(m);
+    }
+    if (n > kMaxCand) {
+      float tmp[EPL];
+#pragma unroll
+      for (int i = 0; i < EPL; ++i) tmp[i] = s[i];
+      for (int r = 0; r < kMaxCand; ++r) {
+        float bv = -INFINITY;
+        int bi = 0x7fffffff;
+#pragma unroll
+        for (int i = 0; i < EPL; ++i) {
+          const int e = lane + 32 * i;
+          if (tmp[i] > bv || (tmp[i] == bv && e < bi)) {
+            bv = tmp[i];
+            bi = e;
+          }
+        }
+        warp_argmax(bv, bi);
+        if (lane == 0) cand[r] = bi;
+#pragma unroll
+        for (int i = 0; i < EPL; ++i)
+          if (lane + 32 * i == bi) tmp[i] = -INFINITY;
+      }
+      n = kMaxCand;
+    }
+    if (lane == 0) ncand_s = n;
+  }
+  __syncthreads();
+  const int ncand = ncand_s;
+  const int hv = H / 8;
+  const uint4* xrow = x + static_cast<size_t>(t) * hv;
+  for (int c = warp; c < ncand; c += 8) {
+    const int e = cand[c];
+    const uint4* wrow = wg + static_cast<size_t>(e) * hv;
+    double acc[4] = {0.0, 0.0, 0.0, 0.0};
+    int j = lane;
+    for (; j + 96 < hv; j += 128) {
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        float xf[8], wf[8];
+        bf16x8_to_f32(__ldg(xrow + j + 32 * u), xf);
+        bf16x8_to_f32(__ldg(wrow + j + 32 * u), wf);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[u] += static_cast<double>(xf[i] * wf[i]);
+      }
+    }
+    for (; j < hv; j += 32) {
+      float xf[8], wf[8];
+      bf16x8_to_f32(__ldg(xrow + j), xf);
+      bf16x8_to_f32(__ldg(wrow + j), wf);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) acc[0] += static_cast<double>(xf[i] * wf[i]);
+    }
+    double a = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
+    if (lane == 0) cs[c] = sqrt(softplus_f64(a + (exact_bias ? static_cast<double>(exact_bias[e]) : 0.0)));
+  }
+  __syncthreads();
+  if (warp != 0) return;
+  double v0 = lane < ncand ? cs[lane] : -INFINITY;
+  double v1 = lane + 32 < ncand ? cs[lane + 32] : -INFINITY;
+  const int e0 = lane < ncand ? cand[lane] : 0x7fffffff;
+  const int e1 = lane + 32 < ncand ? cand[lane + 32] : 0x7fffffff;
+  double sel_s[kMaxK];
+  int sel_e[kMaxK];
+  double sum = 0.0;
+  for (int r = 0; r < k; ++r) {
+    double bv;
+    int bi;
+    if (v0 > v1 || (v0 == v1 && e0 < e1)) {
+      bv = v0;
+      bi = e0;
+    } else {
+      bv = v1;
+      bi = e1;
+    }
+    warp_argmax_d(bv, bi);
+    if (e0 == bi) v0 = -INFINITY;
+    if (e1 == bi) v1 = -INFINITY;
+    sel_s[r] = bv;
+    sel_e[r] = bi;
+    sum += bv;
+  }
+  if (lane == 0) {
+    for (int r = 0; r < k; ++r) {
+      const int e = sel_e[r];
+      if (e < 0 || e >= E) report_status(status, kStatusDevice);
+      idx_out[static_cast<size_t>(t) * k + r] = e;
+      w_out[static_cast<size_t>(t) * k + r] = static_cast<float>(route_scale * (sel_s[r] / sum));
+    }
+  }
+}
+
 }  // namespace
+
+cudaError_t router_set_attributes() {
+  return cudaFuncSetAttribute(router_small_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmallTok * 1024 * 2);
+}
+
+int router_small_slice(int H) {
+  for (int p : {1024, 512, 256, 128})
+    if (H % p == 0) return p;
+  return 0;
+}
+
+cudaError_t launch_router_small(const void* x, const void* wg, float* part, int T, int H, int E, cudaStream_t s) {
+  const int P = router_small_slice(H);
+  if (P == 0 || T > kSmallTok) return cudaErrorInvalidValue;
+  const size_t smem = static_cast<size_t>(T) * P * 2;
+  const dim3 grid((E + 7) / 8, H / P);
+  router_small_kernel<<<grid, 256, smem, s>>>(static_cast<const uint4*>(x), static_cast<const uint4*>(wg), part, T,
+                                              H, E, P);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_topk_small(const float* part, int nparts, const void* x, const void* wg, const float* bias, int T,
+                              int H, int E, int k, float route_scale, float delta, int32_t* idx, float* w, float* z,
+                              int* status, cudaStream_t s, const float* exact_bias) {
+  if (k > kMaxK || E > 32 * kMaxEPL) return cudaErrorInvalidValue;
+  const uint4* xv = static_cast<const uint4*>(x);
+  const uint4* wv = static_cast<const uint4*>(wg);
+  const int epl = (E + 31) / 32;
+#define MOE_TOPKS_CASE(N)                                                                                      \
+  if (epl <= N) {                                                                                              \
+    topk_cta_kernel<N><<<T, 256, 0, s>>>(part, nparts, xv, wv, bias, T, H, E, k, route_scale, delta, idx, w, z, \
+                                         status, exact_bias);                                                  \
+    return cudaGetLastError();                                                                                 \
+  }
+  MOE_TOPKS_CASE(1)
+  MOE_TOPKS_CASE(4)
+  MOE_TOPKS_CASE(12)
+  MOE_TOPKS_CASE(16)
+#undef MOE_TOPKS_CASE
+  return cudaErrorInvalidValue;
+}
 
 cudaError_t launch_router_logits(const void* x, const void* wg, const float* bias, float* z, int T, int H, int E,
                                  cudaStream_t s) {

@@ -202,3 +202,19 @@ def test_quantize_mxfp4_bitexact(cuda_device):
     q_ref, s_ref = omx.quantize_mxfp4_packed(parity.f64(w))
     assert np.array_equal(s.cpu().numpy(), s_ref)
     assert np.array_equal(q.cpu().numpy(), q_ref)
+
+
+@pytest.mark.parametrize("T", [7, 37, 200])
+def test_dspark_shaped_layer(cuda_device, T):
+    """The DSpark drafter's routing shape (128 routed experts, 3 active; config.json
+    dspark_n_routed_experts / dspark_n_activated_experts) at small widths."""
+    wl = synth.Workload("dspark_small", T=T, H=512, I=256, E=128, k=3, seed=1005)
+    lay = {k: (v.to(cuda_device) if isinstance(v, torch.Tensor) else v) for k, v in synth.make_layer(wl).items()}
+    layer = moe.MoELayer.from_layer(lay, top_k=wl.k, max_tokens=T)
+    try:
+        y, idx, w = _run(layer, lay["x"])
+        rep = parity.compare_layer(lay, np.arange(T), y.float().cpu().numpy(), idx.cpu().numpy(), w.cpu().numpy(),
+                                   wl.k, wl.route_scale, wl.swiglu_limit)
+        assert rep["rel"] < parity.TOL_Y
+    finally:
+        layer.close()
