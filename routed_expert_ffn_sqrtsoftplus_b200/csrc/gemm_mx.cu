@@ -344,9 +344,9 @@ cudaError_t launch(const CUtensorMap& tmA, const CUtensorMap& tmB, const MxGemmA
   return cudaGetLastError();
 }
 
-constexpr int kGu32Stages = 5;   // 5 * (32 + 4 + 1.5) KB
+constexpr int kGu32Stages = 6;   // 6 * (32 + 4 + 1.5) KB
 constexpr int kGu64Stages = 5;   // 5 * (32 + 8 + 1.5) KB
-constexpr int kDn32Stages = 9;   // 9 * (16 + 4 + 1) KB
+constexpr int kDn32Stages = 10;  // 10 * (16 + 4 + 1) KB
 constexpr int kDn64Stages = 8;   // 8 * (16 + 8 + 1) KB
 
 }  // namespace
