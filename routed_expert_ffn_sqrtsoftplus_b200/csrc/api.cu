@@ -414,12 +414,12 @@ moe_status moe_forward(moe_handle* h, const void* x, int32_t T, void* y, int32_t
   const int nslots = T * k;
   const int nchunks = (nslots + kPermChunk - 1) / kPermChunk;
   // Token tiles. Few tokens: 32-row tiles and deep smem rings (weight streaming).
-  // Many tokens per expert: 256-row tiles so each weight tile is read once and
-  // every staged byte feeds twice the MMA work (one TMEM accumulator).
+  // Many tokens per expert: kBnLarge-row tiles so each weight tile is read once
+  // (one TMEM accumulator for gate/up).
   const bool small = T <= 32;
   const bool large = !small && static_cast<int64_t>(T) * k >= 24LL * E;
-  const int bn_gu = small ? 32 : (large ? 256 : 128);   // BF16 token tiles
-  const int bn_dn = small ? 32 : 256;
+  const int bn_gu = small ? 32 : (large ? kBnLarge : 128);   // BF16 token tiles
+  const int bn_dn = small ? 32 : kBnLarge;
   const bool wide = large && h->wide_ok && !h->mx;      // 256-row W2 tiles
   const int bn_mx = small ? 32 : 64;                    // MXFP4 token tiles (gate/up and down)
 
@@ -451,9 +451,9 @@ moe_status moe_forward(moe_handle* h, const void* x, int32_t T, void* y, int32_t
     a.col_bias = h->bias;
     a.status = h->status;
     a.timeout_ns = h->timeout_ns;
-    const int nt = a.dense_m_tiles * ((T + 255) / 256);
+    const int nt = a.dense_m_tiles * ((T + kBnLarge - 1) / kBnLarge);
     h->prof_mark(kKRouterGemm, s);
-    MOE_TRY_CUDA(launch_gemm_down(h->tm_wg, tm_x, a, 256, nt < h->num_sms ? nt : h->num_sms, s));
+    MOE_TRY_CUDA(launch_gemm_down(h->tm_wg, tm_x, a, kBnLarge, nt < h->num_sms ? nt : h->num_sms, s));
     h->prof_done(s);
   }
   if (T > kSmallRouterMaxTokens) {

@@ -232,7 +232,16 @@ __device__ __forceinline__ void mx_scale(float amax, int emax, int& code, float&
 }
 
 // ---------------------------------------------------------------- math
-__device__ __forceinline__ float silu_f32(float g) { return g / (1.0f + __expf(-g)); }
+// silu(g) = g * sigmoid(g). With e = exp(-|g|) in (0, 1] the denominator 1 + e
+// lies in [1, 2], so the fast reciprocal is accurate to a few ulp for every g and
+// no element takes a slow path (an IEEE divide's slow-path branch would keep the
+// compiler from interleaving the elements of a 16-column epilogue chunk);
+// sigmoid(g) = 1 / (1 + e) for g >= 0 and e / (1 + e) for g < 0.
+__device__ __forceinline__ float silu_f32(float g) {
+  const float e = __expf(-fabsf(g));
+  const float r = __fdividef(1.0f, 1.0f + e);
+  return g * (g >= 0.0f ? r : e * r);
+}
 
 __device__ __forceinline__ float clamped_swiglu_f32(float g, float u, float limit) {
   g = fminf(g, limit);

@@ -379,9 +379,13 @@ cudaError_t launch(const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtenso
   return cudaGetLastError();
 }
 
-// Ring depths: as many stages of (A box + B boxes) as fit in 227 KB.
-//   gate/up  BN 32: 6 x (32 + 4) KB   BN 128: 4 x (32 + 16) KB   BN 256: 3 x (32 + 32) KB
-//   down     BN 32: 10 x (16 + 4) KB  BN 256: 4 x (16 + 32) KB   wide: 3 x (32 + 32) KB
+// Ring depths: as many stages of (A box + B boxes) as fit in 227 KB, unless set.
+//   gate/up  BN 32: 6 x (32 + 4) KB   BN 128: 4 x (32 + 16) KB
+//   down     BN 32: 10 x (16 + 4) KB
+//   large    BN 256: 3 (gate/up, wide down) or 4 (down); BN 192: 4 or 5
+constexpr int ring_fit(int a_bytes, int b_bytes) {
+  return (227 * 1024 - 1024 - 512) / (a_bytes + b_bytes);
+}
 #ifndef MOE_STAGES_GU_SMALL
 #define MOE_STAGES_GU_SMALL 6
 #endif
@@ -389,23 +393,23 @@ cudaError_t launch(const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtenso
 #define MOE_STAGES_GU_MID 4
 #endif
 #ifndef MOE_STAGES_GU_LARGE
-#define MOE_STAGES_GU_LARGE 3
+#define MOE_STAGES_GU_LARGE ring_fit(256 * 128, kBnLarge * 128)
 #endif
 #ifndef MOE_STAGES_DN_SMALL
 #define MOE_STAGES_DN_SMALL 10
 #endif
 #ifndef MOE_STAGES_DN_LARGE
-#define MOE_STAGES_DN_LARGE 4
+#define MOE_STAGES_DN_LARGE ring_fit(128 * 128, kBnLarge * 128)
 #endif
 #ifndef MOE_STAGES_DN_WIDE
-#define MOE_STAGES_DN_WIDE 3
+#define MOE_STAGES_DN_WIDE ring_fit(256 * 128, kBnLarge * 128)
 #endif
 #define MOE_GU_SMALL true, 2, 32, MOE_STAGES_GU_SMALL
 #define MOE_GU_MID true, 2, 128, MOE_STAGES_GU_MID
-#define MOE_GU_LARGE true, 2, 256, MOE_STAGES_GU_LARGE
+#define MOE_GU_LARGE true, 2, kBnLarge, MOE_STAGES_GU_LARGE
 #define MOE_DN_SMALL false, 1, 32, MOE_STAGES_DN_SMALL
-#define MOE_DN_LARGE false, 1, 256, MOE_STAGES_DN_LARGE
-#define MOE_DN_WIDE false, 2, 256, MOE_STAGES_DN_WIDE
+#define MOE_DN_LARGE false, 1, kBnLarge, MOE_STAGES_DN_LARGE
+#define MOE_DN_WIDE false, 2, kBnLarge, MOE_STAGES_DN_WIDE
 
 }  // namespace
 
@@ -424,18 +428,18 @@ cudaError_t launch_gemm_gateup(const CUtensorMap& tmA, const CUtensorMap& tmB, c
                                const GemmArgs& a, int bn, int grid, cudaStream_t s) {
   if (bn == 32) return launch<MOE_GU_SMALL>(tmA, tmB, tmBsh, a, grid, s);
   if (bn == 128) return launch<MOE_GU_MID>(tmA, tmB, tmBsh, a, grid, s);
-  if (bn == 256) return launch<MOE_GU_LARGE>(tmA, tmB, tmBsh, a, grid, s);
+  if (bn == kBnLarge) return launch<MOE_GU_LARGE>(tmA, tmB, tmBsh, a, grid, s);
   return cudaErrorInvalidValue;
 }
 
 cudaError_t launch_gemm_down(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmArgs& a, int bn, int grid,
                              cudaStream_t s, bool wide) {
   if (wide) {
-    if (bn == 256) return launch<MOE_DN_WIDE>(tmA, tmB, tmB, a, grid, s);
+    if (bn == kBnLarge) return launch<MOE_DN_WIDE>(tmA, tmB, tmB, a, grid, s);
     return cudaErrorInvalidValue;
   }
   if (bn == 32) return launch<MOE_DN_SMALL>(tmA, tmB, tmB, a, grid, s);
-  if (bn == 256) return launch<MOE_DN_LARGE>(tmA, tmB, tmB, a, grid, s);
+  if (bn == kBnLarge) return launch<MOE_DN_LARGE>(tmA, tmB, tmB, a, grid, s);
   return cudaErrorInvalidValue;
 }
 

@@ -98,8 +98,15 @@ cudaError_t launch_gather_rows(const void* x, const int32_t* perm, int nrows, in
                                cudaStream_t s);
 
 // ---- grouped GEMMs (tcgen05)
-// bn: 32 (few tokens per group), 128 or 256 (gate/up; 256 keeps one TMEM
-// accumulator) and 32 or 256 (down).
+// Token-tile width of the many-tokens-per-expert GEMMs (gate/up, down and the
+// router GEMM): a multiple of 32 in [32, 256].
+#ifndef MOE_BN_LARGE
+#define MOE_BN_LARGE 256
+#endif
+constexpr int kBnLarge = MOE_BN_LARGE;
+static_assert(kBnLarge % 32 == 0 && kBnLarge >= 32 && kBnLarge <= 256, "large token tile");
+// bn: 32 (few tokens per group), 128 or kBnLarge (gate/up) and 32 or kBnLarge
+// (down).
 cudaError_t launch_gemm_gateup(const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap& tmBsh,
                                const GemmArgs& a, int bn, int grid, cudaStream_t s);
 // wide: each tile covers 256 rows of W2 (two 128-row MMAs sharing the token tile);
