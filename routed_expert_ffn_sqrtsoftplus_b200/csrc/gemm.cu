@@ -15,7 +15,9 @@
 //   warp 0      TMA producer: per 64-wide K step one A box (weights) and the B
 //               boxes (token rows) into one stage of the shared-memory ring
 //   warp 1      MMA issuer: tcgen05.mma kind::f16, accumulators in TMEM
-//   warps 2..5  epilogue: tcgen05.ld -> math -> global stores
+//   warps 2..   epilogue (kEpiWarps): tcgen05.ld -> math -> global stores; warp w
+//               reads TMEM lane quarter w % 4, and the kEpiWarps / 4 warps of a
+//               quarter take interleaved 16-column chunks of the tile
 // A ring of full/empty mbarriers decouples TMA and MMA (weights and tokens of a
 // stage travel together: separate, differently deep rings for the two measured
 // slower on B200). One or two TMEM accumulator buffers (tmem_full/tmem_empty)
@@ -29,7 +31,13 @@ namespace moe {
 
 namespace {
 
-constexpr int kThreads = 192;
+#ifndef MOE_EPI_WARPS
+#define MOE_EPI_WARPS 8
+#endif
+constexpr int kEpiWarps = MOE_EPI_WARPS;  // a multiple of 4
+constexpr int kEpiGroups = kEpiWarps / 4;
+constexpr int kThreads = 64 + 32 * kEpiWarps;
+static_assert(kEpiWarps % 4 == 0 && kEpiWarps >= 4 && kEpiWarps <= 16, "epilogue warps");
 constexpr int kBK = 64;           // K elements per stage (128 bytes of BF16 = one swizzle row)
 constexpr int kBBoxRows = 32;     // token rows per B TMA box
 constexpr int kBBoxBytes = kBBoxRows * 128;
@@ -167,7 +175,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&tfull[i], 1);
-      mbar_init(&tempty[i], 4);  // one arrive per epilogue warp
+      mbar_init(&tempty[i], kEpiWarps);  // one arrive per epilogue warp
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -274,8 +282,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   } else {
-    // ------------------------------------------------------------ epilogue (warps 2..5)
-    const int q = warp & 3;  // TMEM lane quarter this warp may access
+    // ------------------------------------------------------------ epilogue (warps 2..)
+    const int q = warp & 3;                  // TMEM lane quarter this warp may access
+    const int cfirst = ((warp - 2) / 4) * 16;  // this warp's first 16-column chunk
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int t = tfirst; t < ntiles; t += gridDim.x) {
@@ -291,7 +300,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool rows_ok = tl.out_row0 >= 0 && tl.out_row0 + tl.nrows <= args.out_rows;
       if (!rows_ok && lane == 0 && q == 0) report_status(args.status, kStatusDevice);
       const bool m_ok = m < args.m_limit && rows_ok;
-      for (int c0 = 0; c0 < n_mma; c0 += 16) {
+      for (int c0 = cfirst; c0 < n_mma; c0 += 16 * kEpiGroups) {
         uint32_t g[16];
         tmem_ld16(tb + c0, g);
         if constexpr (kGateUp) {
