@@ -421,7 +421,7 @@ moe_status moe_forward(moe_handle* h, const void* x, int32_t T, void* y, int32_t
   const int bn_gu = small ? 32 : (large ? kBnLarge : 128);   // BF16 token tiles
   const int bn_dn = small ? 32 : kBnLarge;
   const bool wide = large && h->wide_ok && !h->mx;      // 256-row W2 tiles
-  const int bn_mx = small ? 32 : 64;                    // MXFP4 token tiles (gate/up and down)
+  const int bn_mx = small ? 32 : (large ? kBnMxLarge : 64);  // MXFP4 token tiles (gate/up and down)
 
   CUtensorMap tm_x;
   if (!make_tmap_bf16(&tm_x, x, static_cast<uint64_t>(T), static_cast<uint64_t>(H), 32)) return MOE_ERR_CUDA;

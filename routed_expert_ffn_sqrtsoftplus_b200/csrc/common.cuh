@@ -217,17 +217,20 @@ __host__ __device__ constexpr uint32_t idesc_mx_e2m1_e4m3(uint32_t M, uint32_t N
 }
 
 // E8M0 scale code and the exact reciprocal scale for an MX block with the given
-// amax (OCP MX v1.0: shared exponent floor(log2 amax) - emax, clamped; code 0 for
-// an all-zero block).
+// amax (OCP MX v1.0: shared exponent floor(log2 amax) - emax, clamped to the
+// E8M0 range; code 0 for an all-zero block). floor(log2 amax) is read from the
+// float's exponent field (subnormal amax: from the position of the leading
+// mantissa bit), and 2^-sh is assembled directly (2^-127 is the subnormal 1 << 22).
 __device__ __forceinline__ void mx_scale(float amax, int emax, int& code, float& inv_scale) {
   code = 0;
   inv_scale = 0.f;
   if (amax > 0.f) {
-    int ex;
-    frexpf(amax, &ex);
-    int sh = max(-127, min(127, (ex - 1) - emax));
+    const uint32_t bits = __float_as_uint(amax);
+    const int be = static_cast<int>((bits >> 23) & 0xFFu);
+    const int e = be != 0 ? be - 127 : (31 - __clz(static_cast<int>(bits & 0x7FFFFFu))) - 149;
+    const int sh = max(-127, min(127, e - emax));
     code = sh + 127;
-    inv_scale = ldexpf(1.0f, -sh);
+    inv_scale = sh < 127 ? __uint_as_float(static_cast<uint32_t>(127 - sh) << 23) : __uint_as_float(1u << 22);
   }
 }
 

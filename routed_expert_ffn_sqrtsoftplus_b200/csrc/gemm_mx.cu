@@ -8,7 +8,8 @@
 // type), B = token rows (E4M3), scale factors in TMEM, fp32 accumulation.
 //
 // Same persistent, warp-specialised structure as the BF16 kernel (warp 0 TMA,
-// warp 1 MMA, warps 2-5 epilogue; smem ring + two TMEM accumulators). One
+// warp 1 MMA, 8 epilogue warps, two per TMEM lane quarter taking interleaved
+// 16-column chunks; smem ring + two TMEM accumulators). One
 // stage covers 128 values of K: A box 128 x (256 | 128) rows, B boxes 128 x 32
 // token rows, and two 1-D bulk copies of pre-arranged scale-factor atoms (512 B
 // per 128 rows x 4 blocks of 32). The MMA warp copies the atoms into this
@@ -26,7 +27,9 @@ namespace moe {
 
 namespace {
 
-constexpr int kThreads = 192;
+constexpr int kEpiWarps = 8;  // two per TMEM lane quarter
+constexpr int kEpiGroups = kEpiWarps / 4;
+constexpr int kThreads = 64 + 32 * kEpiWarps;
 constexpr int kBK = 128;          // K values per stage
 constexpr int kBBoxRows = 32;
 constexpr int kBBoxBytes = kBBoxRows * 128;
@@ -119,7 +122,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&tfull[i], 1);
-      mbar_init(&tempty[i], 4);
+      mbar_init(&tempty[i], kEpiWarps);
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -249,7 +252,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    const int q = warp & 3;
+    const int q = warp & 3;                    // TMEM lane quarter this warp may access
+    const int cfirst = ((warp - 2) / 4) * 16;  // this warp's first 16-column chunk
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int t = tfirst; t < tend; t += gridDim.x) {
@@ -272,7 +276,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         down_base_row = tl.row0 - args.group_off[tl.group];
         down_ntile_base = args.dn_ntile_base[tl.group];
       }
-      for (int c0 = 0; c0 < n_mma; c0 += 16) {
+      for (int c0 = cfirst; c0 < n_mma; c0 += 16 * kEpiGroups) {
         uint32_t g[16];
         tmem_ld16(tb + c0, g);
         if constexpr (kGateUp) {
@@ -348,6 +352,13 @@ constexpr int kGu32Stages = 6;   // 6 * (32 + 4 + 1.5) KB
 constexpr int kGu64Stages = 5;   // 5 * (32 + 8 + 1.5) KB
 constexpr int kDn32Stages = 10;  // 10 * (16 + 4 + 1) KB
 constexpr int kDn64Stages = 8;   // 8 * (16 + 8 + 1) KB
+// other widths: as many stages as fit in 227 KB
+constexpr int mx_ring_fit(int a_bytes, int b_bytes, int sf_bytes) {
+  return (227 * 1024 - 1024 - 256) / (a_bytes + b_bytes + sf_bytes);
+}
+constexpr int kGuLStages = mx_ring_fit(256 * 128, kBnMxLarge * 128, 3 * kAtomBytes);
+constexpr int kDnLStages = mx_ring_fit(128 * 128, kBnMxLarge * 128, 2 * kAtomBytes);
+constexpr bool kExtraWidth = kBnMxLarge != 32 && kBnMxLarge != 64;
 
 }  // namespace
 
@@ -357,6 +368,10 @@ cudaError_t gemm_mx_set_attributes() {
   if ((e = set_attr<true, 64, kGu64Stages>()) != cudaSuccess) return e;
   if ((e = set_attr<false, 32, kDn32Stages>()) != cudaSuccess) return e;
   if ((e = set_attr<false, 64, kDn64Stages>()) != cudaSuccess) return e;
+  if constexpr (kExtraWidth) {
+    if ((e = set_attr<true, kBnMxLarge, kGuLStages>()) != cudaSuccess) return e;
+    if ((e = set_attr<false, kBnMxLarge, kDnLStages>()) != cudaSuccess) return e;
+  }
   return cudaSuccess;
 }
 
@@ -364,6 +379,8 @@ cudaError_t launch_gemm_mx_gateup(const CUtensorMap& tmA, const CUtensorMap& tmB
                                   int grid, cudaStream_t s) {
   if (bn == 32) return launch<true, 32, kGu32Stages>(tmA, tmB, a, grid, s);
   if (bn == 64) return launch<true, 64, kGu64Stages>(tmA, tmB, a, grid, s);
+  if constexpr (kExtraWidth)
+    if (bn == kBnMxLarge) return launch<true, kBnMxLarge, kGuLStages>(tmA, tmB, a, grid, s);
   return cudaErrorInvalidValue;
 }
 
@@ -371,6 +388,8 @@ cudaError_t launch_gemm_mx_down(const CUtensorMap& tmA, const CUtensorMap& tmB, 
                                 int grid, cudaStream_t s) {
   if (bn == 32) return launch<false, 32, kDn32Stages>(tmA, tmB, a, grid, s);
   if (bn == 64) return launch<false, 64, kDn64Stages>(tmA, tmB, a, grid, s);
+  if constexpr (kExtraWidth)
+    if (bn == kBnMxLarge) return launch<false, kBnMxLarge, kDnLStages>(tmA, tmB, a, grid, s);
   return cudaErrorInvalidValue;
 }
 

@@ -116,6 +116,13 @@ cudaError_t launch_gemm_down(const CUtensorMap& tmA, const CUtensorMap& tmB, con
 cudaError_t gemm_set_attributes();
 
 // ---- MX (MXFP4 routed experts)
+// Token-tile width of the MX GEMMs when many tokens meet each expert (32 and 64
+// are always built): a multiple of 32 in [32, 128].
+#ifndef MOE_BN_MX_LARGE
+#define MOE_BN_MX_LARGE 96
+#endif
+constexpr int kBnMxLarge = MOE_BN_MX_LARGE;
+static_assert(kBnMxLarge % 32 == 0 && kBnMxLarge >= 32 && kBnMxLarge <= 128, "large MX token tile");
 struct MxGemmArgs {
   const int4* tiles;            // {group | m_tile << 16, token tile id, first row, rows}
   const int* ntiles;            // device index one past the last tile
