@@ -202,17 +202,23 @@ def peaks():
         return 6650.0, 1590.0, 1400.0, "fallback"
 
 
+def source_digest(files) -> str:
+    """First 16 hex digits of the SHA-256 over the named csrc files, in order."""
+    h = hashlib.sha256()
+    for name in files:
+        with open(os.path.join(ROOT, "routed_expert_ffn_sqrtsoftplus_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
 def recorded_traffic(workload: str, kernel: str):
-    """DRAM bytes per launch from a committed ncu summary, if the kernel source is unchanged since."""
+    """DRAM bytes per launch from a committed ncu summary, if the kernel's sources are unchanged since."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(path) as f:
             rec = json.load(f)
         ent = rec[workload][kernel]
-        src = os.path.join(ROOT, "routed_expert_ffn_sqrtsoftplus_b200", "csrc", ent["source"])
-        with open(src, "rb") as f:
-            h = hashlib.sha256(f.read()).hexdigest()[:16]
-        return ent["bytes_per_launch"] if h == ent["source_sha256_16"] else None
+        return ent["bytes_per_launch"] if source_digest(ent["sources"]) == ent["sources_sha256_16"] else None
     except Exception:
         return None
 
