@@ -60,16 +60,23 @@ def parse():
 
 # ----------------------------------------------------------------------------- distributed
 def dist_setup(args):
+    """One process per GPU (torchrun env); NCCL with GPUs, gloo on a host without
+    them (only the oracle reference arm runs there). The process group's timeout is
+    short so ranks that wait on a lost peer end with an error."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
+    gpu = torch.cuda.is_available()
     if world > 1:
         import datetime
         import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
-                                device_id=torch.device("cuda", local))
-    else:
+        if gpu:
+            torch.cuda.set_device(local)
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                    device_id=torch.device("cuda", local))
+        else:
+            dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=120))
+    elif gpu:
         torch.cuda.set_device(0)
     return world, rank, local
 
@@ -81,12 +88,20 @@ def barrier(world):
 
 
 def max_over_ranks(v: float, world: int) -> float:
+    """The largest of the ranks' values (device times are reported as the max over ranks)."""
     if world == 1:
         return v
     import torch.distributed as dist
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([v], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def weak_scaling_value(world: int, tokens_per_rank: int, steps: int, ms_max: float) -> float:
+    """Whole-job tokens/s: every rank runs `steps` layer calls of `tokens_per_rank`
+    tokens; the job takes the slowest rank's time."""
+    return world * tokens_per_rank * steps / (ms_max / 1e3)
 
 
 # ----------------------------------------------------------------------------- clocks
@@ -306,7 +321,7 @@ def run_ours(args, world, rank, local):
     ms = ev0.elapsed_time(ev1)
     ms = max_over_ranks(ms, world)
     ms_per_step = ms / args.steps
-    value = world * T * args.steps / (ms / 1e3)
+    value = weak_scaling_value(world, T, args.steps, ms)
 
     # ---- end-to-end through host buffers
     xh = x.cpu().pin_memory()
@@ -324,7 +339,7 @@ def run_ours(args, world, rank, local):
     torch.cuda.synchronize()
     barrier(world)
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
-    e2e_value = world * T * e2e_steps / (e2e_ms / 1e3)
+    e2e_value = weak_scaling_value(world, T, e2e_steps, e2e_ms)
 
     hbm, tc, tc_sus, src = peaks()
     # dominant kernel = the one with the largest share of device time
@@ -387,7 +402,9 @@ def run_reference(args, world, rank, local):
     wl = workload_from_args(args)
     if rank != 0:
         return None
-    dev = torch.device("cuda", local)
+    # inputs are drawn on the GPU like the other arm's; a host without one draws
+    # them on the CPU (BF16 workloads only: the MXFP4 codec of the set-up runs on the GPU)
+    dev = torch.device("cuda", local) if torch.cuda.is_available() else torch.device("cpu")
     d, mxq = build_layer(wl, dev)
     total_budget = 150.0
     per_step = max(0.2, total_budget / max(1, args.steps + args.warmup))
