@@ -128,6 +128,7 @@ struct moe_handle {
   uint8_t* sfb_gu = nullptr;    // activation scale atoms, gate/up token tiles
   uint8_t* sfb_dn = nullptr;    // h scale atoms, down token tiles
   int32_t* ntile_base_gu = nullptr;
+  int* bn_choice = nullptr;     // token-tile width the permutation chose (many-token BF16 path)
   int32_t* ntile_base_dn = nullptr;
   int* bad = nullptr;
   int64_t max_ntiles_r = 0;
@@ -323,6 +324,7 @@ moe_status moe_create(const moe_config* cfg, const moe_weights* w, moe_stream_t 
   ok = ok && h->alloc(&h->off, (E + S + 1) * 4, ws);
   ok = ok && h->alloc(&h->perm, Tm * k * 4, ws);
   ok = ok && h->alloc(&h->inv, Tm * k * 4, ws);
+  ok = ok && h->alloc(&h->bn_choice, 16, ws);
   ok = ok && h->alloc(&h->tiles_gu, h->max_tiles_gu * 16, ws);
   ok = ok && h->alloc(&h->tiles_dn, h->max_tiles_dn * 16, ws);
   ok = ok && h->alloc(&h->ntiles, 16, ws);
@@ -421,6 +423,10 @@ moe_status moe_forward(moe_handle* h, const void* x, int32_t T, void* y, int32_t
   const int bn_gu = small ? 32 : (large ? kBnLarge : 128);   // BF16 token tiles
   const int bn_dn = small ? 32 : kBnLarge;
   const bool wide = large && h->wide_ok && !h->mx;      // 256-row W2 tiles
+  // many tokens per expert, BF16: the permutation picks kBnAlt-row tiles (a deeper
+  // ring, one tile per expert) when no routed expert has more rows than that, else
+  // kBnLarge; both GEMM widths are launched and the one not chosen returns at once
+  const bool alt = kBnAlt > 0 && wide;
   const int bn_mx = small ? 32 : (large ? kBnMxLarge : 64);  // MXFP4 token tiles (gate/up and down)
 
   CUtensorMap tm_x;
@@ -491,6 +497,8 @@ moe_status moe_forward(moe_handle* h, const void* x, int32_t T, void* y, int32_t
   sa.mx = h->mx ? 1 : 0;
   sa.ntile_base_gu = h->ntile_base_gu;
   sa.ntile_base_dn = h->ntile_base_dn;
+  sa.bn_alt = alt ? kBnAlt : 0;
+  sa.bn_choice = alt ? h->bn_choice : nullptr;
   if (nchunks == 1) {
     h->prof_mark(kKPermScan, s);
     MOE_TRY_CUDA(launch_perm_fused(sa, h->idx, nslots, h->perm, h->inv, h->status, s));
@@ -523,7 +531,15 @@ moe_status moe_forward(moe_handle* h, const void* x, int32_t T, void* y, int32_t
     a.status = h->status;
     a.timeout_ns = h->timeout_ns;
     h->prof_mark(kKGateUp, s);
-    MOE_TRY_CUDA(launch_gemm_gateup(h->tm_w13, h->tm_xp, tm_x, a, bn_gu, h->num_sms, s));
+    if (alt) {
+      a.bn_select = h->bn_choice;
+      a.bn_self = kBnLarge;
+      MOE_TRY_CUDA(launch_gemm_gateup(h->tm_w13, h->tm_xp, tm_x, a, kBnLarge, h->num_sms, s));
+      a.bn_self = kBnAlt;
+      MOE_TRY_CUDA(launch_gemm_gateup(h->tm_w13, h->tm_xp, tm_x, a, kBnAlt, h->num_sms, s));
+    } else {
+      MOE_TRY_CUDA(launch_gemm_gateup(h->tm_w13, h->tm_xp, tm_x, a, bn_gu, h->num_sms, s));
+    }
     h->prof_done(s);
     // 5. down grouped GEMM
     GemmArgs d{};
@@ -539,7 +555,15 @@ moe_status moe_forward(moe_handle* h, const void* x, int32_t T, void* y, int32_t
     d.status = h->status;
     d.timeout_ns = h->timeout_ns;
     h->prof_mark(kKDown, s);
-    MOE_TRY_CUDA(launch_gemm_down(wide ? h->tm_w2w : h->tm_w2, h->tm_h, d, bn_dn, h->num_sms, s, wide));
+    if (alt) {
+      d.bn_select = h->bn_choice;
+      d.bn_self = kBnLarge;
+      MOE_TRY_CUDA(launch_gemm_down(h->tm_w2w, h->tm_h, d, kBnLarge, h->num_sms, s, true));
+      d.bn_self = kBnAlt;
+      MOE_TRY_CUDA(launch_gemm_down(h->tm_w2w, h->tm_h, d, kBnAlt, h->num_sms, s, true));
+    } else {
+      MOE_TRY_CUDA(launch_gemm_down(wide ? h->tm_w2w : h->tm_w2, h->tm_h, d, bn_dn, h->num_sms, s, wide));
+    }
     h->prof_done(s);
   } else {
     // MXFP8 token rows of the routed slots

@@ -152,6 +152,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                         const __grid_constant__ CUtensorMap tmBsh, const GemmArgs args) {
   using C = Cfg<kGateUp, kAMmas, BN, kStages>;
+  // the tile lists were built for the other token-tile width: nothing to do
+  if (args.bn_select != nullptr && *args.bn_select != args.bn_self) return;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
@@ -419,6 +421,10 @@ constexpr int ring_fit(int a_bytes, int b_bytes) {
 #define MOE_DN_SMALL false, 1, 32, MOE_STAGES_DN_SMALL
 #define MOE_DN_LARGE false, 1, kBnLarge, MOE_STAGES_DN_LARGE
 #define MOE_DN_WIDE false, 2, kBnLarge, MOE_STAGES_DN_WIDE
+// the device-chosen alternative width (as many stages as fit)
+constexpr int kBnAltT = kBnAlt > 0 ? kBnAlt : 64;  // an unused placeholder when disabled
+#define MOE_GU_ALT true, 2, kBnAltT, ring_fit(256 * 128, kBnAltT * 128)
+#define MOE_DN_WIDE_ALT false, 2, kBnAltT, ring_fit(256 * 128, kBnAltT * 128)
 
 }  // namespace
 
@@ -430,6 +436,10 @@ cudaError_t gemm_set_attributes() {
   if ((e = set_attr<MOE_DN_SMALL>()) != cudaSuccess) return e;
   if ((e = set_attr<MOE_DN_LARGE>()) != cudaSuccess) return e;
   if ((e = set_attr<MOE_DN_WIDE>()) != cudaSuccess) return e;
+  if constexpr (kBnAlt > 0) {
+    if ((e = set_attr<MOE_GU_ALT>()) != cudaSuccess) return e;
+    if ((e = set_attr<MOE_DN_WIDE_ALT>()) != cudaSuccess) return e;
+  }
   return cudaSuccess;
 }
 
@@ -438,6 +448,8 @@ cudaError_t launch_gemm_gateup(const CUtensorMap& tmA, const CUtensorMap& tmB, c
   if (bn == 32) return launch<MOE_GU_SMALL>(tmA, tmB, tmBsh, a, grid, s);
   if (bn == 128) return launch<MOE_GU_MID>(tmA, tmB, tmBsh, a, grid, s);
   if (bn == kBnLarge) return launch<MOE_GU_LARGE>(tmA, tmB, tmBsh, a, grid, s);
+  if constexpr (kBnAlt > 0)
+    if (bn == kBnAlt) return launch<MOE_GU_ALT>(tmA, tmB, tmBsh, a, grid, s);
   return cudaErrorInvalidValue;
 }
 
@@ -445,6 +457,8 @@ cudaError_t launch_gemm_down(const CUtensorMap& tmA, const CUtensorMap& tmB, con
                              cudaStream_t s, bool wide) {
   if (wide) {
     if (bn == kBnLarge) return launch<MOE_DN_WIDE>(tmA, tmB, tmB, a, grid, s);
+    if constexpr (kBnAlt > 0)
+      if (bn == kBnAlt) return launch<MOE_DN_WIDE_ALT>(tmA, tmB, tmB, a, grid, s);
     return cudaErrorInvalidValue;
   }
   if (bn == 32) return launch<MOE_DN_SMALL>(tmA, tmB, tmB, a, grid, s);

@@ -33,6 +33,8 @@ struct GemmArgs {
   int raw_gateup;               // gate/up: store fp32 G | U (ld = out_ld, U at + I) instead of h
   int* status;                  // device status word
   unsigned long long timeout_ns;
+  const int* bn_select;         // grouped mode: token-tile width chosen on the device (nullptr = always run)
+  int bn_self;                  // this kernel's width: it returns at once unless *bn_select == bn_self
 };
 
 // Kernel kinds for profiling (order = moe_kernel_name()).
@@ -87,6 +89,8 @@ struct ScanArgs {
   int mx;                       // routed tiles carry their token-tile id in .y
   int32_t* ntile_base_gu;       // [E + 1] first token tile of each routed group (gate/up)
   int32_t* ntile_base_dn;       // [E + 1] same for the down GEMM
+  int bn_alt;                   // > 0: use this width for every tile when no routed group has more rows
+  int* bn_choice;               // out: the width the tile lists were built with (bn_alt, or bn_gu_r)
 };
 cudaError_t launch_perm_scan(const ScanArgs& a, cudaStream_t s);
 // count + scan + scatter in one launch when all slots fit one chunk
@@ -105,6 +109,14 @@ cudaError_t launch_gather_rows(const void* x, const int32_t* perm, int nrows, in
 #endif
 constexpr int kBnLarge = MOE_BN_LARGE;
 static_assert(kBnLarge % 32 == 0 && kBnLarge >= 32 && kBnLarge <= 256, "large token tile");
+// Narrower many-token width the permutation picks on the device when no routed
+// expert has more rows (one tile per expert with a deeper ring); 0 = never.
+#ifndef MOE_BN_ALT
+#define MOE_BN_ALT 192
+#endif
+constexpr int kBnAlt = MOE_BN_ALT;
+static_assert(kBnAlt == 0 || (kBnAlt % 32 == 0 && kBnAlt >= 32 && kBnAlt < kBnLarge && kBnAlt != 128 &&
+                              kBnAlt != 32), "alternative token tile");
 // bn: 32 (few tokens per group), 128 or kBnLarge (gate/up) and 32 or kBnLarge
 // (down).
 cudaError_t launch_gemm_gateup(const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap& tmBsh,

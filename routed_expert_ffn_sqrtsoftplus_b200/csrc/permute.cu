@@ -81,6 +81,7 @@ __global__ void __launch_bounds__(1024) perm_scan_kernel(ScanArgs a, int fused, 
   __shared__ int ord_g[kMaxGroups + 1];   // group at tile-order position r
   __shared__ int warp_tot[32];
   __shared__ int tot;
+  __shared__ int maxc_s;
   const int G = a.E + a.S;
   const int tid = threadIdx.x;
   // 1. per-group row counts
@@ -112,7 +113,15 @@ __global__ void __launch_bounds__(1024) perm_scan_kernel(ScanArgs a, int fused, 
       }
     }
   }
+  // token-tile widths: the narrower alternative when no routed group exceeds it
+  if (tid == 0) maxc_s = 0;
   __syncthreads();
+  for (int g = tid; g < a.E; g += blockDim.x) atomicMax(&maxc_s, cnt_s[g]);
+  __syncthreads();
+  const bool alt = a.bn_alt > 0 && maxc_s <= a.bn_alt;
+  const int bn_gu_r = alt ? a.bn_alt : a.bn_gu_r, bn_dn_r = alt ? a.bn_alt : a.bn_dn_r;
+  const int bn_gu_s = alt ? a.bn_alt : a.bn_gu_s, bn_dn_s = alt ? a.bn_alt : a.bn_dn_s;
+  if (tid == 0 && a.bn_choice != nullptr) *a.bn_choice = alt ? a.bn_alt : a.bn_gu_r;
   // 2. scans (G <= 1024: one group per thread)
   {
     const int g = tid;
@@ -125,7 +134,7 @@ __global__ void __launch_bounds__(1024) perm_scan_kernel(ScanArgs a, int fused, 
     const int gr = r < G ? (r < a.S ? a.E + r : r - a.S) : -1;
     const int nr = gr >= 0 ? cnt_s[gr] : 0;
     const bool sh = gr >= a.E;
-    const int bgu = sh ? a.bn_gu_s : a.bn_gu_r, bdn = sh ? a.bn_dn_s : a.bn_dn_r;
+    const int bgu = sh ? bn_gu_s : bn_gu_r, bdn = sh ? bn_dn_s : bn_dn_r;
     const int ntg = (nr + bgu - 1) / bgu, ntd = (nr + bdn - 1) / bdn;
     int tg = block_exclusive_scan(gr >= 0 ? a.m_tiles_gu * ntg : 0, warp_tot, &tot);
     if (gr >= 0) tgu_s[r] = tg;
@@ -180,7 +189,7 @@ __global__ void __launch_bounds__(1024) perm_scan_kernel(ScanArgs a, int fused, 
       const int g = ord_g[lo];
       const bool shared = g >= a.E;
       const bool mx = a.mx && !shared;
-      const int bn = list == 0 ? (shared ? a.bn_gu_s : a.bn_gu_r) : (shared ? a.bn_dn_s : a.bn_dn_r);
+      const int bn = list == 0 ? (shared ? bn_gu_s : bn_gu_r) : (shared ? bn_dn_s : bn_dn_r);
       const int n = cnt_s[g];
       const int ntn = (n + bn - 1) / bn;
       const int local = t - pre[lo];

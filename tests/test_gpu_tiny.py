@@ -56,6 +56,28 @@ def test_tiny_layer_parity_large_T(tiny, T):
     assert rep["rel"] < parity.TOL_Y
 
 
+@pytest.mark.parametrize("T", [300, 700])
+def test_tiny_layer_parity_hot_experts(tiny, cuda_device, T):
+    """A router bias of +6 on experts 0 and 1 sends every token to both: groups of
+    T rows, more than the narrower many-token tile holds, so the permutation keeps
+    the widest tiles and splits each hot expert over several of them."""
+    lay, _ = tiny
+    bias = torch.zeros(WL.E, dtype=torch.float32, device=cuda_device)
+    bias[:2] = 6.0
+    hot = dict(lay, bias=bias)
+    layer = moe.MoELayer.from_layer(hot, top_k=WL.k, max_tokens=700)
+    try:
+        x = lay["x"][:T].contiguous()
+        y, idx, w = _run(layer, x)
+        cnt = np.bincount(idx.cpu().numpy().ravel(), minlength=WL.E)
+        assert cnt[0] == T and cnt[1] == T
+        rep = parity.compare_layer(dict(hot, x=x), np.arange(T), y.float().cpu().numpy(), idx.cpu().numpy(),
+                                   w.cpu().numpy(), WL.k, WL.route_scale, WL.swiglu_limit)
+        assert rep["rel"] < parity.TOL_Y
+    finally:
+        layer.close()
+
+
 @pytest.mark.parametrize("T", [64, 300])
 def test_permutation_is_exact(tiny, T):
     lay, layer = tiny
