@@ -80,6 +80,9 @@ __global__ void __launch_bounds__(kLogitWarps * 32)
 // (31 shuffles leave token l's sum in lane l). Slices are written separately
 // ([slice][T][E]) and summed in slice order by the top-k kernel.
 constexpr int kSmallTok = 32;
+constexpr int kSmallMaxSlice = 1024;                            // P <= 1024
+constexpr int kSmallWChunks = kSmallMaxSlice / 8 / 32;          // Wg chunks per lane
+constexpr int kSmallStage = kSmallTok * kSmallMaxSlice / 8 / 256;  // x chunks per thread
 
 __global__ void __launch_bounds__(256)
     router_small_kernel(const uint4* __restrict__ x, const uint4* __restrict__ wg, float* __restrict__ part, int T,
@@ -88,20 +91,40 @@ __global__ void __launch_bounds__(256)
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int slice = blockIdx.y;
   const int pv = P / 8, hv = H / 8;
-  for (int i = threadIdx.x; i < T * pv; i += blockDim.x) {
-    const int t = i / pv, c = i % pv;
-    xs[i] = __ldg(x + static_cast<size_t>(t) * hv + slice * pv + c);
+  const int e = blockIdx.x * 8 + warp;
+  const uint4* wrow = wg + static_cast<size_t>(e < E ? e : 0) * hv + slice * pv;
+  // this lane's Wg chunks (pv <= 128: at most 4), issued before the x staging so
+  // both sets of loads are in flight together
+  uint4 wv[kSmallWChunks];
+#pragma unroll
+  for (int j = 0; j < kSmallWChunks; ++j)
+    if (lane + 32 * j < pv) wv[j] = __ldg(wrow + lane + 32 * j);
+  // stage the tokens' slice: every load of a thread issued before its stores
+  const int n = T * pv;
+  {
+    uint4 tmp[kSmallStage];
+#pragma unroll
+    for (int j = 0; j < kSmallStage; ++j) {
+      const int i = threadIdx.x + j * 256;
+      if (i < n) tmp[j] = __ldg(x + static_cast<size_t>(i / pv) * hv + slice * pv + i % pv);
+    }
+#pragma unroll
+    for (int j = 0; j < kSmallStage; ++j) {
+      const int i = threadIdx.x + j * 256;
+      if (i < n) xs[i] = tmp[j];
+    }
   }
   __syncthreads();
-  const int e = blockIdx.x * 8 + warp;
   if (e >= E) return;
-  const uint4* wrow = wg + static_cast<size_t>(e) * hv + slice * pv;
   float v[kSmallTok];
 #pragma unroll
   for (int i = 0; i < kSmallTok; ++i) v[i] = 0.f;
-  for (int c = lane; c < pv; c += 32) {
+#pragma unroll
+  for (int j = 0; j < kSmallWChunks; ++j) {
+    const int c = lane + 32 * j;
+    if (c >= pv) break;
     float wf[8];
-    bf16x8_to_f32(__ldg(wrow + c), wf);
+    bf16x8_to_f32(wv[j], wf);
 #pragma unroll
     for (int tt = 0; tt < kSmallTok; ++tt) {
       if (tt < T) {
@@ -153,6 +176,8 @@ __device__ __forceinline__ void warp_argmax_d(double& v, int& i) {
 }
 
 constexpr int kTopkWarps = 8;
+constexpr int kPartBatch = 4;      // logit slices loaded together (top-k CTA kernel)
+constexpr int kWBatch = 10;        // Wg chunks per lane loaded together (exact re-scoring)
 constexpr int kMaxCand = 64;       // candidates refined per token
 constexpr int kMaxEPL = 16;        // experts per lane (E <= 512)
 constexpr int kMaxK = 32;
@@ -313,18 +338,50 @@ __global__ void __launch_bounds__(256)
   __shared__ int cand[kMaxCand];
   __shared__ double cs[kMaxCand];
   __shared__ int ncand_s;
+  extern __shared__ uint4 xrow_s[];  // this token's row (H / 8 chunks), staged by warps 1..7
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int t = blockIdx.x;
-  if (warp == 0) {
+  const int hv = H / 8;
+  const uint4* xrow = x + static_cast<size_t>(t) * hv;
+  if (warp != 0) {
+    for (int c = threadIdx.x - 32; c < hv; c += blockDim.x - 32) xrow_s[c] = __ldg(xrow + c);
+  } else {
+    // summed logit slices, added in slice order; all of a lane's loads are
+    // independent, so they are issued together
     float s[EPL];
+    float zi[EPL];
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) {
+      const int e = lane + 32 * i;
+      zi[i] = (e < E && bias) ? bias[e] : 0.f;
+    }
+    int p = 0;
+    for (; p + kPartBatch <= nparts; p += kPartBatch) {
+      float pv[kPartBatch][EPL];
+#pragma unroll
+      for (int q = 0; q < kPartBatch; ++q)
+#pragma unroll
+        for (int i = 0; i < EPL; ++i) {
+          const int e = lane + 32 * i;
+          pv[q][i] = e < E ? part[(static_cast<size_t>(p + q) * T + t) * E + e] : 0.f;
+        }
+#pragma unroll
+      for (int q = 0; q < kPartBatch; ++q)
+#pragma unroll
+        for (int i = 0; i < EPL; ++i) zi[i] += pv[q][i];
+    }
+    for (; p < nparts; ++p)
+#pragma unroll
+      for (int i = 0; i < EPL; ++i) {
+        const int e = lane + 32 * i;
+        if (e < E) zi[i] += part[(static_cast<size_t>(p) * T + t) * E + e];
+      }
 #pragma unroll
     for (int i = 0; i < EPL; ++i) {
       const int e = lane + 32 * i;
       if (e < E) {
-        float z = bias ? bias[e] : 0.f;
-        for (int p = 0; p < nparts; ++p) z += part[(static_cast<size_t>(p) * T + t) * E + e];
-        if (z_out) z_out[static_cast<size_t>(t) * E + e] = z;
-        s[i] = sqrtf(softplus_f32(z));
+        if (z_out) z_out[static_cast<size_t>(t) * E + e] = zi[i];
+        s[i] = sqrtf(softplus_f32(zi[i]));
       } else {
         s[i] = -INFINITY;
       }
@@ -389,29 +446,28 @@ __global__ void __launch_bounds__(256)
   }
   __syncthreads();
   const int ncand = ncand_s;
-  const int hv = H / 8;
-  const uint4* xrow = x + static_cast<size_t>(t) * hv;
   for (int c = warp; c < ncand; c += 8) {
     const int e = cand[c];
     const uint4* wrow = wg + static_cast<size_t>(e) * hv;
+    // chunk q of this lane is j = lane + 32 q; four accumulators by q mod 4, each
+    // in increasing q; the Wg chunks of a batch are loaded together
     double acc[4] = {0.0, 0.0, 0.0, 0.0};
-    int j = lane;
-    for (; j + 96 < hv; j += 128) {
+    const int nq = (hv - lane + 31) / 32;
+    for (int q0 = 0; q0 < nq; q0 += kWBatch) {
+      uint4 wv[kWBatch];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        float xf[8], wf[8];
-        bf16x8_to_f32(__ldg(xrow + j + 32 * u), xf);
-        bf16x8_to_f32(__ldg(wrow + j + 32 * u), wf);
+      for (int u = 0; u < kWBatch; ++u)
+        if (q0 + u < nq) wv[u] = __ldg(wrow + lane + 32 * (q0 + u));
 #pragma unroll
-        for (int i = 0; i < 8; ++i) acc[u] += static_cast<double>(xf[i] * wf[i]);
+      for (int u = 0; u < kWBatch; ++u) {
+        if (q0 + u < nq) {
+          float xf[8], wf[8];
+          bf16x8_to_f32(xrow_s[lane + 32 * (q0 + u)], xf);
+          bf16x8_to_f32(wv[u], wf);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) acc[(q0 + u) & 3] += static_cast<double>(xf[i] * wf[i]);
+        }
       }
-    }
-    for (; j < hv; j += 32) {
-      float xf[8], wf[8];
-      bf16x8_to_f32(__ldg(xrow + j), xf);
-      bf16x8_to_f32(__ldg(wrow + j), wf);
-#pragma unroll
-      for (int i = 0; i < 8; ++i) acc[0] += static_cast<double>(xf[i] * wf[i]);
     }
     double a = (acc[0] + acc[1]) + (acc[2] + acc[3]);
 #pragma unroll
@@ -479,13 +535,15 @@ cudaError_t launch_router_small(const void* x, const void* wg, float* part, int 
 cudaError_t launch_topk_small(const float* part, int nparts, const void* x, const void* wg, const float* bias, int T,
                               int H, int E, int k, float route_scale, float delta, int32_t* idx, float* w, float* z,
                               int* status, cudaStream_t s, const float* exact_bias) {
-  if (k > kMaxK || E > 32 * kMaxEPL) return cudaErrorInvalidValue;
+  // the token's row is staged in shared memory (within the default 48 KB)
+  if (k > kMaxK || E > 32 * kMaxEPL || static_cast<size_t>(H) * 2 > 40 * 1024) return cudaErrorInvalidValue;
   const uint4* xv = static_cast<const uint4*>(x);
   const uint4* wv = static_cast<const uint4*>(wg);
   const int epl = (E + 31) / 32;
 #define MOE_TOPKS_CASE(N)                                                                                      \
   if (epl <= N) {                                                                                              \
-    topk_cta_kernel<N><<<T, 256, 0, s>>>(part, nparts, xv, wv, bias, T, H, E, k, route_scale, delta, idx, w, z, \
+    topk_cta_kernel<N><<<T, 256, static_cast<size_t>(H) * 2, s>>>(part, nparts, xv, wv, bias, T, H, E, k,      \
+                                                                 route_scale, delta, idx, w, z,                  \
                                          status, exact_bias);                                                  \
     return cudaGetLastError();                                                                                 \
   }
