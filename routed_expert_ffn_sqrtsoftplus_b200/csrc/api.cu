@@ -59,7 +59,7 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 const char* kKernelNames[kKNumKinds] = {"router_logits", "router_gemm",  "topk_refine", "perm_count",
                                         "perm_scan",     "perm_scatter", "gather_rows", "gemm_gateup",
                                         "gemm_down",     "combine",      "quant_x",     "gemm_gateup_mx",
-                                        "gemm_down_mx"};
+                                        "gemm_down_mx",  "swiglu_reduce"};
 
 // 2-D tensor map, 128-byte swizzle, box of box_cols x box_rows elements.
 bool make_tmap(CUtensorMap* m, const void* ptr, CUtensorMapDataType dt, uint64_t rows, uint64_t cols,
@@ -425,7 +425,7 @@ moe_status moe_forward(moe_handle* h, const void* x, int32_t T, void* y, int32_t
   const bool wide = large && h->wide_ok && !h->mx;      // 256-row W2 tiles
   // many tokens per expert, BF16: the permutation picks kBnAlt-row tiles (a deeper
   // ring, one tile per expert) when no routed expert has more rows than that, else
-  // kBnLarge; both GEMM widths are launched and the one not chosen returns at once
+  // kBnLarge; one dual-width launch per GEMM runs the chosen body
   const bool alt = kBnAlt > 0 && wide;
   const int bn_mx = small ? 32 : (large ? kBnMxLarge : 64);  // MXFP4 token tiles (gate/up and down)
 
@@ -533,10 +533,7 @@ moe_status moe_forward(moe_handle* h, const void* x, int32_t T, void* y, int32_t
     h->prof_mark(kKGateUp, s);
     if (alt) {
       a.bn_select = h->bn_choice;
-      a.bn_self = kBnLarge;
-      MOE_TRY_CUDA(launch_gemm_gateup(h->tm_w13, h->tm_xp, tm_x, a, kBnLarge, h->num_sms, s));
-      a.bn_self = kBnAlt;
-      MOE_TRY_CUDA(launch_gemm_gateup(h->tm_w13, h->tm_xp, tm_x, a, kBnAlt, h->num_sms, s));
+      MOE_TRY_CUDA(launch_gemm_gateup_dual(h->tm_w13, h->tm_xp, tm_x, a, h->num_sms, s));
     } else {
       MOE_TRY_CUDA(launch_gemm_gateup(h->tm_w13, h->tm_xp, tm_x, a, bn_gu, h->num_sms, s));
     }
@@ -557,10 +554,7 @@ moe_status moe_forward(moe_handle* h, const void* x, int32_t T, void* y, int32_t
     h->prof_mark(kKDown, s);
     if (alt) {
       d.bn_select = h->bn_choice;
-      d.bn_self = kBnLarge;
-      MOE_TRY_CUDA(launch_gemm_down(h->tm_w2w, h->tm_h, d, kBnLarge, h->num_sms, s, true));
-      d.bn_self = kBnAlt;
-      MOE_TRY_CUDA(launch_gemm_down(h->tm_w2w, h->tm_h, d, kBnAlt, h->num_sms, s, true));
+      MOE_TRY_CUDA(launch_gemm_down_wide_dual(h->tm_w2w, h->tm_h, d, h->num_sms, s));
     } else {
       MOE_TRY_CUDA(launch_gemm_down(wide ? h->tm_w2w : h->tm_w2, h->tm_h, d, bn_dn, h->num_sms, s, wide));
     }
@@ -621,6 +615,8 @@ moe_status moe_forward(moe_handle* h, const void* x, int32_t T, void* y, int32_t
         const int nt = a.dense_m_tiles * a.dense_k_splits;
         h->prof_mark(kKGateUp, s);
         MOE_TRY_CUDA(launch_gemm_gateup(h->tm_w13sh, tm_x, tm_x, a, 32, nt < h->num_sms ? nt : h->num_sms, s));
+        h->prof_done(s);
+        h->prof_mark(kKSwigluReduce, s);
         MOE_TRY_CUDA(launch_swiglu_reduce(a.out ? static_cast<float*>(a.out) : nullptr, h->ks_gu, T, I,
                                           c.swiglu_limit,
                                           static_cast<__nv_bfloat16*>(h->h) + (static_cast<size_t>(T) * k +

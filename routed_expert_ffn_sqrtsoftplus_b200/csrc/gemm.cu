@@ -148,13 +148,9 @@ __device__ __forceinline__ void drain_ring(uint64_t* full, int depth, long issue
 }
 
 template <bool kGateUp, int kAMmas, int BN, int kStages>
-__global__ void __launch_bounds__(kThreads, 1)
-    grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                        const __grid_constant__ CUtensorMap tmBsh, const GemmArgs args) {
+__device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensorMap* tmB, const CUtensorMap* tmBsh,
+                                          const GemmArgs& args, uint8_t* smem_raw) {
   using C = Cfg<kGateUp, kAMmas, BN, kStages>;
-  // the tile lists were built for the other token-tile width: nothing to do
-  if (args.bn_select != nullptr && *args.bn_select != args.bn_self) return;
-  extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
   uint8_t* sB = smem + kStages * C::kABytes;
@@ -184,9 +180,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     fence_mbarrier_init();
   }
   if (warp == kWarpTma && lane == 0) {
-    tma_prefetch_desc(&tmA);
-    tma_prefetch_desc(&tmB);
-    if (kGateUp) tma_prefetch_desc(&tmBsh);
+    tma_prefetch_desc(tmA);
+    tma_prefetch_desc(tmB);
+    if (kGateUp) tma_prefetch_desc(tmBsh);
   }
   if (warp == kWarpMma) {
     tmem_alloc(tmem_base_smem, C::kTmemCols);
@@ -209,7 +205,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       for (int t = tfirst; ok && t < ntiles && !*abort_flag; t += gridDim.x) {
         const Tile tl = load_tile<BN>(args, t);
-        const CUtensorMap* mb = (kGateUp && tl.group >= args.n_routed) ? &tmBsh : &tmB;
+        const CUtensorMap* mb = (kGateUp && tl.group >= args.n_routed) ? tmBsh : tmB;
         const int a_row = (tl.group - args.group_base) * args.a_rows_per_group + tl.m_tile * C::kARows;
         const int nb = (tl.nrows + kBBoxRows - 1) / kBBoxRows;
         const uint32_t bytes = C::kABytes + nb * kBBoxBytes;
@@ -220,7 +216,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           mbar_arrive_expect_tx(&full[stage], bytes);
           const int kx = (tl.kb0 + kb) * kBK;
-          tma_load_2d(sA + stage * C::kABytes, &tmA, &full[stage], kx, a_row, kCacheEvictFirst);
+          tma_load_2d(sA + stage * C::kABytes, tmA, &full[stage], kx, a_row, kCacheEvictFirst);
           for (int j = 0; j < nb; ++j)
             tma_load_2d(sB + stage * C::kBBytes + j * kBBoxBytes, mb, &full[stage], kx, tl.b_row0 + j * kBBoxRows,
                         kCacheEvictLast);
@@ -376,10 +372,45 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 template <bool kGateUp, int kAMmas, int BN, int kStages>
+__global__ void __launch_bounds__(kThreads, 1)
+    grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                        const __grid_constant__ CUtensorMap tmBsh, const GemmArgs args) {
+  extern __shared__ uint8_t smem_raw[];
+  gemm_body<kGateUp, kAMmas, BN, kStages>(&tmA, &tmB, &tmBsh, args, smem_raw);
+}
+
+// Two token-tile widths in one launch: the width the permutation kernel chose
+// (*args.bn_select, written before this grid starts) selects the body.
+template <bool kGateUp, int kAMmas, int BN1, int S1, int BN2, int S2>
+__global__ void __launch_bounds__(kThreads, 1)
+    grouped_gemm_dual_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                             const __grid_constant__ CUtensorMap tmBsh, const GemmArgs args) {
+  extern __shared__ uint8_t smem_raw[];
+  if (*args.bn_select == BN2)
+    gemm_body<kGateUp, kAMmas, BN2, S2>(&tmA, &tmB, &tmBsh, args, smem_raw);
+  else
+    gemm_body<kGateUp, kAMmas, BN1, S1>(&tmA, &tmB, &tmBsh, args, smem_raw);
+}
+
+template <bool kGateUp, int kAMmas, int BN, int kStages>
 cudaError_t set_attr() {
   return cudaFuncSetAttribute(grouped_gemm_kernel<kGateUp, kAMmas, BN, kStages>,
                               cudaFuncAttributeMaxDynamicSharedMemorySize,
                               Cfg<kGateUp, kAMmas, BN, kStages>::kSmemBytes);
+}
+
+template <bool kGateUp, int kAMmas, int BN1, int S1, int BN2, int S2>
+constexpr int dual_smem() {
+  return Cfg<kGateUp, kAMmas, BN1, S1>::kSmemBytes > Cfg<kGateUp, kAMmas, BN2, S2>::kSmemBytes
+             ? Cfg<kGateUp, kAMmas, BN1, S1>::kSmemBytes
+             : Cfg<kGateUp, kAMmas, BN2, S2>::kSmemBytes;
+}
+
+template <bool kGateUp, int kAMmas, int BN1, int S1, int BN2, int S2>
+cudaError_t set_attr_dual() {
+  return cudaFuncSetAttribute(grouped_gemm_dual_kernel<kGateUp, kAMmas, BN1, S1, BN2, S2>,
+                              cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              dual_smem<kGateUp, kAMmas, BN1, S1, BN2, S2>());
 }
 
 template <bool kGateUp, int kAMmas, int BN, int kStages>
@@ -387,6 +418,15 @@ cudaError_t launch(const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtenso
                    int grid, cudaStream_t s) {
   grouped_gemm_kernel<kGateUp, kAMmas, BN, kStages>
       <<<grid, kThreads, Cfg<kGateUp, kAMmas, BN, kStages>::kSmemBytes, s>>>(tmA, tmB, tmBsh, a);
+  return cudaGetLastError();
+}
+
+template <bool kGateUp, int kAMmas, int BN1, int S1, int BN2, int S2>
+cudaError_t launch_dual(const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap& tmBsh,
+                        const GemmArgs& a, int grid, cudaStream_t s) {
+  if (a.bn_select == nullptr) return cudaErrorInvalidValue;
+  grouped_gemm_dual_kernel<kGateUp, kAMmas, BN1, S1, BN2, S2>
+      <<<grid, kThreads, dual_smem<kGateUp, kAMmas, BN1, S1, BN2, S2>(), s>>>(tmA, tmB, tmBsh, a);
   return cudaGetLastError();
 }
 
@@ -421,10 +461,11 @@ constexpr int ring_fit(int a_bytes, int b_bytes) {
 #define MOE_DN_SMALL false, 1, 32, MOE_STAGES_DN_SMALL
 #define MOE_DN_LARGE false, 1, kBnLarge, MOE_STAGES_DN_LARGE
 #define MOE_DN_WIDE false, 2, kBnLarge, MOE_STAGES_DN_WIDE
-// the device-chosen alternative width (as many stages as fit)
+// the device-chosen alternative width (as many stages as fit), paired with the
+// large width in one dual-width kernel
 constexpr int kBnAltT = kBnAlt > 0 ? kBnAlt : 64;  // an unused placeholder when disabled
-#define MOE_GU_ALT true, 2, kBnAltT, ring_fit(256 * 128, kBnAltT * 128)
-#define MOE_DN_WIDE_ALT false, 2, kBnAltT, ring_fit(256 * 128, kBnAltT * 128)
+#define MOE_GU_DUAL true, 2, kBnLarge, MOE_STAGES_GU_LARGE, kBnAltT, ring_fit(256 * 128, kBnAltT * 128)
+#define MOE_DN_WIDE_DUAL false, 2, kBnLarge, MOE_STAGES_DN_WIDE, kBnAltT, ring_fit(256 * 128, kBnAltT * 128)
 
 }  // namespace
 
@@ -437,8 +478,8 @@ cudaError_t gemm_set_attributes() {
   if ((e = set_attr<MOE_DN_LARGE>()) != cudaSuccess) return e;
   if ((e = set_attr<MOE_DN_WIDE>()) != cudaSuccess) return e;
   if constexpr (kBnAlt > 0) {
-    if ((e = set_attr<MOE_GU_ALT>()) != cudaSuccess) return e;
-    if ((e = set_attr<MOE_DN_WIDE_ALT>()) != cudaSuccess) return e;
+    if ((e = set_attr_dual<MOE_GU_DUAL>()) != cudaSuccess) return e;
+    if ((e = set_attr_dual<MOE_DN_WIDE_DUAL>()) != cudaSuccess) return e;
   }
   return cudaSuccess;
 }
@@ -448,8 +489,6 @@ cudaError_t launch_gemm_gateup(const CUtensorMap& tmA, const CUtensorMap& tmB, c
   if (bn == 32) return launch<MOE_GU_SMALL>(tmA, tmB, tmBsh, a, grid, s);
   if (bn == 128) return launch<MOE_GU_MID>(tmA, tmB, tmBsh, a, grid, s);
   if (bn == kBnLarge) return launch<MOE_GU_LARGE>(tmA, tmB, tmBsh, a, grid, s);
-  if constexpr (kBnAlt > 0)
-    if (bn == kBnAlt) return launch<MOE_GU_ALT>(tmA, tmB, tmBsh, a, grid, s);
   return cudaErrorInvalidValue;
 }
 
@@ -457,12 +496,26 @@ cudaError_t launch_gemm_down(const CUtensorMap& tmA, const CUtensorMap& tmB, con
                              cudaStream_t s, bool wide) {
   if (wide) {
     if (bn == kBnLarge) return launch<MOE_DN_WIDE>(tmA, tmB, tmB, a, grid, s);
-    if constexpr (kBnAlt > 0)
-      if (bn == kBnAlt) return launch<MOE_DN_WIDE_ALT>(tmA, tmB, tmB, a, grid, s);
     return cudaErrorInvalidValue;
   }
   if (bn == 32) return launch<MOE_DN_SMALL>(tmA, tmB, tmB, a, grid, s);
   if (bn == kBnLarge) return launch<MOE_DN_LARGE>(tmA, tmB, tmB, a, grid, s);
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace moe
+
+namespace moe {
+
+cudaError_t launch_gemm_gateup_dual(const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap& tmBsh,
+                                    const GemmArgs& a, int grid, cudaStream_t s) {
+  if constexpr (kBnAlt > 0) return launch_dual<MOE_GU_DUAL>(tmA, tmB, tmBsh, a, grid, s);
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_gemm_down_wide_dual(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmArgs& a, int grid,
+                                       cudaStream_t s) {
+  if constexpr (kBnAlt > 0) return launch_dual<MOE_DN_WIDE_DUAL>(tmA, tmB, tmB, a, grid, s);
   return cudaErrorInvalidValue;
 }
 

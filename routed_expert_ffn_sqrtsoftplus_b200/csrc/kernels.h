@@ -33,8 +33,7 @@ struct GemmArgs {
   int raw_gateup;               // gate/up: store fp32 G | U (ld = out_ld, U at + I) instead of h
   int* status;                  // device status word
   unsigned long long timeout_ns;
-  const int* bn_select;         // grouped mode: token-tile width chosen on the device (nullptr = always run)
-  int bn_self;                  // this kernel's width: it returns at once unless *bn_select == bn_self
+  const int* bn_select;         // dual-width launch: the token-tile width the permutation chose
 };
 
 // Kernel kinds for profiling (order = moe_kernel_name()).
@@ -52,6 +51,7 @@ enum KernelKind {
   kKQuantX,
   kKGateUpMx,
   kKDownMx,
+  kKSwigluReduce,
   kKNumKinds
 };
 
@@ -125,6 +125,12 @@ cudaError_t launch_gemm_gateup(const CUtensorMap& tmA, const CUtensorMap& tmB, c
 // the tile list's m tiles are then H / 256.
 cudaError_t launch_gemm_down(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmArgs& a, int bn, int grid,
                              cudaStream_t s, bool wide = false);
+// One launch for both many-token widths (kBnLarge and kBnAlt): a.bn_select holds
+// the permutation kernel's choice; wide W2 tiles for the down GEMM.
+cudaError_t launch_gemm_gateup_dual(const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap& tmBsh,
+                                    const GemmArgs& a, int grid, cudaStream_t s);
+cudaError_t launch_gemm_down_wide_dual(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmArgs& a, int grid,
+                                       cudaStream_t s);
 cudaError_t gemm_set_attributes();
 
 // ---- MX (MXFP4 routed experts)
