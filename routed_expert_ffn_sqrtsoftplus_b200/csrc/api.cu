@@ -132,7 +132,7 @@ struct moe_handle {
   int32_t* ntile_base_dn = nullptr;
   int* bad = nullptr;
   int64_t max_ntiles_r = 0;
-  CUtensorMap tm_w13q, tm_w2q, tm_xq, tm_hq, tm_w13sh, tm_w2sh;
+  CUtensorMap tm_w13q, tm_w2q, tm_w2qw, tm_xq, tm_hq, tm_w13sh, tm_w2sh, tm_w2shw;
   // shared experts alone (MXFP4 layers, few tokens): split-K partial sums
   float* sh_parts_gu = nullptr;  // [S][ks_gu][T][2I]
   float* sh_parts_dn = nullptr;  // [S][ks_dn][T][H]
@@ -371,9 +371,15 @@ moe_status moe_create(const moe_config* cfg, const moe_weights* w, moe_stream_t 
       err |= cudaMemcpyAsync(h->w2sh, w->sh_w2, S * H * I * 2, cudaMemcpyDeviceToDevice, s) != cudaSuccess;
       err |= !make_tmap_bf16(&h->tm_w13sh, h->w13sh, S * 2 * I, H, 256);
       err |= !make_tmap_bf16(&h->tm_w2sh, h->w2sh, S * H, I, 128);
+      // 256-row W2 boxes: the shared groups share the down tile list with the
+      // routed ones, whose tiles are 256 rows of W2 when H % 256 == 0
+      if (H % 256 == 0) err |= !make_tmap_bf16(&h->tm_w2shw, h->w2sh, S * H, I, 256);
     }
     err |= !make_tmap(&h->tm_w13q, h->w13q, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, E * 2 * I, H, H / 2, 128, 256);
     err |= !make_tmap(&h->tm_w2q, h->w2q, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, E * H, I, I / 2, 128, 128);
+    h->wide_ok = H % 256 == 0;
+    if (h->wide_ok)
+      err |= !make_tmap(&h->tm_w2qw, h->w2q, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, E * H, I, I / 2, 128, 256);
     err |= !make_tmap(&h->tm_xq, h->xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, Tm * k, H, H, 128, 32);
     err |= !make_tmap(&h->tm_hq, h->hq, CU_TENSOR_MAP_DATA_TYPE_UINT8, Tm * k, I, I, 128, 32);
   }
@@ -489,7 +495,8 @@ moe_status moe_forward(moe_handle* h, const void* x, int32_t T, void* y, int32_t
   sa.tiles_dn = h->tiles_dn;
   sa.ntiles = h->ntiles;
   sa.m_tiles_gu = h->m_tiles_gu;
-  sa.m_tiles_dn = wide ? H / 256 : h->m_tiles_dn;
+  const bool wide_mx = h->mx && h->wide_ok;             // 256-row MXFP4 W2 tiles
+  sa.m_tiles_dn = (wide || wide_mx) ? H / 256 : h->m_tiles_dn;
   sa.bn_gu_r = h->mx ? bn_mx : bn_gu;
   sa.bn_dn_r = h->mx ? bn_mx : bn_dn;
   sa.bn_gu_s = bn_gu;
@@ -660,7 +667,7 @@ moe_status moe_forward(moe_handle* h, const void* x, int32_t T, void* y, int32_t
     d.status = h->status;
     d.timeout_ns = h->timeout_ns;
     h->prof_mark(kKDownMx, s);
-    MOE_TRY_CUDA(launch_gemm_mx_down(h->tm_w2q, h->tm_hq, d, bn_mx, h->num_sms, s));
+    MOE_TRY_CUDA(launch_gemm_mx_down(wide_mx ? h->tm_w2qw : h->tm_w2q, h->tm_hq, d, bn_mx, h->num_sms, s, wide_mx));
     h->prof_done(s);
     // 5b. shared experts' down in BF16 (split K for few tokens; the combine sums the slices)
     if (sh_split) {
@@ -700,7 +707,7 @@ moe_status moe_forward(moe_handle* h, const void* x, int32_t T, void* y, int32_t
       a.status = h->status;
       a.timeout_ns = h->timeout_ns;
       h->prof_mark(kKDown, s);
-      MOE_TRY_CUDA(launch_gemm_down(h->tm_w2sh, h->tm_h, a, bn_dn, h->num_sms, s));
+      MOE_TRY_CUDA(launch_gemm_down(wide_mx ? h->tm_w2shw : h->tm_w2sh, h->tm_h, a, bn_dn, h->num_sms, s, wide_mx));
       h->prof_done(s);
     }
   }

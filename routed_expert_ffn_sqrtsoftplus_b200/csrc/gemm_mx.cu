@@ -41,21 +41,25 @@ constexpr int pow2_at_least(int v, int lo) {
   return p;
 }
 
-template <bool kGateUp, int BN, int kStages>
+// kWide (down GEMM): a tile covers 256 rows of W2, two 128-row MMAs sharing the
+// token tile, like the gate/up tile's W1 and W3 halves.
+template <bool kGateUp, bool kWide, int BN, int kStages>
 struct MxCfg {
-  static constexpr int kARows = kGateUp ? 256 : 128;
+  static constexpr bool kTwoA = kGateUp || kWide;       // two 128-row MMAs per K step
+  static constexpr int kARows = kTwoA ? 256 : 128;
   static constexpr int kABytes = kARows * 128;          // unpacked E2M1 in shared memory
   static constexpr int kATx = kARows * 64;              // packed bytes the TMA moves
   static constexpr int kBBytes = BN * 128;
-  static constexpr int kSfaBytes = kGateUp ? 2 * kAtomBytes : kAtomBytes;
+  static constexpr int kSfaBytes = kTwoA ? 2 * kAtomBytes : kAtomBytes;
   static constexpr int kSfBytes = kSfaBytes + kAtomBytes;
-  static constexpr int kAccCols = kGateUp ? 2 * BN : BN;
-  static constexpr int kSfCols = kGateUp ? 12 : 8;       // 4 TMEM columns per atom
+  static constexpr int kAccCols = kTwoA ? 2 * BN : BN;
+  static constexpr int kSfCols = kTwoA ? 12 : 8;         // 4 TMEM columns per atom
   static constexpr int kSfColBase = 2 * kAccCols;
   static constexpr int kTmemCols = pow2_at_least(kSfColBase + kStages * kSfCols, 32);
   static constexpr int kBarrierBytes = 256;
   static constexpr int kSmemBytes = 1024 + kStages * (kABytes + kBBytes + kSfBytes) + kBarrierBytes;
   static_assert(kTmemCols <= 512, "TMEM");
+  static_assert((2 * kStages + 5) * 8 + 8 <= kBarrierBytes, "barriers");
   static_assert(BN % kBBoxRows == 0 && BN <= 128, "BN");
   static_assert(kSmemBytes <= 227 * 1024, "shared memory");
 };
@@ -93,11 +97,11 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, co
   }
 }
 
-template <bool kGateUp, int BN, int kStages>
+template <bool kGateUp, bool kWide, int BN, int kStages>
 __global__ void __launch_bounds__(kThreads, 1)
     grouped_gemm_mx_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                            const MxGemmArgs args) {
-  using C = MxCfg<kGateUp, BN, kStages>;
+  using C = MxCfg<kGateUp, kWide, BN, kStages>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
@@ -155,8 +159,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int a_row = tl.group * args.a_rows_per_group + tl.m_tile * C::kARows;
         const int nb = (tl.nrows + kBBoxRows - 1) / kBBoxRows;
         const uint32_t bytes = C::kATx + nb * kBBoxBytes + C::kSfBytes;
+        // W1|W3 atoms: [group][m tile][k block][2 x 512 B]; W2 atoms: [group][128-row
+        // tile][k block][512 B] (a wide tile takes 128-row tiles 2m and 2m + 1)
         const uint8_t* sfa_src =
-            args.sfa + (static_cast<size_t>(tl.group) * args.m_tiles + tl.m_tile) * args.num_kb * C::kSfaBytes;
+            kWide ? args.sfa + (static_cast<size_t>(tl.group) * args.m_tiles + 2 * tl.m_tile) * args.num_kb * kAtomBytes
+                  : args.sfa + (static_cast<size_t>(tl.group) * args.m_tiles + tl.m_tile) * args.num_kb * C::kSfaBytes;
         const uint8_t* sfb_src = args.sfb + static_cast<size_t>(tl.ntile) * args.num_kb * kAtomBytes;
         bool ok = true;
         for (int kb = 0; kb < args.num_kb; ++kb) {
@@ -170,8 +177,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             tma_load_2d(sB + stage * C::kBBytes + j * kBBoxBytes, &tmB, &full[stage], kb * kBK,
                         tl.row0 + j * kBBoxRows, kCacheEvictLast);
           uint8_t* sf = sSF + stage * C::kSfBytes;
-          bulk_load(sf, sfa_src + static_cast<size_t>(kb) * C::kSfaBytes, C::kSfaBytes, &full[stage],
-                    kCacheEvictFirst);
+          if (kWide) {
+            bulk_load(sf, sfa_src + static_cast<size_t>(kb) * kAtomBytes, kAtomBytes, &full[stage], kCacheEvictFirst);
+            bulk_load(sf + kAtomBytes, sfa_src + static_cast<size_t>(args.num_kb + kb) * kAtomBytes, kAtomBytes,
+                      &full[stage], kCacheEvictFirst);
+          } else {
+            bulk_load(sf, sfa_src + static_cast<size_t>(kb) * C::kSfaBytes, C::kSfaBytes, &full[stage],
+                      kCacheEvictFirst);
+          }
           bulk_load(sf + C::kSfaBytes, sfb_src + static_cast<size_t>(kb) * kAtomBytes, kAtomBytes, &full[stage],
                     kCacheEvictLast);
           ++issued;
@@ -218,8 +231,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t sf_cols = tmem_base + C::kSfColBase + stage * C::kSfCols;
           // scale factors of this stage -> TMEM (replicated to all four lane quarters)
           tmem_cp_32x128b_x4(sf_cols, sdesc_plain(sf_addr));
-          if (kGateUp) tmem_cp_32x128b_x4(sf_cols + 4, sdesc_plain(sf_addr + kAtomBytes));
-          const uint32_t sfb_col = sf_cols + (kGateUp ? 8 : 4);
+          if (C::kTwoA) tmem_cp_32x128b_x4(sf_cols + 4, sdesc_plain(sf_addr + kAtomBytes));
+          const uint32_t sfb_col = sf_cols + (C::kTwoA ? 8 : 4);
           tmem_cp_32x128b_x4(sfb_col, sdesc_plain(sf_addr + C::kSfaBytes));
 #pragma unroll
           for (uint32_t k = 0; k < kBK / 32; ++k) {
@@ -228,7 +241,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t accum = (kb | k) != 0;
             umma_mx(d, sdesc_sw128(a_addr + k * 32), bdesc, idesc, sf_cols | (k << 30), sfb_col | (k << 30),
                     accum);
-            if (kGateUp)
+            if (C::kTwoA)
               umma_mx(d + BN, sdesc_sw128(a_addr + 128 * 128 + k * 32), bdesc, idesc, (sf_cols + 4) | (k << 30),
                       sfb_col | (k << 30), accum);
           }
@@ -265,7 +278,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok) break;
       tc_fence_after();
       const uint32_t tb = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * C::kAccCols;
-      const int m = tl.m_tile * 128 + q * 32 + lane;
+      const int m = tl.m_tile * (kWide ? 256 : 128) + q * 32 + lane;
       const bool rows_ok = tl.row0 >= 0 && tl.row0 + tl.nrows <= args.out_rows;
       if (!rows_ok && lane == 0 && q == 0) report_status(args.status, kStatusDevice);
       const bool m_ok = m < args.m_limit && rows_ok;
@@ -315,6 +328,19 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int n = c0 + j;
             if (n < tl.nrows && m_ok) out[static_cast<size_t>(tl.row0 + n) * args.out_ld + m] = __uint_as_float(g[j]);
           }
+          if constexpr (kWide) {
+            // the second 128 rows of W2 (output columns m + 128)
+            uint32_t g2[16];
+            tmem_ld16(tb + BN + c0, g2);
+            tmem_ld_wait();
+            const bool m2_ok = m + 128 < args.m_limit && rows_ok;
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+              const int n = c0 + j;
+              if (n < tl.nrows && m2_ok)
+                out[static_cast<size_t>(tl.row0 + n) * args.out_ld + m + 128] = __uint_as_float(g2[j]);
+            }
+          }
         }
       }
       tc_fence_before();
@@ -335,62 +361,74 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <bool kGateUp, int BN, int kStages>
+template <bool kGateUp, bool kWide, int BN, int kStages>
 cudaError_t set_attr() {
-  return cudaFuncSetAttribute(grouped_gemm_mx_kernel<kGateUp, BN, kStages>,
-                              cudaFuncAttributeMaxDynamicSharedMemorySize, MxCfg<kGateUp, BN, kStages>::kSmemBytes);
+  return cudaFuncSetAttribute(grouped_gemm_mx_kernel<kGateUp, kWide, BN, kStages>,
+                              cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              MxCfg<kGateUp, kWide, BN, kStages>::kSmemBytes);
 }
 
-template <bool kGateUp, int BN, int kStages>
+template <bool kGateUp, bool kWide, int BN, int kStages>
 cudaError_t launch(const CUtensorMap& tmA, const CUtensorMap& tmB, const MxGemmArgs& a, int grid, cudaStream_t s) {
-  grouped_gemm_mx_kernel<kGateUp, BN, kStages>
-      <<<grid, kThreads, MxCfg<kGateUp, BN, kStages>::kSmemBytes, s>>>(tmA, tmB, a);
+  grouped_gemm_mx_kernel<kGateUp, kWide, BN, kStages>
+      <<<grid, kThreads, MxCfg<kGateUp, kWide, BN, kStages>::kSmemBytes, s>>>(tmA, tmB, a);
   return cudaGetLastError();
 }
 
-constexpr int kGu32Stages = 6;   // 6 * (32 + 4 + 1.5) KB
-constexpr int kGu64Stages = 5;   // 5 * (32 + 8 + 1.5) KB
-constexpr int kDn32Stages = 10;  // 10 * (16 + 4 + 1) KB
-constexpr int kDn64Stages = 8;   // 8 * (16 + 8 + 1) KB
-// other widths: as many stages as fit in 227 KB
+// Ring depths: as many stages as fit in 227 KB.
 constexpr int mx_ring_fit(int a_bytes, int b_bytes, int sf_bytes) {
   return (227 * 1024 - 1024 - 256) / (a_bytes + b_bytes + sf_bytes);
 }
-constexpr int kGuLStages = mx_ring_fit(256 * 128, kBnMxLarge * 128, 3 * kAtomBytes);
-constexpr int kDnLStages = mx_ring_fit(128 * 128, kBnMxLarge * 128, 2 * kAtomBytes);
+template <int BN>
+constexpr int kTwoAStages = mx_ring_fit(256 * 128, BN * 128, 3 * kAtomBytes);  // 32: 6, 64: 5, 96: 4
+template <int BN>
+constexpr int kOneAStages = mx_ring_fit(128 * 128, BN * 128, 2 * kAtomBytes);  // 32: 10, 64: 9, 96: 7
 constexpr bool kExtraWidth = kBnMxLarge != 32 && kBnMxLarge != 64;
+
+template <bool kGateUp, bool kWide>
+cudaError_t set_attrs() {
+  constexpr bool two = kGateUp || kWide;
+  cudaError_t e;
+  if ((e = set_attr<kGateUp, kWide, 32, two ? kTwoAStages<32> : kOneAStages<32>>()) != cudaSuccess) return e;
+  if ((e = set_attr<kGateUp, kWide, 64, two ? kTwoAStages<64> : kOneAStages<64>>()) != cudaSuccess) return e;
+  if constexpr (kExtraWidth)
+    if ((e = set_attr<kGateUp, kWide, kBnMxLarge, two ? kTwoAStages<kBnMxLarge> : kOneAStages<kBnMxLarge>>()) !=
+        cudaSuccess)
+      return e;
+  return cudaSuccess;
+}
+
+template <bool kGateUp, bool kWide>
+cudaError_t launch_any(const CUtensorMap& tmA, const CUtensorMap& tmB, const MxGemmArgs& a, int bn, int grid,
+                       cudaStream_t s) {
+  constexpr bool two = kGateUp || kWide;
+  if (bn == 32) return launch<kGateUp, kWide, 32, two ? kTwoAStages<32> : kOneAStages<32>>(tmA, tmB, a, grid, s);
+  if (bn == 64) return launch<kGateUp, kWide, 64, two ? kTwoAStages<64> : kOneAStages<64>>(tmA, tmB, a, grid, s);
+  if constexpr (kExtraWidth)
+    if (bn == kBnMxLarge)
+      return launch<kGateUp, kWide, kBnMxLarge, two ? kTwoAStages<kBnMxLarge> : kOneAStages<kBnMxLarge>>(
+          tmA, tmB, a, grid, s);
+  return cudaErrorInvalidValue;
+}
 
 }  // namespace
 
 cudaError_t gemm_mx_set_attributes() {
   cudaError_t e;
-  if ((e = set_attr<true, 32, kGu32Stages>()) != cudaSuccess) return e;
-  if ((e = set_attr<true, 64, kGu64Stages>()) != cudaSuccess) return e;
-  if ((e = set_attr<false, 32, kDn32Stages>()) != cudaSuccess) return e;
-  if ((e = set_attr<false, 64, kDn64Stages>()) != cudaSuccess) return e;
-  if constexpr (kExtraWidth) {
-    if ((e = set_attr<true, kBnMxLarge, kGuLStages>()) != cudaSuccess) return e;
-    if ((e = set_attr<false, kBnMxLarge, kDnLStages>()) != cudaSuccess) return e;
-  }
+  if ((e = set_attrs<true, false>()) != cudaSuccess) return e;
+  if ((e = set_attrs<false, false>()) != cudaSuccess) return e;
+  if ((e = set_attrs<false, true>()) != cudaSuccess) return e;
   return cudaSuccess;
 }
 
 cudaError_t launch_gemm_mx_gateup(const CUtensorMap& tmA, const CUtensorMap& tmB, const MxGemmArgs& a, int bn,
                                   int grid, cudaStream_t s) {
-  if (bn == 32) return launch<true, 32, kGu32Stages>(tmA, tmB, a, grid, s);
-  if (bn == 64) return launch<true, 64, kGu64Stages>(tmA, tmB, a, grid, s);
-  if constexpr (kExtraWidth)
-    if (bn == kBnMxLarge) return launch<true, kBnMxLarge, kGuLStages>(tmA, tmB, a, grid, s);
-  return cudaErrorInvalidValue;
+  return launch_any<true, false>(tmA, tmB, a, bn, grid, s);
 }
 
 cudaError_t launch_gemm_mx_down(const CUtensorMap& tmA, const CUtensorMap& tmB, const MxGemmArgs& a, int bn,
-                                int grid, cudaStream_t s) {
-  if (bn == 32) return launch<false, 32, kDn32Stages>(tmA, tmB, a, grid, s);
-  if (bn == 64) return launch<false, 64, kDn64Stages>(tmA, tmB, a, grid, s);
-  if constexpr (kExtraWidth)
-    if (bn == kBnMxLarge) return launch<false, kBnMxLarge, kDnLStages>(tmA, tmB, a, grid, s);
-  return cudaErrorInvalidValue;
+                                int grid, cudaStream_t s, bool wide) {
+  return wide ? launch_any<false, true>(tmA, tmB, a, bn, grid, s) : launch_any<false, false>(tmA, tmB, a, bn, grid, s);
 }
 
 }  // namespace moe

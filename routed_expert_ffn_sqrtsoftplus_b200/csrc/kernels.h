@@ -166,8 +166,9 @@ struct MxGemmArgs {
 cudaError_t gemm_mx_set_attributes();
 cudaError_t launch_gemm_mx_gateup(const CUtensorMap& tmA, const CUtensorMap& tmB, const MxGemmArgs& a, int bn,
                                   int grid, cudaStream_t s);
+// wide: tiles of 256 W2 rows (two 128-row MMAs per K step); the tile list's m tiles are H / 256
 cudaError_t launch_gemm_mx_down(const CUtensorMap& tmA, const CUtensorMap& tmB, const MxGemmArgs& a, int bn,
-                                int grid, cudaStream_t s);
+                                int grid, cudaStream_t s, bool wide = false);
 // x rows of the routed slots -> MXFP8: xq[row] = E4M3 codes of x[perm[row] / k], scale
 // atoms by gate/up token tile.
 cudaError_t launch_quant_gather_mx(const void* x, const int32_t* perm, const int32_t* idx, const int32_t* off,
