@@ -429,6 +429,7 @@ moe_status moe_forward(moe_handle* h, const void* x, int32_t T, void* y, int32_t
   const int bn_gu = small ? 32 : (large ? kBnLarge : 128);   // BF16 token tiles
   const int bn_dn = small ? 32 : kBnLarge;
   const bool wide = large && h->wide_ok && !h->mx;      // 256-row W2 tiles
+  const bool wide_small = small && h->wide_ok && !h->mx;  // 256-row W2 tiles, 32-token tiles
   // many tokens per expert, BF16: the permutation picks kBnAlt-row tiles (a deeper
   // ring, one tile per expert) when no routed expert has more rows than that, else
   // kBnLarge; one dual-width launch per GEMM runs the chosen body
@@ -496,7 +497,7 @@ moe_status moe_forward(moe_handle* h, const void* x, int32_t T, void* y, int32_t
   sa.ntiles = h->ntiles;
   sa.m_tiles_gu = h->m_tiles_gu;
   const bool wide_mx = h->mx && h->wide_ok;             // 256-row MXFP4 W2 tiles
-  sa.m_tiles_dn = (wide || wide_mx) ? H / 256 : h->m_tiles_dn;
+  sa.m_tiles_dn = (wide || wide_small || wide_mx) ? H / 256 : h->m_tiles_dn;
   sa.bn_gu_r = h->mx ? bn_mx : bn_gu;
   sa.bn_dn_r = h->mx ? bn_mx : bn_dn;
   sa.bn_gu_s = bn_gu;
@@ -563,7 +564,8 @@ moe_status moe_forward(moe_handle* h, const void* x, int32_t T, void* y, int32_t
       d.bn_select = h->bn_choice;
       MOE_TRY_CUDA(launch_gemm_down_wide_dual(h->tm_w2w, h->tm_h, d, h->num_sms, s));
     } else {
-      MOE_TRY_CUDA(launch_gemm_down(wide ? h->tm_w2w : h->tm_w2, h->tm_h, d, bn_dn, h->num_sms, s, wide));
+      MOE_TRY_CUDA(launch_gemm_down(wide || wide_small ? h->tm_w2w : h->tm_w2, h->tm_h, d, bn_dn, h->num_sms, s,
+                                    wide || wide_small));
     }
     h->prof_done(s);
   } else {

@@ -432,7 +432,7 @@ cudaError_t launch_dual(const CUtensorMap& tmA, const CUtensorMap& tmB, const CU
 
 // Ring depths: as many stages of (A box + B boxes) as fit in 227 KB, unless set.
 //   gate/up  BN 32: 6 x (32 + 4) KB   BN 128: 4 x (32 + 16) KB
-//   down     BN 32: 10 x (16 + 4) KB
+//   down     BN 32: 10 x (16 + 4) KB, wide (256 W2 rows) 6 x (32 + 4) KB
 //   large    BN 256: 3 (gate/up, wide down) or 4 (down); BN 192: 4 or 5
 constexpr int ring_fit(int a_bytes, int b_bytes) {
   return (227 * 1024 - 1024 - 512) / (a_bytes + b_bytes);
@@ -461,6 +461,7 @@ constexpr int ring_fit(int a_bytes, int b_bytes) {
 #define MOE_DN_SMALL false, 1, 32, MOE_STAGES_DN_SMALL
 #define MOE_DN_LARGE false, 1, kBnLarge, MOE_STAGES_DN_LARGE
 #define MOE_DN_WIDE false, 2, kBnLarge, MOE_STAGES_DN_WIDE
+#define MOE_DN_WIDE_SMALL false, 2, 32, ring_fit(256 * 128, 32 * 128)
 // the device-chosen alternative width (as many stages as fit), paired with the
 // large width in one dual-width kernel
 constexpr int kBnAltT = kBnAlt > 0 ? kBnAlt : 64;  // an unused placeholder when disabled
@@ -477,6 +478,7 @@ cudaError_t gemm_set_attributes() {
   if ((e = set_attr<MOE_DN_SMALL>()) != cudaSuccess) return e;
   if ((e = set_attr<MOE_DN_LARGE>()) != cudaSuccess) return e;
   if ((e = set_attr<MOE_DN_WIDE>()) != cudaSuccess) return e;
+  if ((e = set_attr<MOE_DN_WIDE_SMALL>()) != cudaSuccess) return e;
   if constexpr (kBnAlt > 0) {
     if ((e = set_attr_dual<MOE_GU_DUAL>()) != cudaSuccess) return e;
     if ((e = set_attr_dual<MOE_DN_WIDE_DUAL>()) != cudaSuccess) return e;
@@ -496,6 +498,7 @@ cudaError_t launch_gemm_down(const CUtensorMap& tmA, const CUtensorMap& tmB, con
                              cudaStream_t s, bool wide) {
   if (wide) {
     if (bn == kBnLarge) return launch<MOE_DN_WIDE>(tmA, tmB, tmB, a, grid, s);
+    if (bn == 32) return launch<MOE_DN_WIDE_SMALL>(tmA, tmB, tmB, a, grid, s);
     return cudaErrorInvalidValue;
   }
   if (bn == 32) return launch<MOE_DN_SMALL>(tmA, tmB, tmB, a, grid, s);
