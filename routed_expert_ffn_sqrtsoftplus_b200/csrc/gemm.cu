@@ -21,9 +21,11 @@
 // A ring of full/empty mbarriers decouples TMA and MMA (weights and tokens of a
 // stage travel together: separate, differently deep rings for the two measured
 // slower on B200). One or two TMEM accumulator buffers (tmem_full/tmem_empty)
-// let the epilogue of tile i overlap the MMAs of tile i+1 when they fit. Every wait is bounded in time; a wait that runs out
-// records MOE_ERR_TIMEOUT, drains this CTA's in-flight copies and MMAs, frees
-// TMEM and returns.
+// let the epilogue of tile i overlap the MMAs of tile i+1 when they fit.
+// grouped_gemm_dual_kernel holds two token-tile widths (two ring configurations)
+// and runs the one the permutation kernel chose for this batch.
+// Every wait is bounded in time; a wait that runs out records MOE_ERR_TIMEOUT,
+// drains this CTA's in-flight copies and MMAs, frees TMEM and returns.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -433,7 +435,7 @@ cudaError_t launch_dual(const CUtensorMap& tmA, const CUtensorMap& tmB, const CU
 // Ring depths: as many stages of (A box + B boxes) as fit in 227 KB, unless set.
 //   gate/up  BN 32: 6 x (32 + 4) KB   BN 128: 4 x (32 + 16) KB
 //   down     BN 32: 10 x (16 + 4) KB, wide (256 W2 rows) 6 x (32 + 4) KB
-//   large    BN 256: 3 (gate/up, wide down) or 4 (down); BN 192: 4 or 5
+//   large    BN 256: 3 (gate/up, wide down) or 4 (down); BN 192: 4 (gate/up, wide down)
 constexpr int ring_fit(int a_bytes, int b_bytes) {
   return (227 * 1024 - 1024 - 512) / (a_bytes + b_bytes);
 }

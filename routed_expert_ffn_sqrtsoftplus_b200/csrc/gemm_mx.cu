@@ -19,7 +19,9 @@
 //   gate/up: h = silu(min(G, L)) * clamp(U, -L, L), quantised to MXFP8 along the
 //            expert width (a warp owns 32 consecutive rows of I, so the block
 //            amax is a warp reduction) -> E4M3 rows + scale atoms for the down GEMM
-//   down:    fp32 rows, as in the BF16 path
+//   down:    fp32 rows, as in the BF16 path; with kWide a tile covers 256 rows
+//            of W2 (two MMAs sharing the token box, twice the HBM bytes per
+//            ring stage)
 #include "common.cuh"
 #include "kernels.h"
 
