@@ -24,6 +24,10 @@ constexpr float kRefineDelta = 2e-3f;
 constexpr int kTcRouterMinTokens = 256;
 // Token counts up to this use the sliced CUDA-core router and the per-token top-k.
 constexpr int kSmallRouterMaxTokens = 32;
+// Top-k with one CTA per token up to this many tokens (the candidates of a token
+// are re-scored by 8 warps in parallel); one warp per token above (measured on
+// B200: the CTA form halves the time at T=256 and is slower from T=2048 on).
+constexpr int kTopkCtaMaxTokens = 1024;
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
@@ -470,11 +474,18 @@ moe_status moe_forward(moe_handle* h, const void* x, int32_t T, void* y, int32_t
     h->prof_done(s);
   }
   if (T > kSmallRouterMaxTokens) {
-    // scores, top-k with exact refinement of the near-tie candidates, weights (one
-    // warp per token: with thousands of tokens the warps keep every SM busy)
+    // scores, top-k with exact refinement of the near-tie candidates, weights
     h->prof_mark(kKTopk, s);
-    MOE_TRY_CUDA(launch_topk_refine(h->z, x, h->wg, h->bias, T, H, E, k, c.route_scale, kRefineDelta, h->idx,
-                                    h->wts, h->status, s));
+    if (T <= kTopkCtaMaxTokens) {
+      // one CTA per token: the logits (bias included) are a single slice; the
+      // exact re-scoring adds the bias itself
+      MOE_TRY_CUDA(launch_topk_small(h->z, 1, x, h->wg, nullptr, T, H, E, k, c.route_scale, kRefineDelta, h->idx,
+                                     h->wts, nullptr, h->status, s, h->bias));
+    } else {
+      // one warp per token: with thousands of tokens the warps keep every SM busy
+      MOE_TRY_CUDA(launch_topk_refine(h->z, x, h->wg, h->bias, T, H, E, k, c.route_scale, kRefineDelta, h->idx,
+                                      h->wts, h->status, s));
+    }
     h->prof_done(s);
   }
   // 3. permutation and tile lists
