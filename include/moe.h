@@ -122,7 +122,9 @@ typedef struct {
  * weights and the workspace for cfg->max_tokens tokens, and enqueue the weight
  * repack on `stream` (the analogue of the MAX pipeline's one-time routed-expert
  * upload, DeepseekV41Model.load_model). On success *out owns all device memory
- * it allocated. On failure *out is NULL and nothing is leaked.
+ * it allocated. On failure *out is NULL and nothing is leaked. Every weight
+ * pointer must be device (or managed) memory of the current device, else
+ * MOE_ERR_INVALID_ARG before anything is enqueued.
  */
 MOE_API moe_status moe_create(const moe_config* cfg, const moe_weights* w, moe_stream_t stream,
                       moe_handle** out);
@@ -135,7 +137,9 @@ MOE_API moe_status moe_create(const moe_config* cfg, const moe_weights* w, moe_s
  *   topk_w   fp32  [T, k] device or NULL: their weights (sum = route_scale)
  * 0 <= T <= max_tokens; T == 0 enqueues nothing. Allocates nothing and does not
  * synchronise. Calls on one handle must be ordered (one stream at a time): the
- * workspace is shared between calls.
+ * workspace is shared between calls. MOE_ERR_INVALID_ARG, with nothing enqueued,
+ * when the current device is not the handle's or x / y are not device (or
+ * managed) memory of it (a host pointer would fault the kernels).
  */
 MOE_API moe_status moe_forward(moe_handle* h, const void* x, int32_t T, void* y, int32_t* topk_idx,
                        float* topk_w, moe_stream_t stream);
@@ -251,7 +255,9 @@ MOE_API const char* moe_kernel_name(int32_t kind);
  *   topk_idx    int32 [T, top_k] device (output), descending score
  *   topk_w      fp32  [T, top_k] device (output), sum = route_scale
  * hidden % 8 == 0, 1 <= top_k <= min(n_routed, 32), n_routed <= 512. The
- * results equal moe_forward's topk_idx / topk_w for the same inputs.
+ * results equal moe_forward's topk_idx / topk_w for the same inputs. Buffers
+ * that are not device (or managed) memory of the current device give
+ * MOE_ERR_INVALID_ARG with nothing enqueued.
  *
  * The only scratch, the fp32 logits [T, n_routed], lives in a fixed array of
  * MOE_NOALLOC_MAX_LOGITS floats (4 MiB) inside the library; every GPU that

@@ -260,6 +260,15 @@ moe_status moe_create(const moe_config* cfg, const moe_weights* w, moe_stream_t 
       if (p == nullptr || !aligned16(p)) return MOE_ERR_INVALID_ARG;
   }
   if (w->router_bias != nullptr && !aligned16(w->router_bias)) return MOE_ERR_INVALID_ARG;
+  {
+    // the repacking kernels read the weights on the current device
+    int cur = -1;
+    if (cudaGetDevice(&cur) != cudaSuccess) return MOE_ERR_CUDA;
+    const void* all[] = {w->router_w, w->router_bias, w->w1, w->w3, w->w2, w->s1, w->s3, w->s2,
+                         w->sh_w1, w->sh_w3, w->sh_w2};
+    for (const void* p : all)
+      if (p != nullptr && !device_pointer_on(p, cur)) return MOE_ERR_INVALID_ARG;
+  }
   if (get_encode_fn() == nullptr) return MOE_ERR_CUDA;
 
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
@@ -420,6 +429,12 @@ moe_status moe_forward(moe_handle* h, const void* x, int32_t T, void* y, int32_t
     return MOE_OK;
   }
   if (x == nullptr || y == nullptr || !aligned16(x) || !aligned16(y) || x == y) return MOE_ERR_INVALID_ARG;
+  {
+    // kernels launch on the current device and read x / write y directly
+    int cur = -1;
+    if (cudaGetDevice(&cur) != cudaSuccess || cur != h->device) return MOE_ERR_INVALID_ARG;
+    if (!device_pointer_on(x, h->device) || !device_pointer_on(y, h->device)) return MOE_ERR_INVALID_ARG;
+  }
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const moe_config& c = h->cfg;
   const int H = c.hidden, I = c.inter, E = c.n_routed, S = c.n_shared, k = c.top_k;

@@ -7,6 +7,19 @@
 
 namespace moe {
 
+// True when p is device (or managed) memory the kernels of device `dev` may read
+// and write: a host pointer or another GPU's memory handed to a kernel would
+// fault the device, so the entry points reject them before launching anything.
+inline bool device_pointer_on(const void* p, int dev) {
+  cudaPointerAttributes a;
+  if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+    cudaGetLastError();
+    return false;
+  }
+  if (a.type == cudaMemoryTypeManaged) return true;
+  return a.type == cudaMemoryTypeDevice && a.device == dev;
+}
+
 // One GEMM tile: x = group | (m_tile << 16), y = first B row, z = first output row,
 // w = number of valid rows (tokens) in the tile.
 using TileEntry = int4;

@@ -61,6 +61,14 @@ extern "C" moe_status moe_route_noalloc(const void* x, const void* router_w, con
   if (T == 0) return MOE_OK;
   if (x == nullptr || router_w == nullptr || topk_idx == nullptr || topk_w == nullptr) return MOE_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(router_w)) return MOE_ERR_INVALID_ARG;
+  {
+    // every buffer is read or written by the kernels on the current device
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
+    const void* bufs[] = {x, router_w, router_bias, topk_idx, topk_w};
+    for (const void* p : bufs)
+      if (p != nullptr && !moe::device_pointer_on(p, dev)) return MOE_ERR_INVALID_ARG;
+  }
   float* z = nullptr;
   moe_status st = scratch_for_current_device(&z);
   if (st != MOE_OK) return st;

@@ -164,6 +164,28 @@ def test_rejects_too_many_tokens(tiny):
     assert ei.value.status == moe.MOE_ERR_INVALID_ARG
 
 
+def test_forward_rejects_pointers_outside_the_device(tiny):
+    """moe_forward, called through the C ABI with x or y in pinned host memory,
+    returns MOE_ERR_INVALID_ARG before launching anything. (Pinned memory is
+    readable from the device, so even an accepted pointer could not fault.)"""
+    lay, layer = tiny
+    T = 4
+    xd = lay["x"][:T].contiguous()
+    yd = torch.empty_like(xd)
+    xh = xd.cpu().pin_memory()
+    yh = torch.empty_like(xh).pin_memory()
+    L = moe.lib()
+    s = torch.cuda.current_stream().cuda_stream
+    for xp, yp in ((xh, yd), (xd, yh)):
+        st = L.moe_forward(layer._h, xp.data_ptr(), T, yp.data_ptr(), None, None, s)
+        assert st == moe.MOE_ERR_INVALID_ARG
+    torch.cuda.synchronize()
+    assert layer.status() == moe.MOE_OK
+    # the same call with device buffers still runs
+    assert L.moe_forward(layer._h, xd.data_ptr(), T, yd.data_ptr(), None, None, s) == moe.MOE_OK
+    torch.cuda.synchronize()
+
+
 def test_forward_host_matches_device(tiny):
     lay, layer = tiny
     T = 17
