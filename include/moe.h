@@ -72,7 +72,9 @@ typedef enum {
  * moe_intermediate_size, n_routed_experts, n_shared_experts,
  * num_experts_per_tok, routed_scaling_factor, swiglu_limit).
  *
- * Supported: hidden % 128 == 0, inter % 128 == 0, 1 <= top_k <= n_routed <= 512,
+ * Supported: hidden % 128 == 0, inter % 128 == 0, both <= 16384,
+ * 1 <= top_k <= min(n_routed, 32), n_routed <= 512 (the top-k kernels hold up
+ * to 16 scores per lane and 32 selections per token in registers),
  * 0 <= n_shared <= 4, 1 <= max_tokens <= 65536, route_scale > 0 and finite,
  * swiglu_limit >= 0 (INFINITY disables both clamps). Anything else returns
  * MOE_ERR_UNSUPPORTED (shape) or MOE_ERR_INVALID_ARG (NaN, negative, zero).
