@@ -250,6 +250,42 @@ def test_shared_expert_always_on_with_weight_one():
     assert np.allclose(y, om.expert_forward(x, s1[0], s3[0], s2[0], LIM)[0], rtol=1e-15)
 
 
+def _layer_with_shared(S, seed=11):
+    rng = np.random.default_rng(seed)
+    T, H, I, E = 5, 8, 4, 6
+    x = rng.standard_normal((T, H)); wg = rng.standard_normal((E, H))
+    w1 = rng.standard_normal((E, I, H)); w3 = rng.standard_normal((E, I, H)); w2 = rng.standard_normal((E, H, I))
+    s1 = rng.standard_normal((S, I, H)); s3 = rng.standard_normal((S, I, H)); s2 = rng.standard_normal((S, H, I))
+    return x, wg, (w1, w3, w2), (s1, s3, s2)
+
+
+def test_no_shared_expert_is_the_routed_sum():
+    # n_shared = 0: y is the weighted sum over the selected experts, written out here
+    x, wg, (w1, w3, w2), (s1, s3, s2) = _layer_with_shared(0)
+    ex = om.ExpertSource.from_arrays(w1, w3, w2, s1, s3, s2)
+    res = om.moe_forward(x, wg, ex, 2, RS, LIM)
+    want = np.zeros_like(x)
+    for t in range(x.shape[0]):
+        for j in range(2):
+            e = res.route.idx[t, j]
+            want[t] += res.route.w[t, j] * om.expert_forward(x[t:t + 1], w1[e], w3[e], w2[e], LIM)[0][0]
+    assert np.allclose(res.y, want, rtol=1e-13, atol=1e-13)
+
+
+def test_each_shared_expert_adds_with_weight_one():
+    # two shared experts: one with W2 = 0 changes nothing; a copy of the first
+    # adds the same contribution again
+    x, wg, routed, (s1, s3, s2) = _layer_with_shared(1)
+    one = om.moe_forward(x, wg, om.ExpertSource.from_arrays(*routed, s1, s3, s2), 2, RS, LIM).y
+    zero2 = (np.concatenate([s1, s1]), np.concatenate([s3, s3]), np.concatenate([s2, np.zeros_like(s2)]))
+    with_zero = om.moe_forward(x, wg, om.ExpertSource.from_arrays(*routed, *zero2), 2, RS, LIM).y
+    assert np.allclose(with_zero, one, rtol=1e-15, atol=1e-15)
+    twice = (np.concatenate([s1, s1]), np.concatenate([s3, s3]), np.concatenate([s2, s2]))
+    doubled = om.moe_forward(x, wg, om.ExpertSource.from_arrays(*routed, *twice), 2, RS, LIM).y
+    shared = om.expert_forward(x, s1[0], s3[0], s2[0], LIM)[0]
+    assert np.allclose(doubled - one, shared, rtol=1e-12, atol=1e-12)
+
+
 def test_permutation_reference_brute_force():
     rng = np.random.default_rng(2)
     T, k, E = 11, 3, 5
