@@ -190,15 +190,20 @@ class MoELayer:
         torch.cuda.synchronize()
         self.hidden, self.inter, self.n_routed, self.n_shared, self.top_k = H, I, E, S, top_k
         self.max_tokens = max_tokens
+        self.device = router_w.device
 
     # ------------------------------------------------------------------ forward
     def forward(self, x: torch.Tensor, out: Optional[torch.Tensor] = None, topk_idx: Optional[torch.Tensor] = None,
                 topk_w: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
         T = x.shape[0]
         _need(x, "x", torch.bfloat16, (T, self.hidden))
+        if x.device != self.device:
+            raise ValueError(f"x is on {x.device}, the layer on {self.device}")
         if out is None:
             out = torch.empty_like(x)
         _need(out, "out", torch.bfloat16, (T, self.hidden))
+        if out.device != self.device:
+            raise ValueError(f"out is on {out.device}, the layer on {self.device}")
         if topk_idx is not None:
             _need(topk_idx, "topk_idx", torch.int32, (T, self.top_k))
         if topk_w is not None:
