@@ -84,8 +84,8 @@ __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* m) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(m)) : "memory");
 }
 
-// 2-D tiled load of one box into shared memory, completing tx bytes on `bar`.
-// No cluster multicast.
+// 2-D tiled load of one box into this CTA's own shared memory, completing tx
+// bytes on `bar`.
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* m, uint64_t* bar, int32_t x, int32_t y,
                                             uint64_t policy) {
   asm volatile(
