@@ -138,7 +138,9 @@ MOE_API moe_status moe_create(const moe_config* cfg, const moe_weights* w, moe_s
  *   topk_idx int32 [T, k] device or NULL: selected experts, descending score
  *   topk_w   fp32  [T, k] device or NULL: their weights (sum = route_scale)
  * 0 <= T <= max_tokens; T == 0 enqueues nothing. Allocates nothing and does not
- * synchronise. Calls on one handle must be ordered (one stream at a time): the
+ * synchronise. A token whose router scores are not finite (NaN or infinite
+ * input) gets placeholder experts with NaN weights and a NaN output row, and
+ * moe_get_status then reports MOE_ERR_DEVICE; other tokens are unaffected. Calls on one handle must be ordered (one stream at a time): the
  * workspace is shared between calls. MOE_ERR_INVALID_ARG, with nothing enqueued,
  * when the current device is not the handle's or x / y are not device (or
  * managed) memory of it (a host pointer would fault the kernels).
@@ -257,9 +259,16 @@ MOE_API const char* moe_kernel_name(int32_t kind);
  *   topk_idx    int32 [T, top_k] device (output), descending score
  *   topk_w      fp32  [T, top_k] device (output), sum = route_scale
  * hidden % 8 == 0, 1 <= top_k <= min(n_routed, 32), n_routed <= 512. The
- * results equal moe_forward's topk_idx / topk_w for the same inputs. Buffers
- * that are not device (or managed) memory of the current device give
- * MOE_ERR_INVALID_ARG with nothing enqueued.
+ * selection is the same as moe_forward's topk_idx for the same inputs (both
+ * re-score the near-tie candidates exactly; only an exact tie of the float64
+ * scores could resolve differently) and the weights agree within float32
+ * rounding. Buffers that are not device (or managed) memory of the current
+ * device give MOE_ERR_INVALID_ARG with nothing enqueued.
+ *
+ * There is no handle and so no status word: a token whose scores are not
+ * finite (NaN or infinite x, router weights or bias) gets the placeholder
+ * experts 0, 1, ..., top_k - 1 in the slots that found no valid expert, with
+ * NaN weights; check topk_w for NaN when the input may be non-finite.
  *
  * The only scratch, the fp32 logits [T, n_routed], lives in a fixed array of
  * MOE_NOALLOC_MAX_LOGITS floats (4 MiB) inside the library; every GPU that
@@ -267,7 +276,11 @@ MOE_API const char* moe_kernel_name(int32_t kind);
  * MOE_NOALLOC_MAX_LOGITS returns MOE_ERR_UNSUPPORTED and enqueues nothing.
  * Nothing is allocated, by this call or by anything it calls. The first call
  * on a device looks up the array's device address once for that device (with
- * that device current); make that first call before any stream capture. All
+ * that device current); make that first call before any stream capture. The
+ * looked-up address is kept for the life of the process: after
+ * cudaDeviceReset (or anything else that destroys the device's primary
+ * context) it is stale, so do not call this entry point on that device again
+ * in the same process. All
  * calls share the one array, and each call writes every entry it later reads,
  * so nothing needs clearing between calls; calls that overlap on the GPU (on
  * streams not ordered with each other) race on it.

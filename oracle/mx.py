@@ -13,7 +13,7 @@ DeepseekV41Config encodings):
   * a routed expert of the Flash shape occupies 18.8 MB (Strata DEEPSEEK41.md,
     "Where it goes" table), i.e. 4.25 bits per parameter.
 
-Readings adopted where the pages are silent (each listed in the design doc):
+Readings adopted where the pages are silent:
   * block rule = OCP MX v1.0: shared exponent floor(log2(amax)) - emax_elem,
     clamped to the E8M0 range, elements rounded to nearest-even and saturated
     to the element format's largest finite magnitude (E4M3: 448, E2M1: 6);

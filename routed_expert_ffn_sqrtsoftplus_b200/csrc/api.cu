@@ -16,10 +16,6 @@ using namespace moe;
 
 namespace {
 
-// Logit error of the approximate router is far below this (fp32 sums of exact
-// BF16 products, or tensor-core fp32 accumulation); every expert whose
-// approximate score lies within kRefineDelta of the k-th is re-scored exactly.
-constexpr float kRefineDelta = 2e-3f;
 // Token counts above this use the tensor-core router GEMM for the logits.
 constexpr int kTcRouterMinTokens = 256;
 // Token counts up to this use the sliced CUDA-core router and the per-token top-k.

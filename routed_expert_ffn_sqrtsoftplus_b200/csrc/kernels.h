@@ -69,6 +69,11 @@ enum KernelKind {
 };
 
 // ---- router
+// Logit error of the approximate router is far below this (fp32 sums of exact
+// BF16 products, or tensor-core fp32 accumulation); every expert whose
+// approximate score lies within kRefineDelta of the k-th is re-scored exactly.
+// moe_forward and moe_route_noalloc use the same band.
+constexpr float kRefineDelta = 2e-3f;
 cudaError_t launch_router_logits(const void* x, const void* wg, const float* bias, float* z, int T, int H, int E,
                                  cudaStream_t s);
 // Few tokens (T <= 32): fp32 logit slices [H / router_small_slice(H)][T][E] over

@@ -43,6 +43,9 @@ __global__ void __launch_bounds__(128)
   }
   for (int j = 0; j < k; ++j) {
     const int row = __ldg(inv + static_cast<size_t>(t) * k + j);
+    // every slot's row is below T*k; the check keeps a corrupted row index from
+    // reading outside O
+    if (row < 0 || static_cast<size_t>(row) >= routed_rows) continue;
     const float wj = __ldg(w + static_cast<size_t>(t) * k + j);
     const float4 v = __ldg(O + static_cast<size_t>(row) * H4 + c);
     acc.x = fmaf(wj, v.x, acc.x);

@@ -45,9 +45,6 @@ moe_status scratch_for_current_device(float** out) {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-// Same refinement band as moe_forward's router.
-constexpr float kRefineDelta = 2e-3f;
-
 }  // namespace
 
 extern "C" moe_status moe_route_noalloc(const void* x, const void* router_w, const float* router_bias, int32_t T,
@@ -76,7 +73,7 @@ extern "C" moe_status moe_route_noalloc(const void* x, const void* router_w, con
   // The logits kernel overwrites all T*E entries before the top-k kernel reads
   // them, so nothing left in the array by an earlier call is ever used.
   if (moe::launch_router_logits(x, router_w, router_bias, z, T, hidden, n_routed, s) != cudaSuccess ||
-      moe::launch_topk_refine(z, x, router_w, router_bias, T, hidden, n_routed, top_k, route_scale, kRefineDelta,
+      moe::launch_topk_refine(z, x, router_w, router_bias, T, hidden, n_routed, top_k, route_scale, moe::kRefineDelta,
                               topk_idx, topk_w, nullptr, s) != cudaSuccess) {
     cudaGetLastError();
     return MOE_ERR_CUDA;

@@ -175,6 +175,27 @@ __device__ __forceinline__ void warp_argmax_d(double& v, int& i) {
   }
 }
 
+// Writes one token's selection. A token whose scores are not finite numbers
+// (NaN or infinite x, router weights or bias) can leave a selection slot
+// without a valid expert; such a slot gets expert r (an in-range placeholder,
+// so the permutation and the combine never index outside their buffers) and a
+// NaN weight, which makes the token's output NaN, and the device status word
+// records MOE_ERR_DEVICE.
+__device__ __forceinline__ void write_selection(const int* sel_e, const double* sel_s, double sum, int k, int E,
+                                                float route_scale, int32_t* idx, float* w, int* status) {
+  for (int r = 0; r < k; ++r) {
+    int e = sel_e[r];
+    float wr = static_cast<float>(route_scale * (sel_s[r] / sum));
+    if (e < 0 || e >= E) {
+      report_status(status, kStatusDevice);
+      e = r;
+      wr = __int_as_float(0x7fc00000);
+    }
+    idx[r] = e;
+    w[r] = wr;
+  }
+}
+
 constexpr int kTopkWarps = 8;
 constexpr int kPartBatch = 4;      // logit slices loaded together (top-k CTA kernel)
 constexpr int kWBatch = 10;        // Wg chunks per lane loaded together (exact re-scoring)
@@ -312,14 +333,8 @@ __global__ void __launch_bounds__(kTopkWarps * 32)
     sel_e[r] = bi;
     sum += bv;
   }
-  if (lane == 0) {
-    for (int r = 0; r < k; ++r) {
-      const int e = sel_e[r];
-      if (e < 0 || e >= E) report_status(status, kStatusDevice);
-      idx_out[static_cast<size_t>(t) * k + r] = e;
-      w_out[static_cast<size_t>(t) * k + r] = static_cast<float>(route_scale * (sel_s[r] / sum));
-    }
-  }
+  if (lane == 0) write_selection(sel_e, sel_s, sum, k, E, route_scale, idx_out + static_cast<size_t>(t) * k,
+                                  w_out + static_cast<size_t>(t) * k, status);
 }
 
 // Top-k for few tokens, one CTA per token: warp 0 forms the approximate scores
@@ -500,14 +515,8 @@ __global__ void __launch_bounds__(256)
     sel_e[r] = bi;
     sum += bv;
   }
-  if (lane == 0) {
-    for (int r = 0; r < k; ++r) {
-      const int e = sel_e[r];
-      if (e < 0 || e >= E) report_status(status, kStatusDevice);
-      idx_out[static_cast<size_t>(t) * k + r] = e;
-      w_out[static_cast<size_t>(t) * k + r] = static_cast<float>(route_scale * (sel_s[r] / sum));
-    }
-  }
+  if (lane == 0) write_selection(sel_e, sel_s, sum, k, E, route_scale, idx_out + static_cast<size_t>(t) * k,
+                                  w_out + static_cast<size_t>(t) * k, status);
 }
 
 }  // namespace
