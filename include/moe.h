@@ -196,7 +196,15 @@ typedef enum {
   MOE_BUF_INV = 6,      /* int32 [T*k] row of each flat slot */
   MOE_BUF_H = 7,        /* BF16 [T*k + n_shared*T, I] SwiGLU output rows (group order) */
   MOE_BUF_XQ = 8,       /* MXFP4 layers: uint8 E4M3 [T*k, H], MXFP8 codes of the routed rows (perm order) */
-  MOE_BUF_XQ_SCALES = 9 /* MXFP4 layers: their E8M0 scales, packed in 512-byte atoms per token tile */
+  MOE_BUF_XQ_SCALES = 9, /* MXFP4 layers: their E8M0 scales, packed in 512-byte atoms per token tile */
+  MOE_BUF_HQ = 10,       /* MXFP4 layers: uint8 E4M3 [T*k, I], MXFP8 codes of the routed SwiGLU rows
+                            (group order, as MOE_BUF_H) */
+  MOE_BUF_HQ_SCALES = 11 /* MXFP4 layers: their E8M0 scales in 512-byte atoms, one per (down-GEMM
+                            token tile nt, 128-wide slice c of I): row n of the tile, block b of the
+                            slice at byte (nt * I/128 + c) * 512 + (n % 32) * 16 + (n / 32) * 4 + b.
+                            Token tiles: each routed group's rows cut into tiles of 32 rows when
+                            T <= 32, 96 rows when T * top_k >= 24 * n_routed, else 64 rows,
+                            numbered group by group in expert order */
 } moe_buffer;
 
 /*

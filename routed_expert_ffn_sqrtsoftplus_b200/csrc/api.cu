@@ -825,6 +825,16 @@ moe_status moe_inspect(moe_handle* h, int32_t what, void* dst, size_t bytes, moe
       src = h->sfb_gu;
       cap = h->max_ntiles_r * (h->cfg.hidden / 128) * 512;
       break;
+    case MOE_BUF_HQ:
+      if (!h->mx) return MOE_ERR_INVALID_ARG;
+      src = h->hq;
+      cap = Tm * k * I;
+      break;
+    case MOE_BUF_HQ_SCALES:
+      if (!h->mx) return MOE_ERR_INVALID_ARG;
+      src = h->sfb_dn;
+      cap = h->max_ntiles_r * (I / 128) * 512;
+      break;
     default: return MOE_ERR_INVALID_ARG;
   }
   if (bytes > cap) return MOE_ERR_INVALID_ARG;

@@ -32,17 +32,54 @@ def f64(t: torch.Tensor) -> np.ndarray:
     return t.detach().to("cpu").to(torch.float64).numpy()
 
 
-class LayerExperts(om.ExpertSource):
-    """Oracle expert source reading one expert at a time from the generator's tensors."""
+def _bf16_bits_to_f64(u16: np.ndarray) -> np.ndarray:
+    """Exact float64 values of BF16 bit patterns (uint16)."""
+    return (u16.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
 
-    def __init__(self, layer: dict, mx_q: dict | None = None, mx_from_bf16: bool = False):
+
+def _mxfp4_roundtrip_expert(mats):
+    """Worker: the oracle's MXFP4 round trip of one expert's three BF16 matrices
+    (given as uint16 bit patterns); float32 holds every result exactly."""
+    from oracle import mx as omx
+    return tuple(omx.mx_roundtrip(_bf16_bits_to_f64(m), "e2m1").astype(np.float32) for m in mats)
+
+
+def _u16(t: torch.Tensor) -> np.ndarray:
+    return t.detach().to("cpu").contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+def oracle_pool(n: int | None = None):
+    """A spawn-started process pool for the oracle's per-expert work (safe after CUDA is initialised)."""
+    import multiprocessing as mp
+    import os
+    n = n or max(1, min(16, len(os.sched_getaffinity(0))))
+    return mp.get_context("spawn").Pool(n)
+
+
+class LayerExperts(om.ExpertSource):
+    """Oracle expert source reading one expert at a time from the generator's tensors.
+
+    mx_from_bf16: the routed experts are the oracle's own MXFP4 quantisation of the
+    BF16 draw. With a process pool and the list of experts the comparison needs
+    (in the order the oracle visits them), that quantisation runs in the pool,
+    a batch of experts at a time; the oracle itself is unchanged.
+    """
+
+    def __init__(self, layer: dict, mx_q: dict | None = None, mx_from_bf16: bool = False, pool=None,
+                 needed=None):
         S = layer["sh_w1"].shape[0]
         E = layer["w1"].shape[0]
+        self._layer = layer
+        self._pool = pool
+        self._needed = [int(e) for e in needed] if needed is not None else None
+        self._cache = {}
         if mx_from_bf16:
-            # quantise each routed expert with the oracle's own MXFP4 codec
             from oracle import mx as omx
-            rt = lambda w: omx.mx_roundtrip(f64(w), "e2m1")
-            routed = lambda e: (rt(layer["w1"][e]), rt(layer["w3"][e]), rt(layer["w2"][e]))
+            if pool is None or needed is None:
+                rt = lambda w: omx.mx_roundtrip(f64(w), "e2m1")
+                routed = lambda e: (rt(layer["w1"][e]), rt(layer["w3"][e]), rt(layer["w2"][e]))
+            else:
+                routed = self._pooled_mx
             is_mx = True
         elif mx_q is None:
             routed = lambda e: (f64(layer["w1"][e]), f64(layer["w3"][e]), f64(layer["w2"][e]))
@@ -56,6 +93,57 @@ class LayerExperts(om.ExpertSource):
         shared = lambda j: (f64(layer["sh_w1"][j]), f64(layer["sh_w3"][j]), f64(layer["sh_w2"][j]))
         super().__init__(routed, shared, E, S, routed_is_mx=is_mx)
 
+    def _pooled_mx(self, e):
+        if e not in self._cache:
+            self._cache.clear()
+            pos = self._needed.index(e) if e in self._needed else None
+            batch = self._needed[pos:pos + 2 * self._pool._processes] if pos is not None else [e]
+            lay = self._layer
+            jobs = [(_u16(lay["w1"][b]), _u16(lay["w3"][b]), _u16(lay["w2"][b])) for b in batch]
+            for b, mats in zip(batch, self._pool.map(_mxfp4_roundtrip_expert, jobs)):
+                self._cache[b] = mats
+        return tuple(m.astype(np.float64) for m in self._cache[e])
+
+
+def covering_tokens(idx, n_routed, n_shared=0, block=32):
+    """Tokens whose rows reach every `block`-row slice of every expert group.
+
+    The grouped GEMMs lay each expert's rows out in ascending (token, slot) order
+    and cut them into token tiles of at most 256 rows, loaded in 32-row boxes; a
+    mistake in one tile's or one box's offsets shows only in the tokens whose rows
+    fall inside it. Covering every 32-row slice of every routed group (and of each
+    shared group, whose rows are the tokens in order) therefore exercises every
+    token tile, every box, and, because each compared row spans the whole hidden
+    and expert width, every weight tile. Greedy: the first token of each slice not
+    yet reached. Returns sorted token indices.
+    """
+    idx = np.asarray(idx, dtype=np.int64)
+    T, k = idx.shape
+    flat = idx.reshape(-1)
+    order = np.argsort(flat, kind="stable")
+    counts = np.bincount(flat, minlength=n_routed)
+    offsets = np.concatenate([[0], np.cumsum(counts)])
+    row_in_group = np.empty(T * k, dtype=np.int64)
+    row_in_group[order] = np.arange(T * k) - offsets[flat[order]]
+    nblk = (T + block - 1) // block
+    pair = flat * nblk + row_in_group // block          # routed (expert, slice)
+    tok_pairs = pair.reshape(T, k)
+    covered = set()
+    chosen = []
+    first_slot = {}
+    for s in order:                                     # ascending rows inside each expert
+        first_slot.setdefault(int(pair[s]), int(s))
+    for p in sorted(first_slot):
+        if p in covered:
+            continue
+        t = first_slot[p] // k
+        chosen.append(t)
+        covered.update(int(q) for q in tok_pairs[t])
+    if n_shared > 0:
+        have = {t // block for t in chosen}
+        chosen.extend(b * block for b in range(nblk) if b not in have)
+    return np.array(sorted(set(chosen)), dtype=np.int64)
+
 
 def oracle_route(layer, k, rs, tokens=None):
     x = layer["x"] if tokens is None else layer["x"][tokens]
@@ -63,16 +151,16 @@ def oracle_route(layer, k, rs, tokens=None):
     return om.route(f64(x), f64(layer["wg"]), k, rs, bias=bias)
 
 
-def compare_layer(layer, tokens, y_gpu, idx_gpu, w_gpu, k, rs, limit, mx_q=None, mx_from_bf16=False):
+def compare_layer(layer, tokens, y_gpu, idx_gpu, w_gpu, k, rs, limit, mx_q=None, mx_from_bf16=False, pool=None):
     """Compare GPU rows (for `tokens`) with the oracle; returns a report dict, asserts the bars.
 
     With mx_q (packed MXFP4 tensors) or mx_from_bf16 the routed experts are MXFP4 and
-    the oracle mirrors the MXFP8 activation quantisation."""
+    the oracle mirrors the MXFP8 activation quantisation. `pool` (oracle_pool())
+    spreads the oracle's MXFP4 quantisation of the experts over processes."""
     tokens = np.asarray(tokens)
     x = f64(layer["x"][torch.as_tensor(tokens, device=layer["x"].device)])
     wg = f64(layer["wg"])
     bias = None if layer.get("bias") is None else f64(layer["bias"])
-    ex = LayerExperts(layer, mx_q, mx_from_bf16)
     r = om.route(x, wg, k, rs, bias=bias)
     idx_g = np.asarray(idx_gpu, dtype=np.int64)
     sure = r.gap > GAP_EXACT
@@ -81,6 +169,7 @@ def compare_layer(layer, tokens, y_gpu, idx_gpu, w_gpu, k, rs, limit, mx_q=None,
                            f"gpu {idx_g[mism[:1]]} oracle {r.idx[mism[:1]]} gap {r.gap[mism[:1]]}"
     # outputs: use the GPU's selection where the oracle's gap is within the tie band
     override = np.where(sure[:, None], r.idx, idx_g)
+    ex = LayerExperts(layer, mx_q, mx_from_bf16, pool=pool, needed=np.unique(override))
     res = om.moe_forward(x, wg, ex, k, rs, limit, bias=bias, idx_override=override)
     w_or = res.route.w
     dw = np.abs(np.asarray(w_gpu, dtype=np.float64) - w_or).max()
@@ -91,4 +180,32 @@ def compare_layer(layer, tokens, y_gpu, idx_gpu, w_gpu, k, rs, limit, mx_q=None,
     err = float(np.abs(yg - yo).max())
     assert np.all(np.isfinite(yg)), "non-finite GPU output"
     assert err <= TOL_Y * rms, f"max|dy| = {err:.3e} > {TOL_Y} * RMS {rms:.3e}"
-    return dict(max_abs_err=err, rms=rms, rel=err / rms, near_ties=int((~sure).sum()), max_dw=float(dw))
+    rel = err / rms if rms > 0 else 0.0       # rms == 0 (e.g. swiglu_limit 0): err must be exactly 0
+    return dict(max_abs_err=err, rms=rms, rel=rel, near_ties=int((~sure).sum()), max_dw=float(dw),
+                tokens=len(tokens))
+
+
+def check_nan_token(layer, lay, T, bad, k, E, rs, limit, mx_q=None):
+    """Forward T tokens of lay["x"] with token `bad` set to NaN; assert the NaN stays
+    in that token and the others still match the oracle."""
+    import routed_expert_ffn_sqrtsoftplus_b200 as moe
+    x = lay["x"][:T].clone()
+    x[bad] = float("nan")
+    y, idx, w = layer.forward_with_routing(x)
+    torch.cuda.synchronize()
+    # the token's scores are NaN: placeholder experts 0..k-1, NaN weights, NaN row,
+    # and the status word says so; the other tokens are computed as usual
+    assert layer.status() == moe.MOE_ERR_DEVICE
+    assert layer.status() == moe.MOE_OK
+    idx_np, w_np, y_np = idx.cpu().numpy(), w.cpu().numpy(), y.float().cpu().numpy()
+    assert np.all((idx_np >= 0) & (idx_np < E))
+    assert list(idx_np[bad]) == list(range(k))
+    assert np.all(np.isnan(w_np[bad])) and np.all(np.isnan(y_np[bad]))
+    keep = np.setdiff1d(np.arange(T), [bad])
+    rep = compare_layer(dict(lay, x=x), keep, y_np[keep], idx_np[keep], w_np[keep], k, rs,
+                          limit, mx_q=mx_q)
+    assert rep["rel"] < TOL_Y
+    # the next forward on finite input is clean
+    layer.forward(lay["x"][:T].contiguous())
+    torch.cuda.synchronize()
+    assert layer.status() == moe.MOE_OK

@@ -23,7 +23,7 @@ def _free():
     torch.cuda.empty_cache()
 
 
-def _run_workload(name, n_sample, cuda_device):
+def _run_workload(name, cuda_device):
     build.build()
     wl = synth.WORKLOADS[name]
     lay = synth.make_layer(wl, device=cuda_device)
@@ -48,9 +48,9 @@ def _run_workload(name, n_sample, cuda_device):
         cnt = layer.inspect(moe.BUF_COUNTS, torch.empty(G, dtype=torch.int32, device=cuda_device)).cpu().numpy()
         assert cnt[:wl.E].sum() == wl.T * wl.k and np.all(cnt[wl.E:] == wl.T)
         assert np.array_equal(cnt[:wl.E], np.bincount(idx_np.ravel(), minlength=wl.E))
-        # outputs
-        toks = np.arange(wl.T) if n_sample >= wl.T else \
-            np.sort(np.random.default_rng(wl.seed).choice(wl.T, n_sample, replace=False))
+        # outputs: every token at decode; otherwise a sample reaching every 32-row
+        # slice of every expert group (every token tile, B box and weight tile)
+        toks = np.arange(wl.T) if wl.T <= 32 else parity.covering_tokens(idx_np, wl.E, wl.n_shared)
         rep = parity.compare_layer(lay, toks, y_cpu[toks], idx_np[toks], w_np[toks], wl.k, wl.route_scale,
                                    wl.swiglu_limit)
         rep["near_tie_tokens_all"] = int((~sure).sum())
@@ -63,17 +63,17 @@ def _run_workload(name, n_sample, cuda_device):
 
 
 def test_flash_decode_full(cuda_device):
-    rep, _ = _run_workload("flash_decode", 32, cuda_device)
+    rep, _ = _run_workload("flash_decode", cuda_device)
     assert rep["rel"] < parity.TOL_Y
 
 
 def test_flash_prefill_full(cuda_device):
-    rep, cnt = _run_workload("flash_prefill", 24, cuda_device)
+    rep, cnt = _run_workload("flash_prefill", cuda_device)
     assert rep["rel"] < parity.TOL_Y
 
 
 def test_pro_skewed_full(cuda_device):
-    rep, cnt = _run_workload("pro_skewed", 12, cuda_device)
+    rep, cnt = _run_workload("pro_skewed", cuda_device)
     assert rep["rel"] < parity.TOL_Y
     # Zipf-biased routing: the most popular expert takes a large share of the tokens
     assert cnt[:384].max() > 0.5 * synth.WORKLOADS["pro_skewed"].T

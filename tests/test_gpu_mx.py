@@ -6,6 +6,7 @@ import torch
 
 import routed_expert_ffn_sqrtsoftplus_b200 as moe
 from routed_expert_ffn_sqrtsoftplus_b200 import build, synth
+from oracle import moe as om
 from oracle import mx as omx
 
 import parity
@@ -65,6 +66,77 @@ def test_mx_activation_codes_bitexact(tiny_mx):
     assert np.array_equal(omx.decode_e4m3(got), omx.decode_e4m3(codes_ref[rows]))
 
 
+def _hq_values(hq, sf, cnt, T, k, E, I):
+    """Decode the MXFP8 h rows the gate/up epilogue wrote (codes + scale atoms, the
+    layout include/moe.h gives for MOE_BUF_HQ / MOE_BUF_HQ_SCALES)."""
+    bn = 32 if T <= 32 else (96 if T * k >= 24 * E else 64)
+    off = np.concatenate([[0], np.cumsum(cnt)])
+    ntb = np.concatenate([[0], np.cumsum((cnt + bn - 1) // bn)])
+    R = T * k
+    g = np.searchsorted(off, np.arange(R), side="right") - 1
+    j = np.arange(R) - off[g]
+    nt, n = ntb[g] + j // bn, j % bn
+    b = np.arange(I // 32)
+    addr = (nt[:, None] * (I // 128) + b[None, :] // 4) * 512 + (n[:, None] % 32) * 16 + (n[:, None] // 32) * 4 \
+        + b[None, :] % 4
+    codes = sf[addr]
+    vals = omx.dequantize_mx(hq, codes, "e4m3")
+    return vals, codes
+
+
+@pytest.mark.parametrize("T", [16, 64, 300])
+def test_mx_swiglu_rows_match_oracle(tiny_mx, T):
+    """The MXFP8 h rows (E4M3 codes and E8M0 scales) that the MX gate/up epilogue
+    writes, element by element, against the oracle's h of the same expert on the
+    same MXFP8 token: within one E4M3 step at the value's magnitude, scale codes
+    equal wherever the block's amax is not within 1e-4 of a power of two."""
+    lay, mxq, layer = tiny_mx
+    x = lay["x"][:T].contiguous()
+    _, idx, _ = layer.forward_with_routing(x)
+    R = T * WL.k
+    dev = x.device
+    hq = layer.inspect(moe.BUF_HQ, torch.empty((R, WL.I), dtype=torch.uint8, device=dev))
+    sf = layer.inspect(moe.BUF_HQ_SCALES, torch.empty(_hq_scale_cap(), dtype=torch.uint8, device=dev))
+    perm = layer.inspect(moe.BUF_PERM, torch.empty(R, dtype=torch.int32, device=dev))
+    cnt = layer.inspect(moe.BUF_COUNTS, torch.empty(WL.E + WL.n_shared, dtype=torch.int32, device=dev))
+    torch.cuda.synchronize()
+    assert layer.status() == moe.MOE_OK
+    cnt = cnt.cpu().numpy()[:WL.E].astype(np.int64)
+    vals, codes = _hq_values(hq.cpu().numpy(), sf.cpu().numpy(), cnt, T, WL.k, WL.E, WL.I)
+    perm = perm.cpu().numpy()
+    idx = idx.cpu().numpy().reshape(-1)
+    xf = parity.f64(x)
+    ex = parity.LayerExperts(lay, mx_q=mxq)
+    flips = 0
+    for e in range(WL.E):
+        rows = np.nonzero(idx[perm] == e)[0]
+        if len(rows) == 0:
+            continue
+        _, h_or = om.expert_forward(xf[perm[rows] // WL.k], *ex.routed(e), WL.swiglu_limit, mx_act=True)
+        q_or, sc_or = omx.quantize_mx(h_or, "e4m3")
+        amax = np.abs(h_or.reshape(len(rows), -1, 32)).max(axis=-1)
+        l2 = np.log2(np.where(amax > 0, amax, 1.0))
+        near_pow2 = np.abs(l2 - np.round(l2)) < 1.5e-4
+        assert np.all((codes[rows] == sc_or) | near_pow2), f"expert {e}: scale codes differ"
+        X = np.repeat(omx.decode_e8m0(sc_or), 32, axis=-1)
+        bound = 2.0 ** -3 * np.abs(h_or) + 2.0 ** -8 * X
+        err = np.abs(vals[rows] - h_or)
+        assert np.all(err <= bound), f"expert {e}: max err / bound {np.max(err / bound)}"
+        flips += int(np.sum(omx.decode_e4m3(hq.cpu().numpy()[rows]) * X != omx.dequantize_mx(q_or, sc_or, "e4m3")))
+    print(f"T={T}: element codes differing from the oracle's (RNE neighbours): {flips}")
+
+
+def _hq_scale_cap():
+    """Bytes of the h scale atoms a layer with max_tokens 400 holds (tiny shape)."""
+    return (WL.E + (400 * WL.k + 31) // 32) * (WL.I // 128) * 512
+
+
+@pytest.mark.parametrize("T,bad", [(16, 3), (64, 40)])
+def test_mx_nan_token_is_contained(tiny_mx, T, bad):
+    lay, mxq, layer = tiny_mx
+    parity.check_nan_token(layer, lay, T, bad, WL.k, WL.E, WL.route_scale, WL.swiglu_limit, mx_q=mxq)
+
+
 def test_mx_deterministic(tiny_mx):
     lay, _, layer = tiny_mx
     x = lay["x"][:300].contiguous()
@@ -87,10 +159,15 @@ def test_mx_rejects_nan_scale(cuda_device):
 
 
 @pytest.mark.slow
-@pytest.mark.parametrize("name,n_sample", [("flash_mxfp4_decode", 6), ("flash_mxfp4_prefill", 6)])
-def test_flash_mxfp4_full(cuda_device, name, n_sample):
+@pytest.mark.parametrize("name", ["flash_mxfp4_decode", "flash_mxfp4_prefill"])
+def test_flash_mxfp4_full(cuda_device, name):
+    """Full-size MXFP4 layers. Outputs compared on every token at decode, and at
+    prefill on a sample that reaches every 32-row slice of every expert group
+    (every token tile and weight tile of every expert that has rows); the oracle
+    quantises the BF16 draw itself, spread over a spawn-started process pool."""
     build.build()
     wl = synth.WORKLOADS[name]
+    pool = parity.oracle_pool()
     lay = synth.make_layer(wl, device=cuda_device)
     mxq = {}
     for n, sname in (("w1", "s1"), ("w3", "s3"), ("w2", "s2")):
@@ -100,16 +177,21 @@ def test_flash_mxfp4_full(cuda_device, name, n_sample):
         y, idx, w = layer.forward_with_routing(lay["x"])
         torch.cuda.synchronize()
         assert layer.status() == moe.MOE_OK
-        toks = np.arange(wl.T) if n_sample >= wl.T else \
-            np.sort(np.random.default_rng(wl.seed).choice(wl.T, n_sample, replace=False))
+        idx_np = idx.cpu().numpy()
+        toks = np.arange(wl.T) if wl.T <= 32 else parity.covering_tokens(idx_np, wl.E, wl.n_shared)
         y_np = y.float().cpu().numpy()
         assert np.all(np.isfinite(y_np))
-        # the oracle quantises the BF16 draw itself (its codec matches moe_quantize_mxfp4 bit for bit)
-        rep = parity.compare_layer(lay, toks, y_np[toks], idx.cpu().numpy()[toks], w.cpu().numpy()[toks], wl.k,
-                                   wl.route_scale, wl.swiglu_limit, mx_from_bf16=True)
+        # routing of every token against the oracle's float64 router
+        r = parity.oracle_route(lay, wl.k, wl.route_scale)
+        sure = r.gap > parity.GAP_EXACT
+        assert not np.any(sure & np.any(idx_np != r.idx, axis=1))
+        del mxq
+        rep = parity.compare_layer(lay, toks, y_np[toks], idx_np[toks], w.cpu().numpy()[toks], wl.k,
+                                   wl.route_scale, wl.swiglu_limit, mx_from_bf16=True, pool=pool)
         print(name, rep)
         assert rep["rel"] < parity.TOL_Y
     finally:
+        pool.terminate()
         layer.close()
-        del lay, mxq
+        del lay
         torch.cuda.empty_cache()

@@ -262,3 +262,20 @@ def test_dspark_shaped_layer(cuda_device, T):
         assert rep["rel"] < parity.TOL_Y
     finally:
         layer.close()
+
+
+@pytest.mark.parametrize("T,bad", [(16, 5), (300, 123)])
+def test_nan_token_is_contained(tiny, T, bad):
+    lay, layer = tiny
+    parity.check_nan_token(layer, lay, T, bad, WL.k, WL.E, WL.route_scale, WL.swiglu_limit)
+
+
+def test_nan_token_is_contained_warp_topk(cuda_device):
+    """Above 1024 tokens the top-k runs one warp per token."""
+    lay = synth.make_layer(WL.with_tokens(1100), device="cpu")
+    lay = {k: (v.to(cuda_device) if isinstance(v, torch.Tensor) else v) for k, v in lay.items()}
+    layer = moe.MoELayer.from_layer(lay, top_k=WL.k, max_tokens=1100)
+    try:
+        parity.check_nan_token(layer, lay, 1100, 1037, WL.k, WL.E, WL.route_scale, WL.swiglu_limit)
+    finally:
+        layer.close()

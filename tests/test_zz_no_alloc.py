@@ -4,11 +4,14 @@ Some callers cannot call cudaMalloc at all (their device memory belongs to a
 host framework's pool, or their loop forbids allocation once running); for
 them the library offers routing whose one scratch buffer is a fixed array
 inside the library. This test calls that entry point through the C ABI and
-checks it against the routing moe_forward returns for the same tokens, on two
-calls in a row (the second with a different token count, so it runs over what
-the first left in the shared array). It sits in its own file, collected last.
+checks it against the float64 oracle's routing and against the routing
+moe_forward returns for the same tokens, on calls in a row (each with a
+different token count, so each runs over what the one before left in the
+shared array). It sits in its own file, collected last.
 """
 import ctypes
+
+import numpy as np
 
 import pytest
 import torch
@@ -37,22 +40,54 @@ def _route_noalloc(x, wg, bias, k, rs):
     return st, idx, w
 
 
+def _check_against_oracle(lay, T, idx, w, k, rs):
+    """Routing parity bar: indices equal to the float64 oracle's wherever its gap
+    exceeds 1e-6, weights within float32 rounding."""
+    r = parity.oracle_route(dict(lay, x=lay["x"][:T]), k, rs)
+    sure = r.gap > parity.GAP_EXACT
+    idx_np, w_np = idx.cpu().numpy(), w.cpu().numpy()
+    assert not np.any(sure & np.any(idx_np != r.idx, axis=1))
+    assert np.abs(w_np[sure] - r.w[sure]).max() <= parity.TOL_W
+    return sure
+
+
 def test_route_noalloc_matches_forward(cuda_device):
     build.build()
+    Tmax = 2000
     lay = {k: (v.to(cuda_device) if isinstance(v, torch.Tensor) else v)
-           for k, v in synth.make_layer(WL.with_tokens(96)).items()}
-    layer = moe.MoELayer.from_layer(lay, top_k=WL.k, max_tokens=96)
+           for k, v in synth.make_layer(WL.with_tokens(Tmax)).items()}
+    layer = moe.MoELayer.from_layer(lay, top_k=WL.k, max_tokens=Tmax)
     try:
-        for T in (96, 23):                       # two calls in a row, the second smaller
+        # calls in a row over the one shared array: the second smaller than the
+        # first, the third above 1024 tokens (one warp per token in the top-k)
+        for T in (96, 23, Tmax):
             x = lay["x"][:T].contiguous()
             _, idx_ref, w_ref = layer.forward_with_routing(x)
             st, idx, w = _route_noalloc(x, lay["wg"], lay["bias"], WL.k, WL.route_scale)
             torch.cuda.synchronize()
             assert st == moe.MOE_OK
-            assert torch.equal(idx, idx_ref)
+            sure = torch.as_tensor(_check_against_oracle(lay, T, idx, w, WL.k, WL.route_scale), device=idx.device)
+            assert torch.equal(idx[sure], idx_ref[sure])
             assert (w - w_ref).abs().max().item() <= parity.TOL_W
     finally:
         layer.close()
+
+
+def test_route_noalloc_nan_token_gets_placeholders(cuda_device):
+    build.build()
+    lay = {k: (v.to(cuda_device) if isinstance(v, torch.Tensor) else v)
+           for k, v in synth.make_layer(WL.with_tokens(40)).items()}
+    x = lay["x"].clone()
+    x[7] = float("nan")
+    st, idx, w = _route_noalloc(x, lay["wg"], None, WL.k, WL.route_scale)
+    torch.cuda.synchronize()
+    assert st == moe.MOE_OK
+    assert idx[7].tolist() == list(range(WL.k)) and bool(torch.isnan(w[7]).all())
+    keep = [t for t in range(40) if t != 7]
+    assert bool(((idx >= 0) & (idx < WL.E)).all())
+    r = parity.oracle_route(dict(lay, x=lay["x"][keep]), WL.k, WL.route_scale)
+    sure = r.gap > parity.GAP_EXACT
+    assert not np.any(sure & np.any(idx[keep].cpu().numpy() != r.idx, axis=1))
 
 
 def test_route_noalloc_with_bias_and_limit(cuda_device):
