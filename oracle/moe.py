@@ -27,7 +27,7 @@ formulas below are the plainest reading, fixed as follows:
 Matrices are stored [out, in] (row-major, input dimension contiguous), so
 W1 x is ``w1 @ x`` for one token and ``x @ w1.T`` for a batch of rows.
 
-MX mirror mode (routed experts in MXFP4): the routed experts see the token
+MX mirror mode (routed experts in MXFP4 or MXFP8): the routed experts see the token
 quantised to MXFP8 (E4M3, one E8M0 scale per 32 along the hidden dimension)
 and the SwiGLU output h quantised the same way along the expert width; the
 router and the shared expert see the unquantised BF16 values.
@@ -159,6 +159,20 @@ class ExpertSource:
     def from_mxfp4(q1, s1, q3, s3, q2, s2, sh_w1, sh_w3, sh_w2):
         """Packed E2M1 [E, I, H/2] / E8M0 [E, I, H/32] (etc.) routed, BF16 shared."""
         dq = mx.dequantize_mxfp4_packed
+        f = lambda a, e: np.asarray(a[e], dtype=np.float64)
+        return ExpertSource(
+            lambda e: (dq(q1[e], s1[e]), dq(q3[e], s3[e]), dq(q2[e], s2[e])),
+            lambda j: (f(sh_w1, j), f(sh_w3, j), f(sh_w2, j)),
+            len(q1), len(sh_w1), routed_is_mx=True)
+
+
+    @staticmethod
+    def from_mxfp8(q1, s1, q3, s3, q2, s2, sh_w1, sh_w3, sh_w2):
+        """E4M3 codes [E, I, H] / E8M0 [E, I, H/32] (etc.) routed, BF16 shared.
+
+        Routed experts stored in a block-scaled 8-bit format meet MXFP8 activations
+        like the MXFP4 ones, so they are marked for the MX mirror as well."""
+        dq = mx.dequantize_mxfp8
         f = lambda a, e: np.asarray(a[e], dtype=np.float64)
         return ExpertSource(
             lambda e: (dq(q1[e], s1[e]), dq(q3[e], s3[e]), dq(q2[e], s2[e])),

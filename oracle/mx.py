@@ -11,14 +11,20 @@ DeepseekV41Config encodings):
   * the family's block scales are ``float8_e8m0`` with one scale per 32 values
     (inference-research "DeepSeek-V4-Pro" page, FlashMLA KV layout paragraph);
   * a routed expert of the Flash shape occupies 18.8 MB (Strata DEEPSEEK41.md,
-    "Where it goes" table), i.e. 4.25 bits per parameter.
+    "Where it goes" table), i.e. 4.25 bits per parameter;
+  * the checkpoint's other weights are FP8 ("dtype": "fp8", inference/config.json)
+    and MAX's default encoding is float8_e4m3fn (DeepseekV41Config
+    DEFAULT_ENCODING / SUPPORTED_ENCODINGS).
 
 Readings adopted where the pages are silent:
   * block rule = OCP MX v1.0: shared exponent floor(log2(amax)) - emax_elem,
     clamped to the E8M0 range, elements rounded to nearest-even and saturated
     to the element format's largest finite magnitude (E4M3: 448, E2M1: 6);
   * an all-zero block gets scale code 0 and zero elements;
-  * E2M1 packing: element 2j in the low nibble, element 2j+1 in the high nibble.
+  * E2M1 packing: element 2j in the low nibble, element 2j+1 in the high nibble;
+  * FP8 expert weights are MXFP8: E4M3 values with one E8M0 scale per 32 along
+    the input dimension, by the same block rule (the pages give no FP8 scale
+    granularity; this is the family's per-32 E8M0 convention).
 
 Everything here is exact float64 arithmetic: every E2M1, E4M3 and E8M0 value is
 a dyadic rational that float64 represents exactly, and scaling by a power of two
@@ -215,6 +221,21 @@ def quantize_mxfp4_packed(w):
 
 def dequantize_mxfp4_packed(packed, scales):
     return dequantize_mx(unpack_e2m1(packed), scales, "e2m1")
+
+
+def quantize_mxfp8(w):
+    """Weights [..., K] -> (E4M3 codes [..., K] uint8, E8M0 [..., K/32] uint8): MXFP8."""
+    return quantize_mx(w, "e4m3")
+
+
+def dequantize_mxfp8(codes, scales):
+    return dequantize_mx(codes, scales, "e4m3")
+
+
+def mxfp8_bytes(rows, cols):
+    """Storage of an MXFP8 [rows, cols] matrix: 1 byte per value + 1 byte per 32."""
+    assert cols % MX_BLOCK == 0
+    return rows * cols + rows * cols // MX_BLOCK
 
 
 def mxfp4_bytes(rows, cols):

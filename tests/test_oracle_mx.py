@@ -161,3 +161,32 @@ def test_mx_mirror_mode_is_exact_on_representable_inputs():
     assert np.array_equal(h_a, h_b)
     assert np.allclose(o_b, mx.mx_roundtrip(h_a, "e4m3") @ w2[0].T, rtol=1e-14)
     assert not np.allclose(o_a, o_b, rtol=1e-6)
+
+
+def test_mxfp8_expert_values_match_torch_decoders():
+    """MXFP8 weights (E4M3 codes + E8M0 scales per 32) served by from_mxfp8 equal
+    PyTorch's float8_e4m3fn and float8_e8m0fnu decodings of the same bytes, and
+    the routed experts are marked for the MX mirror."""
+    rng = np.random.default_rng(12)
+    E, I_, H_, S = 2, 32, 64, 1
+    w = [rng.standard_normal((E, I_, H_)) / 8, rng.standard_normal((E, I_, H_)) / 8,
+         rng.standard_normal((E, H_, I_)) / 6]
+    q = [mx.quantize_mxfp8(a) for a in w]
+    sh = [np.zeros((S, I_, H_)), np.zeros((S, I_, H_)), np.zeros((S, H_, I_))]
+    src = om.ExpertSource.from_mxfp8(q[0][0], q[0][1], q[1][0], q[1][1], q[2][0], q[2][1], *sh)
+    assert src.routed_is_mx
+    for e in range(E):
+        for got, (codes, scales) in zip(src.routed(e), q):
+            v = torch.from_numpy(codes[e].copy()).view(torch.float8_e4m3fn).to(torch.float64)
+            sc = torch.from_numpy(scales[e].copy()).view(torch.float8_e8m0fnu).to(torch.float64)
+            ref = (v.reshape(v.shape[0], -1, 32) * sc[..., None]).reshape(v.shape).numpy()
+            assert np.array_equal(got, ref)
+    # the stored values are the round trip of the weights they were quantised from
+    assert np.array_equal(src.routed(1)[2], mx.mx_roundtrip(w[2][1], "e4m3"))
+
+
+def test_flash_expert_mxfp8_size():
+    """One byte per value plus one E8M0 byte per 32: 3 H I (1 + 1/32) for a Flash expert."""
+    H_, I_ = 5120, 2304
+    per_expert = 2 * mx.mxfp8_bytes(I_, H_) + mx.mxfp8_bytes(H_, I_)
+    assert per_expert == 3 * H_ * I_ * 33 // 32 == 36_495_360
