@@ -54,6 +54,8 @@ def parse():
     p.add_argument("--experts", type=int, default=None,
                    help="override the routed expert count (small instances for profiler captures)")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-secondary", action="store_true",
+                   help="only the headline workload (skip the MXFP4 and prefill lines)")
     p.add_argument("--cpu-seconds", type=float, default=15.0, help="budget of the CPU baseline sample")
     return p.parse_args()
 
@@ -170,11 +172,12 @@ def workload_from_args(args):
 def build_layer(wl, device):
     d = synth.make_layer(wl, device=device)
     mxq = None
-    if wl.expert_dtype == "mxfp4":
-        from routed_expert_ffn_sqrtsoftplus_b200 import quantize_mxfp4
+    if wl.expert_dtype in ("mxfp4", "mxfp8"):
+        from routed_expert_ffn_sqrtsoftplus_b200 import quantize_mxfp4, quantize_mxfp8
+        quant = quantize_mxfp4 if wl.expert_dtype == "mxfp4" else quantize_mxfp8
         mxq = {}
         for n, s in (("w1", "s1"), ("w3", "s3"), ("w2", "s2")):
-            mxq[n], mxq[s] = quantize_mxfp4(d[n])
+            mxq[n], mxq[s] = quant(d[n])
     return d, mxq
 
 
@@ -184,10 +187,11 @@ def algorithmic(wl, idx: np.ndarray, T: int):
     and out once)."""
     H, I, E, S, k = wl.H, wl.I, wl.E, wl.n_shared, wl.k
     U = len(np.unique(idx))
-    mx = wl.expert_dtype == "mxfp4"
+    mx = wl.expert_dtype in ("mxfp4", "mxfp8")
     if mx:
-        routed13 = (2 * I * H) // 2 + (2 * I * H) // 32
-        routed2 = (H * I) // 2 + (H * I) // 32
+        div = 2 if wl.expert_dtype == "mxfp4" else 1     # values per weight byte
+        routed13 = (2 * I * H) // div + (2 * I * H) // 32
+        routed2 = (H * I) // div + (H * I) // 32
         act = 1                                  # MXFP8 activation bytes per value
     else:
         routed13, routed2, act = 2 * I * H * 2, H * I * 2, 2
@@ -253,7 +257,8 @@ def cpu_oracle_sample(wl, d, mxq, tokens, budget_s):
     if mxq is None:
         routed = lambda e: (f64(d["w1"][e]), f64(d["w3"][e]), f64(d["w2"][e]))
     else:
-        dq = lambda n, s, e: omx.dequantize_mxfp4_packed(mxq[n][e].cpu().numpy(), mxq[s][e].cpu().numpy())
+        dqf = omx.dequantize_mxfp8 if wl.expert_dtype == "mxfp8" else omx.dequantize_mxfp4_packed
+        dq = lambda n, s, e: dqf(mxq[n][e].cpu().numpy(), mxq[s][e].cpu().numpy())
         routed = lambda e: (dq("w1", "s1", e), dq("w3", "s3", e), dq("w2", "s2", e))
     shared = lambda j: (f64(d["sh_w1"][j]), f64(d["sh_w3"][j]), f64(d["sh_w2"][j]))
     ex = om.ExpertSource(routed, shared, wl.E, wl.n_shared, routed_is_mx=mxq is not None)
@@ -277,88 +282,36 @@ def cpu_cores():
 
 
 # ----------------------------------------------------------------------------- main arms
-def run_ours(args, world, rank, local):
-    import routed_expert_ffn_sqrtsoftplus_b200 as moe
-    from routed_expert_ffn_sqrtsoftplus_b200 import build
-    if rank == 0:
-        build.build()
-    barrier(world)
-    wl = workload_from_args(args)
-    T = wl.T
-    dev = torch.device("cuda", local)
-    d, mxq = build_layer(wl, dev)
-    layer = moe.MoELayer.from_layer(d, top_k=wl.k, max_tokens=T, route_scale=wl.route_scale,
-                                    swiglu_limit=wl.swiglu_limit, mx=mxq)
-    x = d["x"]
-    y = torch.empty_like(x)
-    stream = torch.cuda.current_stream()
-    # routing of this batch, for the algorithmic byte count
-    _, idx, _ = layer.forward_with_routing(x)
-    torch.cuda.synchronize()
-    alg = algorithmic(wl, idx.cpu().numpy(), T)
-
-    for _ in range(args.warmup):
-        layer.forward(x, out=y)
-    torch.cuda.synchronize()
-    assert layer.status() == moe.MOE_OK
-
-    # ---- device-timed region
-    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    barrier(world)
-    torch.cuda.synchronize()
-    with ClockSampler(local) as clk:
-        ev0.record(stream)
-        for _ in range(args.steps):
-            layer.forward(x, out=y)
-        ev1.record(stream)
+def read_stream_peak(dev, gib: float = 4.0, reps: int = 5):
+    """Read-only streaming bandwidth of this GPU in GB/s: the best of a few library
+    reductions over a buffer far larger than L2, timed with CUDA events. The weight
+    streams of the GEMMs only read, so this is the ceiling they can approach; the
+    copy bandwidth of MEASURED_PEAKS.json counts a read and a write per byte."""
+    n = int(gib * (1 << 30)) // 4
+    buf = torch.ones(n, dtype=torch.int32, device=dev)
+    best = 0.0
+    for op in (lambda t: t.max(), lambda t: t.sum(dtype=torch.int64)):
+        op(buf)
         torch.cuda.synchronize()
-    barrier(world)
-    st = layer.status()
-    if st != moe.MOE_OK:
-        raise RuntimeError(f"device status {st} after the timed steps")
-    ms = ev0.elapsed_time(ev1)
-    ms = max_over_ranks(ms, world)
-    ms_per_step = ms / args.steps
-    value = weak_scaling_value(world, T, args.steps, ms)
+        for _ in range(reps):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            op(buf)
+            e1.record()
+            torch.cuda.synchronize()
+            best = max(best, n * 4 / (e0.elapsed_time(e1) / 1e3) / 1e9)
+    del buf
+    torch.cuda.empty_cache()
+    return best
 
-    # ---- per-kernel attribution: the same K steps again, with the library's CUDA
-    # events recorded on the launch stream around every kernel (an event between
-    # two kernels also keeps the second from starting early, so these per-kernel
-    # times are a little longer than inside the timed loop above)
-    layer.profile_begin(args.steps)
-    for _ in range(args.steps):
-        layer.forward(x, out=y)
-    torch.cuda.synchronize()
-    prof = layer.profile_end()
-    if layer.status() != moe.MOE_OK:
-        raise RuntimeError("device status after the attribution pass")
 
-    # ---- end-to-end through host buffers
-    xh = x.cpu().pin_memory()
-    yh = torch.empty_like(xh).pin_memory()
-    e2e_steps = max(3, min(args.steps, 50))
-    for _ in range(2):
-        layer.forward_host(xh, yh)
-    torch.cuda.synchronize()
-    barrier(world)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(e2e_steps):
-        layer.forward_host(xh, yh)
-    e1.record(stream)
-    torch.cuda.synchronize()
-    barrier(world)
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
-    e2e_value = weak_scaling_value(world, T, e2e_steps, e2e_ms)
-
-    hbm, tc, tc_sus, src = peaks()
-    # dominant kernel = the one with the largest share of device time
-    kern = max(prof, key=lambda n: prof[n][0])
+def kernel_roofline(kern, prof, alg, hbm, tc, src, read_gbs, wl_name):
+    """Roofline of one kernel: algorithmic bytes (or FLOPs) per launch over its mean
+    launch time (CUDA events on the launch stream), against the measured peaks."""
     k_ms, k_launch = prof[kern]
     k_avg_s = k_ms / k_launch / 1e3
-    launches = sum(c for _, c in prof.values())
     a_bytes, a_flops = alg["kern"].get(kern, (alg["step_bytes"], alg["step_flops"]))
-    # block-scaled MXF8 x MXF4 MMAs run at the FP8 rate: twice the measured BF16 peak (nominal 4.5 / 2.25)
+    # block-scaled MXF8 x MXF4/MXF8 MMAs run at the FP8 rate: twice the measured BF16 peak (nominal 4.5 / 2.25)
     tc_k = tc * 2 if kern.endswith("_mx") else tc
     t_hbm = a_bytes / (hbm * 1e9)
     t_tc = a_flops / (tc_k * 1e12)
@@ -367,44 +320,191 @@ def run_ours(args, world, rank, local):
     else:
         roof = {"bound": "tensor", "achieved": a_flops / k_avg_s / 1e12, "peak": tc_k, "unit": "TFLOP/s"}
     roof["frac"] = roof["achieved"] / roof["peak"]
-    roof["traffic"] = recorded_traffic(wl.name, kern)
+    roof["traffic"] = recorded_traffic(wl_name, kern)
     roof["kernel"] = kern
     roof["peak_source"] = (f"{src} (MEASURED_PEAKS.json)" if src == "measured" else "fallback") + \
         (", MXF8 = 2 x BF16" if kern.endswith("_mx") and roof["bound"] == "tensor" else "")
-    step_s = ms_per_step / 1e3
-    layer_roof = {"bytes": alg["step_bytes"], "flops": alg["step_flops"],
-                  "hbm_frac": alg["step_bytes"] / step_s / (hbm * 1e9),
-                  "tensor_frac": alg["step_flops"] / step_s / (tc * 1e12),
-                  "distinct_experts": alg["U"]}
+    if roof["bound"] == "hbm" and read_gbs:
+        roof["read_peak_gbs"] = read_gbs
+        roof["frac_of_read_peak"] = roof["achieved"] / read_gbs
+    roof["achieved_tflops"] = a_flops / k_avg_s / 1e12
+    roof["launch_ms"] = k_avg_s * 1e3
+    return roof
 
+
+def measure(wl, steps, warmup, world, local, read_gbs=None, flush_l2=False, e2e_steps=None, keep_weights=False):
+    """Create the layer for workload `wl`, time `steps` forwards (inputs resident),
+    attribute device time per kernel, time the host-buffer path, free the layer.
+    Returns (results, the generated inputs, the MXFP4 tensors or None); the expert
+    weights are dropped from the inputs unless keep_weights. Every rank runs the
+    same steps in the same order."""
+    import routed_expert_ffn_sqrtsoftplus_b200 as moe
+    T = wl.T
+    dev = torch.device("cuda", local)
+    d, mxq = build_layer(wl, dev)
+    layer = moe.MoELayer.from_layer(d, top_k=wl.k, max_tokens=T, route_scale=wl.route_scale,
+                                    swiglu_limit=wl.swiglu_limit, mx=mxq)
+    if not keep_weights:
+        mxq = None
+        for n in ("w1", "w3", "w2", "sh_w1", "sh_w3", "sh_w2"):
+            d.pop(n, None)               # the library holds its own copy
+        torch.cuda.empty_cache()
+    x = d["x"]
+    y = torch.empty_like(x)
+    stream = torch.cuda.current_stream()
+    _, idx, _ = layer.forward_with_routing(x)
+    torch.cuda.synchronize()
+    alg = algorithmic(wl, idx.cpu().numpy(), T)
+    for _ in range(warmup):
+        layer.forward(x, out=y)
+    torch.cuda.synchronize()
+    if layer.status() != moe.MOE_OK:
+        raise RuntimeError(f"device status after the warm-up of {wl.name}")
+
+    # ---- device-timed region
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        ev0.record(stream)
+        for _ in range(steps):
+            layer.forward(x, out=y)
+        ev1.record(stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    if layer.status() != moe.MOE_OK:
+        raise RuntimeError(f"device status after the timed steps of {wl.name}")
+    ms = max_over_ranks(ev0.elapsed_time(ev1), world)
+    res = {"value": weak_scaling_value(world, T, steps, ms), "ms_per_step": ms / steps, "steps": steps,
+           "warmup": warmup, "clocks": clk.summary()}
+
+    # ---- L2 flushed: a buffer twice the L2 size written before every timed step
+    if flush_l2:
+        junk = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
+        tot = 0.0
+        for i in range(steps):
+            junk.fill_(float(i))
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            layer.forward(x, out=y)
+            b.record(stream)
+            b.synchronize()
+            tot += a.elapsed_time(b)
+        tot = max_over_ranks(tot, world)
+        del junk
+        res["l2_flushed"] = {"value": weak_scaling_value(world, T, steps, tot), "ms_per_step": tot / steps,
+                             "flush": f"{2 * L2_BYTES >> 20} MiB written before each step, outside its events"}
+
+    # ---- per-kernel attribution: the same steps again with the library's CUDA events
+    # on the launch stream around every kernel (an event between two kernels also keeps
+    # the second from starting early, so these times are a little longer)
+    layer.profile_begin(steps)
+    for _ in range(steps):
+        layer.forward(x, out=y)
+    torch.cuda.synchronize()
+    prof = layer.profile_end()
+    if layer.status() != moe.MOE_OK:
+        raise RuntimeError(f"device status after the attribution pass of {wl.name}")
+
+    # ---- end to end through host buffers (pinned x in, y out, inside the timed region)
+    xh = x.cpu().pin_memory()
+    yh = torch.empty_like(xh).pin_memory()
+    n_e2e = e2e_steps or max(3, min(steps, 50))
+    for _ in range(2):
+        layer.forward_host(xh, yh)
+    torch.cuda.synchronize()
+    barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(n_e2e):
+        layer.forward_host(xh, yh)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
+    res["e2e"] = {"value": weak_scaling_value(world, T, n_e2e, e2e_ms), "unit": "tokens/s",
+                  "h2d_bytes_per_step": T * wl.H * 2, "d2h_bytes_per_step": T * wl.H * 2}
+
+    hbm, tc, tc_sus, src = peaks()
+    kern = max(prof, key=lambda n: prof[n][0])          # the kernel with the largest share of device time
+    res["roofline"] = kernel_roofline(kern, prof, alg, hbm, tc, src, read_gbs, wl.name)
+    res["kernel_rooflines"] = {n: kernel_roofline(n, prof, alg, hbm, tc, src, read_gbs, wl.name)
+                               for n in prof if n in alg["kern"] and n != kern}
+    step_s = res["ms_per_step"] / 1e3
+    res["layer_roofline"] = {"bytes": alg["step_bytes"], "flops": alg["step_flops"],
+                             "hbm_frac": alg["step_bytes"] / step_s / (hbm * 1e9),
+                             "tensor_frac": alg["step_flops"] / step_s / (tc * 1e12),
+                             "distinct_experts": alg["U"]}
+    if read_gbs:
+        res["layer_roofline"]["read_peak_frac"] = alg["step_bytes"] / step_s / (read_gbs * 1e9)
+    res["kernels_ms_per_step"] = {n: v[0] / steps for n, v in sorted(prof.items())}
+    res["gpu_launches"] = sum(c for _, c in prof.values())
+    res["config"] = {"workload": wl.name, "T": T, "hidden": wl.H, "inter": wl.I, "n_routed": wl.E,
+                     "n_shared": wl.n_shared, "top_k": wl.k, "route_scale": wl.route_scale,
+                     "swiglu_limit": wl.swiglu_limit, "expert_dtype": wl.expert_dtype,
+                     "parallelism": f"replicas x{world}",
+                     "l2": f"no flush: each step streams {alg['step_bytes'] / 1e9:.2f} GB of weights > 126 MB L2"}
+    res["dtype"] = {"bf16": "bf16", "mxfp4": "mxfp4xmxfp8", "mxfp8": "mxfp8xmxfp8"}.get(wl.expert_dtype,
+                                                                                      wl.expert_dtype)
+    layer.close()
+    return res, d, mxq
+
+
+# Workloads measured after the headline inside the same run (one layer at a time),
+# so the one JSON line covers the metric's BF16 and MXFP4 shapes.
+SECONDARY = ("flash_mxfp4_decode", "flash_mxfp4_prefill", "flash_prefill", "flash_mxfp8_decode",
+             "flash_mxfp8_prefill")
+
+
+def run_ours(args, world, rank, local):
+    from routed_expert_ffn_sqrtsoftplus_b200 import build
+    if rank == 0:
+        build.build()
+    barrier(world)
+    wl = workload_from_args(args)
+    dev = torch.device("cuda", local)
+    read_gbs = read_stream_peak(dev)
+    head, d, mxq = measure(wl, args.steps, args.warmup, world, local, read_gbs=read_gbs, flush_l2=True,
+                           keep_weights=rank == 0 and world == 1 and not args.no_cpu_baseline)
     out = {
         "metric": "MoE layer tokens/s (Flash shape, BF16 & MXFP4) + % of HBM/tensor roofline",
-        "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "bf16" if wl.expert_dtype == "bf16" else "mxfp4xmxfp8",
+        "value": head["value"], "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": head["ms_per_step"], "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": head["dtype"],
         "data": "synthetic (seeded N(0,1/fan_in) BF16 weights, N(0,1) tokens)",
-        "config": {"workload": wl.name, "T": T, "hidden": wl.H, "inter": wl.I, "n_routed": wl.E,
-                   "n_shared": wl.n_shared, "top_k": wl.k, "route_scale": wl.route_scale,
-                   "swiglu_limit": wl.swiglu_limit, "expert_dtype": wl.expert_dtype,
-                   "parallelism": f"replicas x{world}",
-                   "l2": f"no flush: each step streams {alg['step_bytes'] / 1e9:.2f} GB of weights > 126 MB L2"},
-        "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": T * wl.H * 2,
-                "d2h_bytes_per_step": T * wl.H * 2},
-        "roofline": roof,
-        "layer_roofline": layer_roof,
-        "kernels_ms_per_step": {n: v[0] / args.steps for n, v in sorted(prof.items())},
+        "config": head["config"],
+        "e2e": head["e2e"],
+        "roofline": head["roofline"],
+        "kernel_rooflines": head["kernel_rooflines"],
+        "layer_roofline": head["layer_roofline"],
+        "l2_flushed": head["l2_flushed"],
+        "kernels_ms_per_step": head["kernels_ms_per_step"],
         "kernel_timing": "per-kernel CUDA events in a second pass of the same steps (roofline, kernels_ms_per_step)",
-        "gpu_launches": launches,
-        "clocks": clk.summary(),
+        "gpu_launches": head["gpu_launches"],
+        "clocks": head["clocks"],
+        "read_stream_peak_gbs": read_gbs,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         rng = np.random.default_rng(0)
-        toks = rng.permutation(T)
+        toks = rng.permutation(wl.T)
         n, dt = cpu_oracle_sample(wl, d, mxq, toks, args.cpu_seconds)
         out["cpu_baseline"] = {"value": n / dt, "unit": "tokens/s", "cores": cpu_cores(), "kind": "oracle",
-                               "sample": f"{n} of {T} tokens, one at a time; each hit expert's weights copied "
+                               "sample": f"{n} of {wl.T} tokens, one at a time; each hit expert's weights copied "
                                          f"from the device and upcast to float64 inside the timing"}
-    layer.close()
+    del d, mxq
+    torch.cuda.empty_cache()
+    if not args.no_secondary and args.workload == "flash_decode" and not args.tokens and not args.experts:
+        sec = {}
+        steps, warm = min(args.steps, 30), max(3, min(args.warmup, 5))
+        for name in SECONDARY:
+            r, dd, _ = measure(synth.WORKLOADS[name], steps, warm, world, local, read_gbs=read_gbs)
+            del dd
+            torch.cuda.empty_cache()
+            sec[name] = {k: r[k] for k in ("value", "ms_per_step", "steps", "warmup", "dtype", "e2e", "roofline",
+                                           "kernel_rooflines", "layer_roofline", "kernels_ms_per_step",
+                                           "gpu_launches", "clocks", "config")}
+            sec[name]["unit"] = "tokens/s"
+        out["secondary"] = sec
     return out
 
 

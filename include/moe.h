@@ -39,7 +39,7 @@
 extern "C" {
 #endif
 
-#define MOE_ABI_VERSION 1
+#define MOE_ABI_VERSION 2
 
 #if defined(__GNUC__)
 #define MOE_API __attribute__((visibility("default")))
@@ -64,7 +64,10 @@ typedef enum {
 
 typedef enum {
   MOE_DT_BF16 = 0, /* routed experts in BF16 */
-  MOE_DT_MXFP4 = 1 /* routed experts in MXFP4: E2M1 values + one E8M0 scale per 32 along K */
+  MOE_DT_MXFP4 = 1, /* routed experts in MXFP4: E2M1 values + one E8M0 scale per 32 along K */
+  MOE_DT_MXFP8 = 2  /* routed experts in MXFP8: E4M3 values + one E8M0 scale per 32 along K (the
+                       checkpoint's "dtype": "fp8" and MAX's float8_e4m3fn encoding; the pages give no
+                       FP8 scale granularity, so the block is the family's E8M0-per-32) */
 } moe_expert_dtype;
 
 /*
@@ -102,6 +105,11 @@ typedef struct {
  *                  element 2j in the low nibble of byte j (float4_e2m1fnx2);
  *                  s1, s3 uint8 [E, I, H/32]; s2 uint8 [E, H, I/32]: E8M0
  *                  scales (2^(code-127)), code 0xFF (NaN) is rejected.
+ *   MXFP8 experts: w1, w3 uint8 [E, I, H]; w2 uint8 [E, H, I]: E4M3 codes
+ *                  (float8_e4m3fn); s1, s3, s2 E8M0 scales as for MXFP4.
+ *   With MXFP4 or MXFP8 experts the routed experts see the token and their
+ *   SwiGLU output quantised to MXFP8 (E4M3, E8M0 per 32, OCP MX v1.0 rule);
+ *   the router and the shared experts see BF16.
  *   sh_w1, sh_w3 BF16 [n_shared, I, H]; sh_w2 BF16 [n_shared, H, I] (always BF16)
  * Every pointer must be 16-byte aligned.
  */
@@ -185,6 +193,17 @@ MOE_API int32_t moe_abi_version(void);
 MOE_API moe_status moe_quantize_mxfp4(const void* src_bf16, int64_t rows, int32_t cols, uint8_t* dst_packed,
                               uint8_t* dst_scales, moe_stream_t stream);
 
+/*
+ * Quantise BF16 [rows, cols] (device) to MXFP8 with the same OCP MX v1.0 rule
+ * and E4M3 elements: per block of 32 along cols, scale = 2^(floor(log2(amax)) - 8)
+ * clamped to the E8M0 range (all-zero block: code 0), elements rounded to
+ * nearest-even E4M3 and saturated at +-448. Writes codes [rows, cols] and scales
+ * [rows, cols/32]. cols % 32 == 0; src and dst_codes 16-byte aligned. Enqueued
+ * on `stream`.
+ */
+MOE_API moe_status moe_quantize_mxfp8(const void* src_bf16, int64_t rows, int32_t cols, uint8_t* dst_codes,
+                              uint8_t* dst_scales, moe_stream_t stream);
+
 /* Internal buffers of the LAST forward that moe_inspect can copy out. */
 typedef enum {
   MOE_BUF_LOGITS = 0,   /* fp32 [T, E] router logits before refinement (approximate) */
@@ -195,11 +214,11 @@ typedef enum {
   MOE_BUF_PERM = 5,     /* int32 [T*k] flat slot t*k+j of each routed row (expert-major) */
   MOE_BUF_INV = 6,      /* int32 [T*k] row of each flat slot */
   MOE_BUF_H = 7,        /* BF16 [T*k + n_shared*T, I] SwiGLU output rows (group order) */
-  MOE_BUF_XQ = 8,       /* MXFP4 layers: uint8 E4M3 [T*k, H], MXFP8 codes of the routed rows (perm order) */
-  MOE_BUF_XQ_SCALES = 9, /* MXFP4 layers: their E8M0 scales, packed in 512-byte atoms per token tile */
-  MOE_BUF_HQ = 10,       /* MXFP4 layers: uint8 E4M3 [T*k, I], MXFP8 codes of the routed SwiGLU rows
+  MOE_BUF_XQ = 8,       /* MXFP4 / MXFP8 layers: uint8 E4M3 [T*k, H], MXFP8 codes of the routed rows (perm order) */
+  MOE_BUF_XQ_SCALES = 9, /* MXFP4 / MXFP8 layers: their E8M0 scales, packed in 512-byte atoms per token tile */
+  MOE_BUF_HQ = 10,       /* MXFP4 / MXFP8 layers: uint8 E4M3 [T*k, I], MXFP8 codes of the routed SwiGLU rows
                             (group order, as MOE_BUF_H) */
-  MOE_BUF_HQ_SCALES = 11 /* MXFP4 layers: their E8M0 scales in 512-byte atoms, one per (down-GEMM
+  MOE_BUF_HQ_SCALES = 11 /* MXFP4 / MXFP8 layers: their E8M0 scales in 512-byte atoms, one per (down-GEMM
                             token tile nt, 128-wide slice c of I): row n of the tile, block b of the
                             slice at byte (nt * I/128 + c) * 512 + (n % 32) * 16 + (n / 32) * 4 + b.
                             Token tiles: each routed group's rows cut into tiles of 32 rows when

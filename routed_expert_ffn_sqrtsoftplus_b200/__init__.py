@@ -24,7 +24,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "_lib", "libmoe_b200.so")
 
 MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_OOM, MOE_ERR_CUDA, MOE_ERR_TIMEOUT, MOE_ERR_DEVICE = range(7)
-MOE_DT_BF16, MOE_DT_MXFP4 = 0, 1
+MOE_DT_BF16, MOE_DT_MXFP4, MOE_DT_MXFP8 = 0, 1, 2
 
 # moe_buffer ids
 (BUF_LOGITS, BUF_TOPK_IDX, BUF_TOPK_W, BUF_COUNTS, BUF_OFFSETS, BUF_PERM, BUF_INV, BUF_H, BUF_XQ, BUF_XQ_SCALES,
@@ -33,7 +33,7 @@ MOE_DT_BF16, MOE_DT_MXFP4 = 0, 1
 EXPORTED = ("moe_create", "moe_forward", "moe_forward_host", "moe_get_status", "moe_status_string",
             "moe_destroy", "moe_abi_version", "moe_quantize_mxfp4", "moe_inspect", "moe_set_wait_timeout",
             "moe_selftest_wait_timeout", "moe_get_info", "moe_profile_begin", "moe_profile_end",
-            "moe_num_kernel_kinds", "moe_kernel_name", "moe_route_noalloc")
+            "moe_num_kernel_kinds", "moe_kernel_name", "moe_route_noalloc", "moe_quantize_mxfp8")
 
 
 class MoEError(RuntimeError):
@@ -81,6 +81,7 @@ def lib() -> ctypes.CDLL:
             "moe_destroy": (None, [P]),
             "moe_abi_version": (I32, []),
             "moe_quantize_mxfp4": (I32, [P, I64, I32, P, P, P]),
+            "moe_quantize_mxfp8": (I32, [P, I64, I32, P, P, P]),
             "moe_inspect": (I32, [P, I32, P, ctypes.c_size_t, P]),
             "moe_set_wait_timeout": (I32, [P, U64]),
             "moe_selftest_wait_timeout": (I32, [P, U64, P]),
@@ -149,6 +150,18 @@ def quantize_mxfp4(w: torch.Tensor, stream=None):
     return packed, scales
 
 
+def quantize_mxfp8(w: torch.Tensor, stream=None):
+    """BF16 [..., K] (CUDA) -> (E4M3 codes uint8 [..., K], E8M0 uint8 [..., K/32]) on the device."""
+    _need(w, "w", torch.bfloat16)
+    K = w.shape[-1]
+    rows = w.numel() // K
+    codes = torch.empty(w.shape, dtype=torch.uint8, device=w.device)
+    scales = torch.empty(w.shape[:-1] + (K // 32,), dtype=torch.uint8, device=w.device)
+    _check(lib().moe_quantize_mxfp8(_ptr(w), rows, K, _ptr(codes), _ptr(scales), _stream(stream)),
+           "moe_quantize_mxfp8")
+    return codes, scales
+
+
 class MoELayer:
     """One routed-expert FFN layer resident on the current CUDA device."""
 
@@ -169,16 +182,17 @@ class MoELayer:
             _need(w1, "w1", torch.bfloat16, (E, I, H)); _need(w3, "w3", torch.bfloat16, (E, I, H))
             _need(w2, "w2", torch.bfloat16, (E, H, I))
             dt = MOE_DT_BF16
-        elif expert_dtype == "mxfp4":
-            _need(w1, "w1", torch.uint8, (E, I, H // 2)); _need(w3, "w3", torch.uint8, (E, I, H // 2))
-            _need(w2, "w2", torch.uint8, (E, H, I // 2))
+        elif expert_dtype in ("mxfp4", "mxfp8"):
+            div = 2 if expert_dtype == "mxfp4" else 1
+            _need(w1, "w1", torch.uint8, (E, I, H // div)); _need(w3, "w3", torch.uint8, (E, I, H // div))
+            _need(w2, "w2", torch.uint8, (E, H, I // div))
             for n, t, shp in (("s1", s1, (E, I, H // 32)), ("s3", s3, (E, I, H // 32)), ("s2", s2, (E, H, I // 32))):
                 if t is None:
-                    raise ValueError(f"{n} is required for MXFP4 experts")
+                    raise ValueError(f"{n} is required for {expert_dtype} experts")
                 _need(t, n, torch.uint8, shp)
-            dt = MOE_DT_MXFP4
+            dt = MOE_DT_MXFP4 if expert_dtype == "mxfp4" else MOE_DT_MXFP8
         else:
-            raise ValueError("expert_dtype must be 'bf16' or 'mxfp4'")
+            raise ValueError("expert_dtype must be 'bf16', 'mxfp4' or 'mxfp8'")
         if S > 0:
             _need(sh_w1, "sh_w1", torch.bfloat16, (S, I, H)); _need(sh_w3, "sh_w3", torch.bfloat16, (S, I, H))
             _need(sh_w2, "sh_w2", torch.bfloat16, (S, H, I))
@@ -283,7 +297,8 @@ class MoELayer:
                    swiglu_limit: float = 10.0, mx: Optional[dict] = None, stream=None) -> "MoELayer":
         """Build from a dict of tensors (x ignored): wg, bias, w1, w3, w2, sh_w1, sh_w3, sh_w2.
 
-        With ``mx`` = dict(w1, s1, w3, s3, w2, s2) of MXFP4 tensors the routed experts are MXFP4.
+        With ``mx`` = dict(w1, s1, w3, s3, w2, s2) of MXFP4 (packed, w1 [E, I, H/2]) or
+        MXFP8 (w1 [E, I, H]) tensors the routed experts are stored in that format.
         """
         E, I, H = layer["w1"].shape
         S = layer["sh_w1"].shape[0] if layer.get("sh_w1") is not None else 0
@@ -293,5 +308,6 @@ class MoELayer:
                   swiglu_limit=swiglu_limit, stream=stream)
         if mx is None:
             return cls(w1=layer["w1"], w3=layer["w3"], w2=layer["w2"], expert_dtype="bf16", **kw)
+        fmt = "mxfp8" if mx["w1"].shape[-1] == H else "mxfp4"
         return cls(w1=mx["w1"], w3=mx["w3"], w2=mx["w2"], s1=mx["s1"], s3=mx["s3"], s2=mx["s2"],
-                   expert_dtype="mxfp4", **kw)
+                   expert_dtype=fmt, **kw)

@@ -116,7 +116,8 @@ struct moe_handle {
   bool wide_ok = false;         // H % 256 == 0
 
   // MXFP4 routed experts (expert_dtype == MOE_DT_MXFP4)
-  bool mx = false;
+  bool mx = false;              // routed experts block-scaled (MXFP4 or MXFP8)
+  bool a8 = false;              // ... and MXFP8 (E4M3 weights, one byte per value)
   uint8_t* w13q = nullptr;      // packed E2M1, gate/up tile order
   uint8_t* w2q = nullptr;       // packed E2M1
   uint8_t* sfa13 = nullptr;     // scale atoms of W1|W3
@@ -201,7 +202,8 @@ moe_status validate_config(const moe_config* c) {
   if (c->hidden % 128 != 0 || c->inter % 128 != 0) return MOE_ERR_UNSUPPORTED;
   if (c->n_routed > 512 || c->top_k > 32 || c->n_shared > 4 || c->max_tokens > 65536) return MOE_ERR_UNSUPPORTED;
   if (c->hidden > 16384 || c->inter > 16384) return MOE_ERR_UNSUPPORTED;
-  if (c->expert_dtype != MOE_DT_BF16 && c->expert_dtype != MOE_DT_MXFP4) return MOE_ERR_INVALID_ARG;
+  if (c->expert_dtype != MOE_DT_BF16 && c->expert_dtype != MOE_DT_MXFP4 && c->expert_dtype != MOE_DT_MXFP8)
+    return MOE_ERR_INVALID_ARG;
   return MOE_OK;
 }
 
@@ -245,7 +247,8 @@ moe_status moe_create(const moe_config* cfg, const moe_weights* w, moe_stream_t 
   if (cfg == nullptr || w == nullptr) return MOE_ERR_INVALID_ARG;
   moe_status st = validate_config(cfg);
   if (st != MOE_OK) return st;
-  const bool mx = cfg->expert_dtype == MOE_DT_MXFP4;
+  const bool mx = cfg->expert_dtype == MOE_DT_MXFP4 || cfg->expert_dtype == MOE_DT_MXFP8;
+  const bool a8 = cfg->expert_dtype == MOE_DT_MXFP8;
   const void* req[] = {w->router_w, w->w1, w->w3, w->w2};
   for (const void* p : req)
     if (p == nullptr || !aligned16(p)) return MOE_ERR_INVALID_ARG;
@@ -272,6 +275,7 @@ moe_status moe_create(const moe_config* cfg, const moe_weights* w, moe_stream_t 
   if (h == nullptr) return MOE_ERR_OOM;
   h->cfg = *cfg;
   h->mx = mx;
+  h->a8 = a8;
   if (cudaGetDevice(&h->device) != cudaSuccess ||
       cudaDeviceGetAttribute(&h->num_sms, cudaDevAttrMultiProcessorCount, h->device) != cudaSuccess ||
       gemm_set_attributes() != cudaSuccess || gemm_mx_set_attributes() != cudaSuccess ||
@@ -301,8 +305,8 @@ moe_status moe_create(const moe_config* cfg, const moe_weights* w, moe_stream_t 
     ok = ok && h->alloc(&h->w2, (E + S) * H * I * 2, wb);
     ok = ok && h->alloc(&h->xp, Tm * k * H * 2, ws);
   } else {
-    ok = ok && h->alloc(&h->w13q, E * 2 * I * H / 2, wb);
-    ok = ok && h->alloc(&h->w2q, E * H * I / 2, wb);
+    ok = ok && h->alloc(&h->w13q, E * 2 * I * (a8 ? H : H / 2), wb);
+    ok = ok && h->alloc(&h->w2q, E * H * (a8 ? I : I / 2), wb);
     ok = ok && h->alloc(&h->sfa13, E * (I / 128) * (H / 128) * 1024, wb);
     ok = ok && h->alloc(&h->sfa2, E * (H / 128) * (I / 128) * 512, wb);
     if (S > 0) {
@@ -368,8 +372,8 @@ moe_status moe_create(const moe_config* cfg, const moe_weights* w, moe_stream_t 
   } else {
     err |= cudaMemsetAsync(h->bad, 0, 16, s) != cudaSuccess;
     err |= launch_repack_w13_bytes(w->w1, w->w3, nullptr, nullptr, static_cast<int>(E), 0, static_cast<int>(I),
-                                   static_cast<int>(H / 2), h->w13q, s) != cudaSuccess;
-    err |= cudaMemcpyAsync(h->w2q, w->w2, E * H * I / 2, cudaMemcpyDeviceToDevice, s) != cudaSuccess;
+                                   static_cast<int>(a8 ? H : H / 2), h->w13q, s) != cudaSuccess;
+    err |= cudaMemcpyAsync(h->w2q, w->w2, E * H * (a8 ? I : I / 2), cudaMemcpyDeviceToDevice, s) != cudaSuccess;
     err |= launch_sf_atoms(w->s1, w->s3, static_cast<int>(E), static_cast<int>(I), static_cast<int>(H), h->sfa13,
                            h->bad, s) != cudaSuccess;
     err |= launch_sf_atoms(w->s2, nullptr, static_cast<int>(E), static_cast<int>(H), static_cast<int>(I), h->sfa2,
@@ -384,11 +388,13 @@ moe_status moe_create(const moe_config* cfg, const moe_weights* w, moe_stream_t 
       // routed ones, whose tiles are 256 rows of W2 when H % 256 == 0
       if (H % 256 == 0) err |= !make_tmap_bf16(&h->tm_w2shw, h->w2sh, S * H, I, 256);
     }
-    err |= !make_tmap(&h->tm_w13q, h->w13q, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, E * 2 * I, H, H / 2, 128, 256);
-    err |= !make_tmap(&h->tm_w2q, h->w2q, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, E * H, I, I / 2, 128, 128);
+    // MXFP4: packed E2M1 pairs, unpacked by the TMA to one value per byte in shared
+    // memory; MXFP8: E4M3 bytes as stored. Either way 128 values = 128 smem bytes per row.
+    const CUtensorMapDataType wdt = a8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B;
+    err |= !make_tmap(&h->tm_w13q, h->w13q, wdt, E * 2 * I, H, a8 ? H : H / 2, 128, 256);
+    err |= !make_tmap(&h->tm_w2q, h->w2q, wdt, E * H, I, a8 ? I : I / 2, 128, 128);
     h->wide_ok = H % 256 == 0;
-    if (h->wide_ok)
-      err |= !make_tmap(&h->tm_w2qw, h->w2q, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, E * H, I, I / 2, 128, 256);
+    if (h->wide_ok) err |= !make_tmap(&h->tm_w2qw, h->w2q, wdt, E * H, I, a8 ? I : I / 2, 128, 256);
     err |= !make_tmap(&h->tm_xq, h->xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, Tm * k, H, H, 128, 32);
     err |= !make_tmap(&h->tm_hq, h->hq, CU_TENSOR_MAP_DATA_TYPE_UINT8, Tm * k, I, I, 128, 32);
   }
@@ -619,7 +625,7 @@ moe_status moe_forward(moe_handle* h, const void* x, int32_t T, void* y, int32_t
     g.status = h->status;
     g.timeout_ns = h->timeout_ns;
     h->prof_mark(kKGateUpMx, s);
-    MOE_TRY_CUDA(launch_gemm_mx_gateup(h->tm_w13q, h->tm_xq, g, bn_mx, h->num_sms, s));
+    MOE_TRY_CUDA(launch_gemm_mx_gateup(h->tm_w13q, h->tm_xq, g, bn_mx, h->num_sms, s, h->a8));
     h->prof_done(s);
     // 4b. shared experts' gate/up in BF16. With few tokens the shared expert has
     // only I/128 weight tiles: split K so every SM streams part of it, then sum
@@ -691,7 +697,8 @@ moe_status moe_forward(moe_handle* h, const void* x, int32_t T, void* y, int32_t
     d.status = h->status;
     d.timeout_ns = h->timeout_ns;
     h->prof_mark(kKDownMx, s);
-    MOE_TRY_CUDA(launch_gemm_mx_down(wide_mx ? h->tm_w2qw : h->tm_w2q, h->tm_hq, d, bn_mx, h->num_sms, s, wide_mx));
+    MOE_TRY_CUDA(
+        launch_gemm_mx_down(wide_mx ? h->tm_w2qw : h->tm_w2q, h->tm_hq, d, bn_mx, h->num_sms, s, wide_mx, h->a8));
     h->prof_done(s);
     // 5b. shared experts' down in BF16 (split K for few tokens; the combine sums the slices)
     if (sh_split) {
@@ -797,6 +804,17 @@ moe_status moe_quantize_mxfp4(const void* src_bf16, int64_t rows, int32_t cols, 
   if (src_bf16 == nullptr || dst_packed == nullptr || dst_scales == nullptr) return MOE_ERR_INVALID_ARG;
   if (!aligned16(src_bf16) || !aligned16(dst_packed)) return MOE_ERR_INVALID_ARG;
   MOE_TRY_CUDA(launch_quantize_mxfp4(src_bf16, rows, cols, dst_packed, dst_scales,
+                                     reinterpret_cast<cudaStream_t>(stream)));
+  return MOE_OK;
+}
+
+moe_status moe_quantize_mxfp8(const void* src_bf16, int64_t rows, int32_t cols, uint8_t* dst_codes,
+                              uint8_t* dst_scales, moe_stream_t stream) {
+  if (rows < 0 || cols <= 0 || cols % 32 != 0) return MOE_ERR_INVALID_ARG;
+  if (rows == 0) return MOE_OK;
+  if (src_bf16 == nullptr || dst_codes == nullptr || dst_scales == nullptr) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(src_bf16) || !aligned16(dst_codes)) return MOE_ERR_INVALID_ARG;
+  MOE_TRY_CUDA(launch_quantize_mxfp8(src_bf16, rows, cols, dst_codes, dst_scales,
                                      reinterpret_cast<cudaStream_t>(stream)));
   return MOE_OK;
 }

@@ -215,6 +215,11 @@ __host__ __device__ constexpr uint32_t idesc_mx_e2m1_e4m3(uint32_t M, uint32_t N
   return (sfb_id << 4) | (5u << 7) | (0u << 10) | ((N >> 3) << 17) | (1u << 23) | ((M >> 4) << 24) |
          (sfa_id << 29);
 }
+// The same with A in E4M3 (format 0): MXFP8 weights against MXFP8 activations.
+__host__ __device__ constexpr uint32_t idesc_mx_e4m3_e4m3(uint32_t M, uint32_t N, uint32_t sfa_id, uint32_t sfb_id) {
+  return (sfb_id << 4) | (0u << 7) | (0u << 10) | ((N >> 3) << 17) | (1u << 23) | ((M >> 4) << 24) |
+         (sfa_id << 29);
+}
 
 // E8M0 scale code and the exact reciprocal scale for an MX block with the given
 // amax (OCP MX v1.0: shared exponent floor(log2 amax) - emax, clamped to the

@@ -1,11 +1,13 @@
-// Grouped expert GEMMs for MXFP4 routed experts on tcgen05 block-scaled MMAs.
+// Grouped expert GEMMs for block-scaled routed experts on tcgen05 block-scaled MMAs.
 //
 // Routed expert weights are MXFP4 (E2M1 values, one E8M0 scale per 32 along K;
-// DeepSeek V4.1 config "expert_dtype": "fp4", MAX encoding float4_e2m1fnx2) and
-// the activations they meet are MXFP8 (E4M3, one E8M0 scale per 32), so every
-// MMA is tcgen05.mma.kind::mxf8f6f4.block_scale: A = 128 weight rows (E2M1,
-// unpacked to one byte per value in shared memory by the 16U4_ALIGN16B TMA
-// type), B = token rows (E4M3), scale factors in TMEM, fp32 accumulation.
+// DeepSeek V4.1 config "expert_dtype": "fp4", MAX encoding float4_e2m1fnx2) or
+// MXFP8 (E4M3 values, the same scales; MAX encoding float8_e4m3fn) and the
+// activations they meet are MXFP8 (E4M3, one E8M0 scale per 32), so every MMA
+// is tcgen05.mma.kind::mxf8f6f4.block_scale: A = 128 weight rows (E2M1, unpacked
+// to one byte per value in shared memory by the 16U4_ALIGN16B TMA type, or E4M3
+// loaded as it is stored), B = token rows (E4M3), scale factors in TMEM, fp32
+// accumulation.
 //
 // Same persistent, warp-specialised structure as the BF16 kernel (warp 0 TMA,
 // warp 1 MMA, 8 epilogue warps, two per TMEM lane quarter taking interleaved
@@ -45,12 +47,14 @@ constexpr int pow2_at_least(int v, int lo) {
 
 // kWide (down GEMM): a tile covers 256 rows of W2, two 128-row MMAs sharing the
 // token tile, like the gate/up tile's W1 and W3 halves.
-template <bool kGateUp, bool kWide, int BN, int kStages>
+// kAF8: A (the weights) is E4M3, one byte per value in HBM and in shared memory;
+// otherwise E2M1, packed two per byte in HBM and unpacked to one per byte by the TMA.
+template <bool kGateUp, bool kWide, int BN, int kStages, bool kAF8>
 struct MxCfg {
   static constexpr bool kTwoA = kGateUp || kWide;       // two 128-row MMAs per K step
   static constexpr int kARows = kTwoA ? 256 : 128;
-  static constexpr int kABytes = kARows * 128;          // unpacked E2M1 in shared memory
-  static constexpr int kATx = kARows * 64;              // packed bytes the TMA moves
+  static constexpr int kABytes = kARows * 128;          // one byte per value in shared memory
+  static constexpr int kATx = kAF8 ? kABytes : kARows * 64;  // bytes the TMA moves from HBM
   static constexpr int kBBytes = BN * 128;
   static constexpr int kSfaBytes = kTwoA ? 2 * kAtomBytes : kAtomBytes;
   static constexpr int kSfBytes = kSfaBytes + kAtomBytes;
@@ -99,11 +103,11 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, co
   }
 }
 
-template <bool kGateUp, bool kWide, int BN, int kStages>
+template <bool kGateUp, bool kWide, int BN, int kStages, bool kAF8>
 __global__ void __launch_bounds__(kThreads, 1)
     grouped_gemm_mx_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                            const MxGemmArgs args) {
-  using C = MxCfg<kGateUp, kWide, BN, kStages>;
+  using C = MxCfg<kGateUp, kWide, BN, kStages, kAF8>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
@@ -238,7 +242,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_cp_32x128b_x4(sfb_col, sdesc_plain(sf_addr + C::kSfaBytes));
 #pragma unroll
           for (uint32_t k = 0; k < kBK / 32; ++k) {
-            const uint32_t idesc = idesc_mx_e2m1_e4m3(128, n_mma, k, k);
+            const uint32_t idesc = kAF8 ? idesc_mx_e4m3_e4m3(128, n_mma, k, k) : idesc_mx_e2m1_e4m3(128, n_mma, k, k);
             const uint64_t bdesc = sdesc_sw128(b_addr + k * 32);
             const uint32_t accum = (kb | k) != 0;
             umma_mx(d, sdesc_sw128(a_addr + k * 32), bdesc, idesc, sf_cols | (k << 30), sfb_col | (k << 30),
@@ -363,17 +367,17 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <bool kGateUp, bool kWide, int BN, int kStages>
+template <bool kGateUp, bool kWide, int BN, int kStages, bool kAF8>
 cudaError_t set_attr() {
-  return cudaFuncSetAttribute(grouped_gemm_mx_kernel<kGateUp, kWide, BN, kStages>,
+  return cudaFuncSetAttribute(grouped_gemm_mx_kernel<kGateUp, kWide, BN, kStages, kAF8>,
                               cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              MxCfg<kGateUp, kWide, BN, kStages>::kSmemBytes);
+                              MxCfg<kGateUp, kWide, BN, kStages, kAF8>::kSmemBytes);
 }
 
-template <bool kGateUp, bool kWide, int BN, int kStages>
+template <bool kGateUp, bool kWide, int BN, int kStages, bool kAF8>
 cudaError_t launch(const CUtensorMap& tmA, const CUtensorMap& tmB, const MxGemmArgs& a, int grid, cudaStream_t s) {
-  grouped_gemm_mx_kernel<kGateUp, kWide, BN, kStages>
-      <<<grid, kThreads, MxCfg<kGateUp, kWide, BN, kStages>::kSmemBytes, s>>>(tmA, tmB, a);
+  grouped_gemm_mx_kernel<kGateUp, kWide, BN, kStages, kAF8>
+      <<<grid, kThreads, MxCfg<kGateUp, kWide, BN, kStages, kAF8>::kSmemBytes, s>>>(tmA, tmB, a);
   return cudaGetLastError();
 }
 
@@ -387,28 +391,30 @@ template <int BN>
 constexpr int kOneAStages = mx_ring_fit(128 * 128, BN * 128, 2 * kAtomBytes);  // 32: 10, 64: 9, 96: 7
 constexpr bool kExtraWidth = kBnMxLarge != 32 && kBnMxLarge != 64;
 
-template <bool kGateUp, bool kWide>
+template <bool kGateUp, bool kWide, bool kAF8>
 cudaError_t set_attrs() {
   constexpr bool two = kGateUp || kWide;
   cudaError_t e;
-  if ((e = set_attr<kGateUp, kWide, 32, two ? kTwoAStages<32> : kOneAStages<32>>()) != cudaSuccess) return e;
-  if ((e = set_attr<kGateUp, kWide, 64, two ? kTwoAStages<64> : kOneAStages<64>>()) != cudaSuccess) return e;
+  if ((e = set_attr<kGateUp, kWide, 32, two ? kTwoAStages<32> : kOneAStages<32>, kAF8>()) != cudaSuccess) return e;
+  if ((e = set_attr<kGateUp, kWide, 64, two ? kTwoAStages<64> : kOneAStages<64>, kAF8>()) != cudaSuccess) return e;
   if constexpr (kExtraWidth)
-    if ((e = set_attr<kGateUp, kWide, kBnMxLarge, two ? kTwoAStages<kBnMxLarge> : kOneAStages<kBnMxLarge>>()) !=
-        cudaSuccess)
+    if ((e = set_attr<kGateUp, kWide, kBnMxLarge, two ? kTwoAStages<kBnMxLarge> : kOneAStages<kBnMxLarge>,
+                      kAF8>()) != cudaSuccess)
       return e;
   return cudaSuccess;
 }
 
-template <bool kGateUp, bool kWide>
+template <bool kGateUp, bool kWide, bool kAF8>
 cudaError_t launch_any(const CUtensorMap& tmA, const CUtensorMap& tmB, const MxGemmArgs& a, int bn, int grid,
                        cudaStream_t s) {
   constexpr bool two = kGateUp || kWide;
-  if (bn == 32) return launch<kGateUp, kWide, 32, two ? kTwoAStages<32> : kOneAStages<32>>(tmA, tmB, a, grid, s);
-  if (bn == 64) return launch<kGateUp, kWide, 64, two ? kTwoAStages<64> : kOneAStages<64>>(tmA, tmB, a, grid, s);
+  if (bn == 32)
+    return launch<kGateUp, kWide, 32, two ? kTwoAStages<32> : kOneAStages<32>, kAF8>(tmA, tmB, a, grid, s);
+  if (bn == 64)
+    return launch<kGateUp, kWide, 64, two ? kTwoAStages<64> : kOneAStages<64>, kAF8>(tmA, tmB, a, grid, s);
   if constexpr (kExtraWidth)
     if (bn == kBnMxLarge)
-      return launch<kGateUp, kWide, kBnMxLarge, two ? kTwoAStages<kBnMxLarge> : kOneAStages<kBnMxLarge>>(
+      return launch<kGateUp, kWide, kBnMxLarge, two ? kTwoAStages<kBnMxLarge> : kOneAStages<kBnMxLarge>, kAF8>(
           tmA, tmB, a, grid, s);
   return cudaErrorInvalidValue;
 }
@@ -417,20 +423,28 @@ cudaError_t launch_any(const CUtensorMap& tmA, const CUtensorMap& tmB, const MxG
 
 cudaError_t gemm_mx_set_attributes() {
   cudaError_t e;
-  if ((e = set_attrs<true, false>()) != cudaSuccess) return e;
-  if ((e = set_attrs<false, false>()) != cudaSuccess) return e;
-  if ((e = set_attrs<false, true>()) != cudaSuccess) return e;
+  if ((e = set_attrs<true, false, false>()) != cudaSuccess) return e;
+  if ((e = set_attrs<false, false, false>()) != cudaSuccess) return e;
+  if ((e = set_attrs<false, true, false>()) != cudaSuccess) return e;
+  if ((e = set_attrs<true, false, true>()) != cudaSuccess) return e;
+  if ((e = set_attrs<false, false, true>()) != cudaSuccess) return e;
+  if ((e = set_attrs<false, true, true>()) != cudaSuccess) return e;
   return cudaSuccess;
 }
 
 cudaError_t launch_gemm_mx_gateup(const CUtensorMap& tmA, const CUtensorMap& tmB, const MxGemmArgs& a, int bn,
-                                  int grid, cudaStream_t s) {
-  return launch_any<true, false>(tmA, tmB, a, bn, grid, s);
+                                  int grid, cudaStream_t s, bool a_fp8) {
+  return a_fp8 ? launch_any<true, false, true>(tmA, tmB, a, bn, grid, s)
+               : launch_any<true, false, false>(tmA, tmB, a, bn, grid, s);
 }
 
 cudaError_t launch_gemm_mx_down(const CUtensorMap& tmA, const CUtensorMap& tmB, const MxGemmArgs& a, int bn,
-                                int grid, cudaStream_t s, bool wide) {
-  return wide ? launch_any<false, true>(tmA, tmB, a, bn, grid, s) : launch_any<false, false>(tmA, tmB, a, bn, grid, s);
+                                int grid, cudaStream_t s, bool wide, bool a_fp8) {
+  if (a_fp8)
+    return wide ? launch_any<false, true, true>(tmA, tmB, a, bn, grid, s)
+                : launch_any<false, false, true>(tmA, tmB, a, bn, grid, s);
+  return wide ? launch_any<false, true, false>(tmA, tmB, a, bn, grid, s)
+              : launch_any<false, false, false>(tmA, tmB, a, bn, grid, s);
 }
 
 }  // namespace moe

@@ -182,11 +182,12 @@ struct MxGemmArgs {
   unsigned long long timeout_ns;
 };
 cudaError_t gemm_mx_set_attributes();
+// a_fp8: the weights are MXFP8 (E4M3, one byte per value) instead of MXFP4
 cudaError_t launch_gemm_mx_gateup(const CUtensorMap& tmA, const CUtensorMap& tmB, const MxGemmArgs& a, int bn,
-                                  int grid, cudaStream_t s);
+                                  int grid, cudaStream_t s, bool a_fp8);
 // wide: tiles of 256 W2 rows (two 128-row MMAs per K step); the tile list's m tiles are H / 256
 cudaError_t launch_gemm_mx_down(const CUtensorMap& tmA, const CUtensorMap& tmB, const MxGemmArgs& a, int bn,
-                                int grid, cudaStream_t s, bool wide = false);
+                                int grid, cudaStream_t s, bool wide, bool a_fp8);
 // x rows of the routed slots -> MXFP8: xq[row] = E4M3 codes of x[perm[row] / k], scale
 // atoms by gate/up token tile.
 cudaError_t launch_quant_gather_mx(const void* x, const int32_t* perm, const int32_t* idx, const int32_t* off,
@@ -212,6 +213,8 @@ cudaError_t launch_swiglu_reduce(const float* parts, int n_parts, int T, int I, 
 
 // ---- MX utilities
 cudaError_t launch_quantize_mxfp4(const void* src, int64_t rows, int cols, uint8_t* packed, uint8_t* scales,
+                                  cudaStream_t s);
+cudaError_t launch_quantize_mxfp8(const void* src, int64_t rows, int cols, uint8_t* codes, uint8_t* scales,
                                   cudaStream_t s);
 
 // ---- repack

@@ -173,6 +173,46 @@ __global__ void __launch_bounds__(256)
   scales[b] = static_cast<uint8_t>(code);
 }
 
+// One thread per 32-element block: OCP MX rule with E4M3 elements (MXFP8), the
+// same rule the activations use, conversion rounding to nearest-even and
+// saturating at +-448.
+__global__ void __launch_bounds__(256)
+    quantize_mxfp8_kernel(const uint4* __restrict__ src, int64_t nblocks, uint4* __restrict__ codes,
+                          uint8_t* __restrict__ scales) {
+  const int64_t b = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (b >= nblocks) return;
+  float v[32];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const uint4 u = __ldg(src + b * 4 + q);
+    const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float2 f = __bfloat1622float2(p[i]);
+      v[q * 8 + 2 * i] = f.x;
+      v[q * 8 + 2 * i + 1] = f.y;
+    }
+  }
+  float amax = 0.f;
+#pragma unroll
+  for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(v[i]));
+  int code;
+  float inv;
+  mx_scale(amax, 8, code, inv);
+  uint32_t w[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const __nv_fp8x2_storage_t lo =
+        __nv_cvt_float2_to_fp8x2(make_float2(v[4 * i] * inv, v[4 * i + 1] * inv), __NV_SATFINITE, __NV_E4M3);
+    const __nv_fp8x2_storage_t hi =
+        __nv_cvt_float2_to_fp8x2(make_float2(v[4 * i + 2] * inv, v[4 * i + 3] * inv), __NV_SATFINITE, __NV_E4M3);
+    w[i] = static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
+  }
+  codes[b * 2] = make_uint4(w[0], w[1], w[2], w[3]);
+  codes[b * 2 + 1] = make_uint4(w[4], w[5], w[6], w[7]);
+  scales[b] = static_cast<uint8_t>(code);
+}
+
 __global__ void wait_timeout_probe_kernel(int* status, unsigned long long timeout_ns) {
   __shared__ uint64_t bar;
   if (threadIdx.x == 0) {
@@ -237,6 +277,15 @@ cudaError_t launch_quantize_mxfp4(const void* src, int64_t rows, int cols, uint8
   if (nblocks == 0) return cudaSuccess;
   quantize_mxfp4_kernel<<<static_cast<unsigned>((nblocks + 255) / 256), 256, 0, s>>>(
       static_cast<const uint4*>(src), nblocks, reinterpret_cast<uint4*>(packed), scales);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_quantize_mxfp8(const void* src, int64_t rows, int cols, uint8_t* codes, uint8_t* scales,
+                                  cudaStream_t s) {
+  const int64_t nblocks = rows * (cols / 32);
+  if (nblocks == 0) return cudaSuccess;
+  quantize_mxfp8_kernel<<<static_cast<unsigned>((nblocks + 255) / 256), 256, 0, s>>>(
+      static_cast<const uint4*>(src), nblocks, reinterpret_cast<uint4*>(codes), scales);
   return cudaGetLastError();
 }
 

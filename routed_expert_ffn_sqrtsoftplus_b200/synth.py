@@ -13,14 +13,17 @@ DeepSeek-V4-Pro config paragraph; distributions as stated per workload):
   flash_prefill       T=8192, same layer as flash_decode
   flash_mxfp4_decode  T=16,   same layer, routed experts to be stored as MXFP4
   flash_mxfp4_prefill T=4096, same
+  flash_mxfp8_decode  T=32,   same layer, routed experts to be stored as MXFP8
+                      (E4M3 + E8M0 per 32)
+  flash_mxfp8_prefill T=8192, same
   pro_skewed          T=2048, H=7168, I=3072, 384 + 1, top-6, with a Zipf
                       per-expert logit bias b_e = 2 ln(1/rank_e) over a seeded
                       random expert permutation (a few experts get most tokens)
   dspark              T=256,  H=5120, I=2304, 128 routed + 1 shared, top-3
                       (the drafter's expert count and top-k from the config;
                       its widths are not printed, the main layer's are assumed)
-All use route_scale 1.5 and swiglu_limit 10. The MXFP4 workloads draw BF16
-weights exactly like flash_decode; quantising them is the consumer's job.
+All use route_scale 1.5 and swiglu_limit 10. The MXFP4 and MXFP8 workloads draw
+BF16 weights exactly like flash_decode; quantising them is the consumer's job.
 """
 from __future__ import annotations
 
@@ -42,7 +45,7 @@ class Workload:
     k: int = 6
     route_scale: float = 1.5
     swiglu_limit: float = 10.0
-    expert_dtype: str = "bf16"          # "bf16" | "mxfp4" (routed experts)
+    expert_dtype: str = "bf16"          # "bf16" | "mxfp4" | "mxfp8" (routed experts)
     zipf_bias: bool = False
     seed: int = 1000
 
@@ -62,6 +65,10 @@ WORKLOADS = {
                                    expert_dtype="mxfp4", seed=1003),
     "flash_mxfp4_prefill": Workload("flash_mxfp4_prefill", T=4096, H=5120, I=2304, E=384,
                                     expert_dtype="mxfp4", seed=1003),
+    "flash_mxfp8_decode": Workload("flash_mxfp8_decode", T=32, H=5120, I=2304, E=384,
+                                   expert_dtype="mxfp8", seed=1006),
+    "flash_mxfp8_prefill": Workload("flash_mxfp8_prefill", T=8192, H=5120, I=2304, E=384,
+                                    expert_dtype="mxfp8", seed=1006),
     "pro_skewed": Workload("pro_skewed", T=2048, H=7168, I=3072, E=384, zipf_bias=True, seed=1004),
     "dspark": Workload("dspark", T=256, H=5120, I=2304, E=128, k=3, seed=1005),
 }

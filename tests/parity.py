@@ -37,11 +37,13 @@ def _bf16_bits_to_f64(u16: np.ndarray) -> np.ndarray:
     return (u16.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
 
 
-def _mxfp4_roundtrip_expert(mats):
-    """Worker: the oracle's MXFP4 round trip of one expert's three BF16 matrices
-    (given as uint16 bit patterns); float32 holds every result exactly."""
+def _mx_roundtrip_expert(job):
+    """Worker: the oracle's MX round trip (element format 'e2m1' or 'e4m3') of one
+    expert's three BF16 matrices (uint16 bit patterns); float32 holds every result
+    exactly."""
     from oracle import mx as omx
-    return tuple(omx.mx_roundtrip(_bf16_bits_to_f64(m), "e2m1").astype(np.float32) for m in mats)
+    fmt, mats = job
+    return tuple(omx.mx_roundtrip(_bf16_bits_to_f64(m), fmt).astype(np.float32) for m in mats)
 
 
 def _u16(t: torch.Tensor) -> np.ndarray:
@@ -59,24 +61,26 @@ def oracle_pool(n: int | None = None):
 class LayerExperts(om.ExpertSource):
     """Oracle expert source reading one expert at a time from the generator's tensors.
 
-    mx_from_bf16: the routed experts are the oracle's own MXFP4 quantisation of the
-    BF16 draw. With a process pool and the list of experts the comparison needs
+    mx_from_bf16: the routed experts are the oracle's own MXFP4 (mx_fmt 'e2m1') or
+    MXFP8 ('e4m3') quantisation of the BF16 draw; mx_q: given MXFP4 (packed) or
+    MXFP8 tensors. With a process pool and the list of experts the comparison needs
     (in the order the oracle visits them), that quantisation runs in the pool,
     a batch of experts at a time; the oracle itself is unchanged.
     """
 
     def __init__(self, layer: dict, mx_q: dict | None = None, mx_from_bf16: bool = False, pool=None,
-                 needed=None):
+                 needed=None, mx_fmt: str = "e2m1"):
         S = layer["sh_w1"].shape[0]
         E = layer["w1"].shape[0]
         self._layer = layer
         self._pool = pool
         self._needed = [int(e) for e in needed] if needed is not None else None
         self._cache = {}
+        self._fmt = mx_fmt
         if mx_from_bf16:
             from oracle import mx as omx
             if pool is None or needed is None:
-                rt = lambda w: omx.mx_roundtrip(f64(w), "e2m1")
+                rt = lambda w: omx.mx_roundtrip(f64(w), mx_fmt)
                 routed = lambda e: (rt(layer["w1"][e]), rt(layer["w3"][e]), rt(layer["w2"][e]))
             else:
                 routed = self._pooled_mx
@@ -86,7 +90,9 @@ class LayerExperts(om.ExpertSource):
             is_mx = False
         else:
             from oracle import mx as omx
-            dq = lambda q, s, e: omx.dequantize_mxfp4_packed(q[e].cpu().numpy(), s[e].cpu().numpy())
+            fp8 = mx_q["w1"].shape[-1] == layer["w1"].shape[-1]
+            dqf = omx.dequantize_mxfp8 if fp8 else omx.dequantize_mxfp4_packed
+            dq = lambda q, s, e: dqf(q[e].cpu().numpy(), s[e].cpu().numpy())
             routed = lambda e: (dq(mx_q["w1"], mx_q["s1"], e), dq(mx_q["w3"], mx_q["s3"], e),
                                 dq(mx_q["w2"], mx_q["s2"], e))
             is_mx = True
@@ -99,8 +105,8 @@ class LayerExperts(om.ExpertSource):
             pos = self._needed.index(e) if e in self._needed else None
             batch = self._needed[pos:pos + 2 * self._pool._processes] if pos is not None else [e]
             lay = self._layer
-            jobs = [(_u16(lay["w1"][b]), _u16(lay["w3"][b]), _u16(lay["w2"][b])) for b in batch]
-            for b, mats in zip(batch, self._pool.map(_mxfp4_roundtrip_expert, jobs)):
+            jobs = [(self._fmt, (_u16(lay["w1"][b]), _u16(lay["w3"][b]), _u16(lay["w2"][b]))) for b in batch]
+            for b, mats in zip(batch, self._pool.map(_mx_roundtrip_expert, jobs)):
                 self._cache[b] = mats
         return tuple(m.astype(np.float64) for m in self._cache[e])
 
@@ -151,7 +157,8 @@ def oracle_route(layer, k, rs, tokens=None):
     return om.route(f64(x), f64(layer["wg"]), k, rs, bias=bias)
 
 
-def compare_layer(layer, tokens, y_gpu, idx_gpu, w_gpu, k, rs, limit, mx_q=None, mx_from_bf16=False, pool=None):
+def compare_layer(layer, tokens, y_gpu, idx_gpu, w_gpu, k, rs, limit, mx_q=None, mx_from_bf16=False, pool=None,
+                  mx_fmt="e2m1"):
     """Compare GPU rows (for `tokens`) with the oracle; returns a report dict, asserts the bars.
 
     With mx_q (packed MXFP4 tensors) or mx_from_bf16 the routed experts are MXFP4 and
@@ -169,7 +176,7 @@ def compare_layer(layer, tokens, y_gpu, idx_gpu, w_gpu, k, rs, limit, mx_q=None,
                            f"gpu {idx_g[mism[:1]]} oracle {r.idx[mism[:1]]} gap {r.gap[mism[:1]]}"
     # outputs: use the GPU's selection where the oracle's gap is within the tie band
     override = np.where(sure[:, None], r.idx, idx_g)
-    ex = LayerExperts(layer, mx_q, mx_from_bf16, pool=pool, needed=np.unique(override))
+    ex = LayerExperts(layer, mx_q, mx_from_bf16, pool=pool, needed=np.unique(override), mx_fmt=mx_fmt)
     res = om.moe_forward(x, wg, ex, k, rs, limit, bias=bias, idx_override=override)
     w_or = res.route.w
     dw = np.abs(np.asarray(w_gpu, dtype=np.float64) - w_or).max()
