@@ -218,12 +218,17 @@ typedef enum {
   MOE_BUF_XQ_SCALES = 9, /* MXFP4 / MXFP8 layers: their E8M0 scales, packed in 512-byte atoms per token tile */
   MOE_BUF_HQ = 10,       /* MXFP4 / MXFP8 layers: uint8 E4M3 [T*k, I], MXFP8 codes of the routed SwiGLU rows
                             (group order, as MOE_BUF_H) */
-  MOE_BUF_HQ_SCALES = 11 /* MXFP4 / MXFP8 layers: their E8M0 scales in 512-byte atoms, one per (down-GEMM
+  MOE_BUF_HQ_SCALES = 11, /* MXFP4 / MXFP8 layers: their E8M0 scales in 512-byte atoms, one per (down-GEMM
                             token tile nt, 128-wide slice c of I): row n of the tile, block b of the
                             slice at byte (nt * I/128 + c) * 512 + (n % 32) * 16 + (n / 32) * 4 + b.
                             Token tiles: each routed group's rows cut into tiles of 32 rows when
                             T <= 32, 96 rows when T * top_k >= 24 * n_routed, else 64 rows,
                             numbered group by group in expert order */
+  MOE_BUF_NTILES = 12,   /* int32 [4]: tiles in the gate/up and down lists, and where their shared-expert
+                            tiles end */
+  MOE_BUF_TILES_GU = 13, /* int32 [n, 4] gate/up tile list: {group | m_tile << 16, B row or token-tile id,
+                            first output row, rows} in the order the persistent CTAs take them */
+  MOE_BUF_TILES_DN = 14  /* int32 [n, 4] the same for the down GEMM */
 } moe_buffer;
 
 /*

@@ -28,7 +28,7 @@ MOE_DT_BF16, MOE_DT_MXFP4, MOE_DT_MXFP8 = 0, 1, 2
 
 # moe_buffer ids
 (BUF_LOGITS, BUF_TOPK_IDX, BUF_TOPK_W, BUF_COUNTS, BUF_OFFSETS, BUF_PERM, BUF_INV, BUF_H, BUF_XQ, BUF_XQ_SCALES,
- BUF_HQ, BUF_HQ_SCALES) = range(12)
+ BUF_HQ, BUF_HQ_SCALES, BUF_NTILES, BUF_TILES_GU, BUF_TILES_DN) = range(15)
 
 EXPORTED = ("moe_create", "moe_forward", "moe_forward_host", "moe_get_status", "moe_status_string",
             "moe_destroy", "moe_abi_version", "moe_quantize_mxfp4", "moe_inspect", "moe_set_wait_timeout",

@@ -853,6 +853,9 @@ moe_status moe_inspect(moe_handle* h, int32_t what, void* dst, size_t bytes, moe
       src = h->sfb_dn;
       cap = h->max_ntiles_r * (I / 128) * 512;
       break;
+    case MOE_BUF_NTILES: src = h->ntiles; cap = 16; break;
+    case MOE_BUF_TILES_GU: src = h->tiles_gu; cap = h->max_tiles_gu * 16; break;
+    case MOE_BUF_TILES_DN: src = h->tiles_dn; cap = h->max_tiles_dn * 16; break;
     default: return MOE_ERR_INVALID_ARG;
   }
   if (bytes > cap) return MOE_ERR_INVALID_ARG;

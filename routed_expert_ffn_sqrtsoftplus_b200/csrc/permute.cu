@@ -17,7 +17,9 @@ namespace moe {
 
 namespace {
 
-constexpr int kMaxGroups = 1024;  // routed + shared groups (one scan thread each)
+constexpr int kMaxGroups = 1024;      // routed experts of the histogram and scatter kernels
+constexpr int kMaxScanGroups = 544;   // routed (<= 512) + shared (<= 4) groups of the scan kernel
+constexpr int kMaxSegs = 2 * kMaxScanGroups;  // tile-list segments (shared, full, partial)
 
 __global__ void __launch_bounds__(256)
     perm_count_kernel(const int32_t* __restrict__ idx, int nslots, int E, int32_t* __restrict__ chunk_cnt,
@@ -72,13 +74,14 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* warp_tot, int* t
 // and scatters the slots itself, so one launch replaces three.
 __global__ void __launch_bounds__(1024) perm_scan_kernel(ScanArgs a, int fused, const int32_t* idx, int nslots,
                                                         int32_t* perm, int32_t* inv, int* status) {
-  __shared__ int cnt_s[kMaxGroups];
-  __shared__ int off_s[kMaxGroups + 1];
-  __shared__ int tgu_s[kMaxGroups + 1];   // first gate/up tile of each group (tile order)
-  __shared__ int tdn_s[kMaxGroups + 1];
-  __shared__ int ngu_s[kMaxGroups + 1];   // first token tile of each routed group
-  __shared__ int ndn_s[kMaxGroups + 1];
-  __shared__ int ord_g[kMaxGroups + 1];   // group at tile-order position r
+  __shared__ int cnt_s[kMaxScanGroups];
+  __shared__ int off_s[kMaxScanGroups + 1];
+  __shared__ int ngu_s[kMaxScanGroups + 1];      // first token tile of each routed group
+  __shared__ int ndn_s[kMaxScanGroups + 1];
+  __shared__ int seg_pre[2][kMaxSegs + 1];       // first tile of each list segment (gate/up, down)
+  __shared__ int part_g[2][kMaxScanGroups];      // routed group of each partial-tile segment
+  __shared__ int rem_s[kMaxScanGroups];          // rows of each routed group's partial token tile
+  __shared__ int nseg_s[2];
   __shared__ int warp_tot[32];
   __shared__ int tot;
   __shared__ int maxc_s;
@@ -129,37 +132,59 @@ __global__ void __launch_bounds__(1024) perm_scan_kernel(ScanArgs a, int fused, 
     int o = block_exclusive_scan(n, warp_tot, &tot);
     if (g < G) off_s[g] = o;
     if (tid == 0) off_s[G] = tot;
-    // tile order: shared groups first, then routed
-    const int r = tid;
-    const int gr = r < G ? (r < a.S ? a.E + r : r - a.S) : -1;
-    const int nr = gr >= 0 ? cnt_s[gr] : 0;
-    const bool sh = gr >= a.E;
-    const int bgu = sh ? bn_gu_s : bn_gu_r, bdn = sh ? bn_dn_s : bn_dn_r;
-    const int ntg = (nr + bgu - 1) / bgu, ntd = (nr + bdn - 1) / bdn;
-    int tg = block_exclusive_scan(gr >= 0 ? a.m_tiles_gu * ntg : 0, warp_tot, &tot);
-    if (gr >= 0) tgu_s[r] = tg;
-    if (tid == 0) {
-      tgu_s[G] = tot;
-      a.ntiles[0] = tot;
-    }
-    int td = block_exclusive_scan(gr >= 0 ? a.m_tiles_dn * ntd : 0, warp_tot, &tot);
-    if (gr >= 0) tdn_s[r] = td;
-    if (tid == 0) {
-      tdn_s[G] = tot;
-      a.ntiles[1] = tot;
-    }
-    int ng = block_exclusive_scan(gr >= 0 && !sh ? ntg : 0, warp_tot, &tot);
-    if (gr >= 0 && !sh) ngu_s[gr] = ng;
+    // token-tile bases of the routed groups, in group order (MX scale atoms)
+    const bool routed = g < a.E;
+    int ng = block_exclusive_scan(routed ? (n + bn_gu_r - 1) / bn_gu_r : 0, warp_tot, &tot);
+    if (routed) ngu_s[g] = ng;
     if (tid == 0) ngu_s[a.E] = tot;
-    int nd = block_exclusive_scan(gr >= 0 && !sh ? ntd : 0, warp_tot, &tot);
-    if (gr >= 0 && !sh) ndn_s[gr] = nd;
+    int nd = block_exclusive_scan(routed ? (n + bn_dn_r - 1) / bn_dn_r : 0, warp_tot, &tot);
+    if (routed) ndn_s[g] = nd;
     if (tid == 0) ndn_s[a.E] = tot;
-    if (gr >= 0) ord_g[r] = gr;
   }
-  __syncthreads();
+  // Tile-list order, for persistent CTAs that take every gridDim-th tile: the
+  // costliest tiles first, so the last round holds the cheapest ones.
+  //   segments 0 .. S-1          every tile of shared group j (T rows)
+  //   segments S .. S+E-1        the full token tiles of routed group g, all m tiles
+  //   segments S+E .. S+E+P-1    the partial last token tile of each routed group
+  //                              that has one, by its row count descending
+  //                              (ties: lower group first), all m tiles
+  // Thread i owns segments 2i and 2i + 1 of the scan (S + 2E <= 2 * blockDim).
+  for (int list = 0; list < 2; ++list) {
+    const int bnr = list == 0 ? bn_gu_r : bn_dn_r, bns = list == 0 ? bn_gu_s : bn_dn_s;
+    const int mtl = list == 0 ? a.m_tiles_gu : a.m_tiles_dn;
+    for (int g = tid; g < a.E; g += blockDim.x) rem_s[g] = cnt_s[g] % bnr;
+    __syncthreads();
+    for (int g = tid; g < a.E; g += blockDim.x) {
+      const int rg = rem_s[g];
+      if (rg > 0) {
+        int rank = 0;
+        for (int h = 0; h < a.E; ++h) {
+          const int rh = rem_s[h];
+          rank += (rh > rg) || (rh == rg && h < g);
+        }
+        part_g[list][rank] = g;
+      }
+    }
+    const int npart = __syncthreads_count(tid < a.E && rem_s[tid] > 0);
+    const int ns = a.S + a.E + npart;
+    const int sh_tiles = mtl * ((a.T + bns - 1) / bns);
+    int c[2];
+    for (int q = 0; q < 2; ++q) {
+      const int sgi = 2 * tid + q;
+      c[q] = sgi >= ns ? 0 : sgi < a.S ? sh_tiles : sgi < a.S + a.E ? mtl * (cnt_s[sgi - a.S] / bnr) : mtl;
+    }
+    const int ex = block_exclusive_scan(c[0] + c[1], warp_tot, &tot);
+    if (2 * tid <= ns) seg_pre[list][2 * tid] = ex;
+    if (2 * tid + 1 <= ns) seg_pre[list][2 * tid + 1] = ex + c[0];
+    if (tid == 0) {
+      nseg_s[list] = ns;
+      a.ntiles[list] = tot;
+    }
+    __syncthreads();
+  }
   if (tid == 0) {
-    a.ntiles[2] = a.S > 0 ? tgu_s[a.S] : 0;
-    a.ntiles[3] = a.S > 0 ? tdn_s[a.S] : 0;
+    a.ntiles[2] = seg_pre[0][a.S];   // shared tiles end (= 0 without shared experts)
+    a.ntiles[3] = seg_pre[1][a.S];
   }
   // 3. outputs
   for (int g = tid; g <= G; g += blockDim.x) {
@@ -174,26 +199,42 @@ __global__ void __launch_bounds__(1024) perm_scan_kernel(ScanArgs a, int fused, 
   if (!fused)
     for (int g = tid; g < a.E; g += blockDim.x)
       for (int c = 0; c < a.nchunks; ++c) a.chunk_cnt[static_cast<size_t>(c) * a.E + g] += off_s[g];
-  // tile lists, spread over all threads: tile -> group by binary search over the
-  // tile-order prefix, then (m tile, token tile) inside the group
+  // tile lists, spread over all threads: tile -> segment by binary search over the
+  // segment prefix (the last segment starting at or before it is never empty),
+  // then (group, m tile, token tile) inside the segment
   for (int list = 0; list < 2; ++list) {
-    const int* pre = list == 0 ? tgu_s : tdn_s;
+    const int* pre = seg_pre[list];
+    const int ns = nseg_s[list];
+    const int bnr = list == 0 ? bn_gu_r : bn_dn_r, bns = list == 0 ? bn_gu_s : bn_dn_s;
     int4* out = list == 0 ? a.tiles_gu : a.tiles_dn;
-    const int total = pre[G];
+    const int total = pre[ns];
     for (int t = tid; t < total; t += blockDim.x) {
-      int lo = 0, hi = G - 1;
-      while (lo < hi) {  // last r with pre[r] <= t
+      int lo = 0, hi = ns - 1;
+      while (lo < hi) {  // last segment with pre <= t
         const int mid = (lo + hi + 1) >> 1;
         if (pre[mid] <= t) lo = mid; else hi = mid - 1;
       }
-      const int g = ord_g[lo];
+      const int local = t - pre[lo];
+      int g, mt, nt;
+      if (lo < a.S) {
+        g = a.E + lo;
+        const int ntn = (a.T + bns - 1) / bns;
+        mt = local / ntn;
+        nt = local % ntn;
+      } else if (lo < a.S + a.E) {
+        g = lo - a.S;
+        const int nf = cnt_s[g] / bnr;
+        mt = local / nf;
+        nt = local % nf;
+      } else {
+        g = part_g[list][lo - a.S - a.E];
+        mt = local;
+        nt = cnt_s[g] / bnr;
+      }
       const bool shared = g >= a.E;
       const bool mx = a.mx && !shared;
-      const int bn = list == 0 ? (shared ? bn_gu_s : bn_gu_r) : (shared ? bn_dn_s : bn_dn_r);
+      const int bn = shared ? bns : bnr;
       const int n = cnt_s[g];
-      const int ntn = (n + bn - 1) / bn;
-      const int local = t - pre[lo];
-      const int mt = local / ntn, nt = local % ntn;
       const int r0 = nt * bn;
       int y;
       if (list == 0)
@@ -345,14 +386,14 @@ cudaError_t launch_perm_count(const int32_t* idx, int nslots, int E, int32_t* ch
 }
 
 cudaError_t launch_perm_scan(const ScanArgs& a, cudaStream_t s) {
-  if (a.E + a.S > kMaxGroups) return cudaErrorInvalidValue;
+  if (a.E + a.S > kMaxScanGroups) return cudaErrorInvalidValue;
   perm_scan_kernel<<<1, 1024, 0, s>>>(a, 0, nullptr, 0, nullptr, nullptr, nullptr);
   return cudaGetLastError();
 }
 
 cudaError_t launch_perm_fused(const ScanArgs& a, const int32_t* idx, int nslots, int32_t* perm, int32_t* inv,
                               int* status, cudaStream_t s) {
-  if (a.E + a.S > kMaxGroups || nslots > kPermChunk) return cudaErrorInvalidValue;
+  if (a.E + a.S > kMaxScanGroups || nslots > kPermChunk) return cudaErrorInvalidValue;
   perm_scan_kernel<<<1, 1024, 0, s>>>(a, 1, idx, nslots, perm, inv, status);
   return cudaGetLastError();
 }

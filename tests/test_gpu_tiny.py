@@ -279,3 +279,57 @@ def test_nan_token_is_contained_warp_topk(cuda_device):
         parity.check_nan_token(layer, lay, 1100, 1037, WL.k, WL.E, WL.route_scale, WL.swiglu_limit)
     finally:
         layer.close()
+
+
+def _check_tile_list(tiles, n_shared_end, cnt, off, E, gateup):
+    """Every group's rows covered once per weight tile; shared tiles first; the
+    routed tiles by row count, non-increasing (full tiles, then partial ones by size)."""
+    g = tiles[:, 0] & 0xFFFF
+    mt = tiles[:, 0] >> 16
+    y, z, rows = tiles[:, 1], tiles[:, 2], tiles[:, 3]
+    assert np.all(g[:n_shared_end] >= E) and np.all(g[n_shared_end:] < E)
+    r = rows[n_shared_end:]
+    assert np.all(r[:-1] >= r[1:]), "routed tiles are not longest first"
+    assert np.all(rows > 0)
+    m_tiles = int(mt.max()) + 1
+    for grp in range(len(cnt)):
+        sel = g == grp
+        if cnt[grp] == 0:
+            assert not sel.any()
+            continue
+        assert set(mt[sel].tolist()) == set(range(m_tiles))
+        for m in range(m_tiles):
+            s2 = sel & (mt == m)
+            cover = np.zeros(cnt[grp], dtype=np.int64)
+            for zz, rr in zip(z[s2], rows[s2]):
+                cover[zz - off[grp]: zz - off[grp] + rr] += 1
+            assert np.all(cover == 1), f"group {grp} m tile {m}: rows covered {cover.min()}..{cover.max()} times"
+    if gateup:
+        shared = g >= E
+        assert np.array_equal(y[~shared], z[~shared]) and np.array_equal(y[shared], z[shared] - off[g[shared]])
+    else:
+        assert np.array_equal(y, z)
+
+
+@pytest.mark.parametrize("T,hot", [(17, False), (64, False), (300, False), (700, False), (300, True), (700, True)])
+def test_tile_lists_are_complete_and_longest_first(tiny, cuda_device, T, hot):
+    lay, layer = tiny
+    made = None
+    if hot:
+        bias = torch.zeros(WL.E, dtype=torch.float32, device=cuda_device)
+        bias[:2] = 6.0
+        made = layer = moe.MoELayer.from_layer(dict(lay, bias=bias), top_k=WL.k, max_tokens=700)
+    try:
+        x = lay["x"][:T].contiguous()
+        _run(layer, x)
+        dev = x.device
+        G = WL.E + WL.n_shared
+        nt = layer.inspect(moe.BUF_NTILES, torch.empty(4, dtype=torch.int32, device=dev)).cpu().numpy()
+        cnt = layer.inspect(moe.BUF_COUNTS, torch.empty(G, dtype=torch.int32, device=dev)).cpu().numpy()
+        off = layer.inspect(moe.BUF_OFFSETS, torch.empty(G + 1, dtype=torch.int32, device=dev)).cpu().numpy()
+        for which, n, ns, gateup in ((moe.BUF_TILES_GU, nt[0], nt[2], True), (moe.BUF_TILES_DN, nt[1], nt[3], False)):
+            tl = layer.inspect(which, torch.empty((int(n), 4), dtype=torch.int32, device=dev)).cpu().numpy()
+            _check_tile_list(tl.astype(np.int64), int(ns), cnt.astype(np.int64), off.astype(np.int64), WL.E, gateup)
+    finally:
+        if made is not None:
+            made.close()
