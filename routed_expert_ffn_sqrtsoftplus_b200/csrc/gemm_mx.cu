@@ -38,6 +38,11 @@ constexpr int kBK = 128;          // K values per stage
 constexpr int kBBoxRows = 32;
 constexpr int kBBoxBytes = kBBoxRows * 128;
 constexpr int kAtomBytes = 512;   // scale factors of 128 rows x 4 blocks
+// Weight boxes prefetched into L2 this many ring stages ahead of the loads (0 = none).
+#ifndef MOE_MX_PREFETCH
+#define MOE_MX_PREFETCH 0
+#endif
+constexpr int kPrefetch = MOE_MX_PREFETCH;
 
 constexpr int pow2_at_least(int v, int lo) {
   int p = lo;
@@ -160,6 +165,22 @@ __global__ void __launch_bounds__(kThreads, 1)
       int stage = 0;
       uint32_t phase = 0;
       long issued = 0;
+      // L2 prefetch cursor: walks the same (tile, K block) sequence kPrefetch stages ahead
+      int pf_t = tfirst, pf_kb = 0, pf_row = 0;
+      auto prefetch_next = [&]() {
+        if (pf_t >= tend) return;
+        if (pf_kb == 0) {
+          const Tile pt = load_tile<BN>(args, pf_t);
+          pf_row = pt.group * args.a_rows_per_group + pt.m_tile * C::kARows;
+        }
+        tma_prefetch_2d(&tmA, pf_kb * kBK, pf_row);
+        if (++pf_kb == args.num_kb) {
+          pf_kb = 0;
+          pf_t += gridDim.x;
+        }
+      };
+      if constexpr (kPrefetch > 0)
+        for (int i = 0; i < kPrefetch; ++i) prefetch_next();
       for (int t = tfirst; t < tend && !*abort_flag; t += gridDim.x) {
         const Tile tl = load_tile<BN>(args, t);
         const int a_row = tl.group * args.a_rows_per_group + tl.m_tile * C::kARows;
@@ -193,6 +214,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           bulk_load(sf + C::kSfaBytes, sfb_src + static_cast<size_t>(kb) * kAtomBytes, kAtomBytes, &full[stage],
                     kCacheEvictLast);
+          if constexpr (kPrefetch > 0) prefetch_next();
           ++issued;
           if (++stage == kStages) {
             stage = 0;
