@@ -113,6 +113,31 @@ def route(x, wg, k, route_scale, bias=None, idx_override=None):
     return Route(z=z, s=s, idx=idx, w=w, gap=gap)
 
 
+def hash_route(x, wg, table, token_ids, route_scale, bias=None):
+    """Routing of a hash layer (MAX DeepseekV41Config num_hash_layers; the
+    DeepSeek-V4-Pro config paragraph: "num_hash_layers 3").
+
+    The pages name hash layers but give no hash function. Reading adopted: a hash
+    layer takes its k experts from a fixed table of the vocabulary,
+    table [vocab, k] of distinct expert indices (a layer weight, like the router),
+    row token_ids[t] for token t, in the table's order, in place of the router's
+    top-k; the weights are the sqrtsoftplus scores of those experts, normalised
+    over the k and scaled by route_scale, exactly as for learned routing.
+    """
+    table = np.asarray(table, dtype=np.int64)
+    token_ids = np.asarray(token_ids, dtype=np.int64)
+    sel = table[token_ids]
+    return route(x, wg, sel.shape[1], route_scale, bias=bias, idx_override=sel)
+
+
+def moe_forward_hashed(x, wg, experts, table, token_ids, route_scale, limit, bias=None, mx_act=None):
+    """The layer with hash routing: the selection of hash_route, everything else as moe_forward."""
+    table = np.asarray(table, dtype=np.int64)
+    sel = table[np.asarray(token_ids, dtype=np.int64)]
+    return moe_forward(x, wg, experts, sel.shape[1], route_scale, limit, bias=bias, idx_override=sel,
+                       mx_act=mx_act)
+
+
 # ----------------------------------------------------------------------------
 # experts
 # ----------------------------------------------------------------------------
