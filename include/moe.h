@@ -157,6 +157,30 @@ MOE_API moe_status moe_forward(moe_handle* h, const void* x, int32_t T, void* y,
                        float* topk_w, moe_stream_t stream);
 
 /*
+ * Hash-routed layers (MAX DeepseekV41Config num_hash_layers; DeepSeek-V4-Pro has
+ * 3). The pages name them but give no hash function; this library reads them
+ * as: token t takes the top_k experts of row token_ids[t] of a fixed vocabulary
+ * table, in the row's order, in place of the router's top-k; the weights are
+ * the sqrtsoftplus scores of those experts (router logits + bias as for learned
+ * routing) normalised over the top_k and scaled by route_scale. Everything after
+ * the routing is the same layer.
+ *
+ * moe_set_hash_table: table int32 [vocab, top_k] device, every entry in
+ * [0, n_routed) and no expert twice in a row, else MOE_ERR_INVALID_ARG (the
+ * check runs on `stream`, and this call synchronises it). The library keeps
+ * its own copy (the only device allocation after moe_create; MOE_ERR_OOM if it
+ * fails); a later call replaces the table.
+ *
+ * moe_forward_hashed: as moe_forward, with token_ids int32 [T] device (the
+ * tokens' vocabulary ids). MOE_ERR_INVALID_ARG when no table was set. An id
+ * outside [0, vocab) gives that token the placeholder experts 0..top_k-1 with
+ * NaN weights and a NaN output row, and moe_get_status reports MOE_ERR_DEVICE.
+ */
+MOE_API moe_status moe_set_hash_table(moe_handle* h, const int32_t* table, int32_t vocab, moe_stream_t stream);
+MOE_API moe_status moe_forward_hashed(moe_handle* h, const void* x, const int32_t* token_ids, int32_t T, void* y,
+                                      int32_t* topk_idx, float* topk_w, moe_stream_t stream);
+
+/*
  * moe_forward on HOST buffers: copies x (BF16 [T, H], host, ideally pinned)
  * into a handle-owned device staging buffer, runs the layer, and copies y
  * (and topk_idx / topk_w when not NULL, host [T, k]) back, all enqueued on

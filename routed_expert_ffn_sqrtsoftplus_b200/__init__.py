@@ -33,7 +33,8 @@ MOE_DT_BF16, MOE_DT_MXFP4, MOE_DT_MXFP8 = 0, 1, 2
 EXPORTED = ("moe_create", "moe_forward", "moe_forward_host", "moe_get_status", "moe_status_string",
             "moe_destroy", "moe_abi_version", "moe_quantize_mxfp4", "moe_inspect", "moe_set_wait_timeout",
             "moe_selftest_wait_timeout", "moe_get_info", "moe_profile_begin", "moe_profile_end",
-            "moe_num_kernel_kinds", "moe_kernel_name", "moe_route_noalloc", "moe_quantize_mxfp8")
+            "moe_num_kernel_kinds", "moe_kernel_name", "moe_route_noalloc", "moe_quantize_mxfp8",
+            "moe_set_hash_table", "moe_forward_hashed")
 
 
 class MoEError(RuntimeError):
@@ -82,6 +83,8 @@ def lib() -> ctypes.CDLL:
             "moe_abi_version": (I32, []),
             "moe_quantize_mxfp4": (I32, [P, I64, I32, P, P, P]),
             "moe_quantize_mxfp8": (I32, [P, I64, I32, P, P, P]),
+            "moe_set_hash_table": (I32, [P, P, I32, P]),
+            "moe_forward_hashed": (I32, [P, P, P, I32, P, P, P, P]),
             "moe_inspect": (I32, [P, I32, P, ctypes.c_size_t, P]),
             "moe_set_wait_timeout": (I32, [P, U64]),
             "moe_selftest_wait_timeout": (I32, [P, U64, P]),
@@ -228,6 +231,35 @@ class MoELayer:
         return out
 
     __call__ = forward
+
+    def set_hash_table(self, table: torch.Tensor, stream=None):
+        """Vocabulary table int32 [vocab, top_k] of a hash-routed layer (copied by the library)."""
+        _need(table, "table", torch.int32)
+        if table.dim() != 2 or table.shape[1] != self.top_k:
+            raise ValueError(f"table must be [vocab, {self.top_k}]")
+        _check(lib().moe_set_hash_table(self._h, _ptr(table), table.shape[0], _stream(stream)),
+               "moe_set_hash_table")
+
+    def forward_hashed(self, x: torch.Tensor, token_ids: torch.Tensor, out: Optional[torch.Tensor] = None,
+                       topk_idx: Optional[torch.Tensor] = None, topk_w: Optional[torch.Tensor] = None,
+                       stream=None) -> torch.Tensor:
+        """The layer with hash routing: experts from the table row of each token's id."""
+        T = x.shape[0]
+        _need(x, "x", torch.bfloat16, (T, self.hidden))
+        _need(token_ids, "token_ids", torch.int32, (T,))
+        if out is None:
+            out = torch.empty_like(x)
+        _need(out, "out", torch.bfloat16, (T, self.hidden))
+        for n, t in (("x", x), ("token_ids", token_ids), ("out", out)):
+            if t.device != self.device:
+                raise ValueError(f"{n} is on {t.device}, the layer on {self.device}")
+        if topk_idx is not None:
+            _need(topk_idx, "topk_idx", torch.int32, (T, self.top_k))
+        if topk_w is not None:
+            _need(topk_w, "topk_w", torch.float32, (T, self.top_k))
+        _check(lib().moe_forward_hashed(self._h, _ptr(x), _ptr(token_ids), T, _ptr(out), _ptr(topk_idx),
+                                        _ptr(topk_w), _stream(stream)), "moe_forward_hashed")
+        return out
 
     def forward_with_routing(self, x: torch.Tensor, stream=None):
         T = x.shape[0]

@@ -59,7 +59,7 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 const char* kKernelNames[kKNumKinds] = {"router_logits", "router_gemm",  "topk_refine", "perm_count",
                                         "perm_scan",     "perm_scatter", "gather_rows", "gemm_gateup",
                                         "gemm_down",     "combine",      "quant_x",     "gemm_gateup_mx",
-                                        "gemm_down_mx",  "swiglu_reduce"};
+                                        "gemm_down_mx",  "swiglu_reduce", "hash_route"};
 
 // 2-D tensor map, 128-byte swizzle, box of box_cols x box_rows elements.
 bool make_tmap(CUtensorMap* m, const void* ptr, CUtensorMapDataType dt, uint64_t rows, uint64_t cols,
@@ -132,12 +132,17 @@ struct moe_handle {
   int* bn_choice = nullptr;     // token-tile width the permutation chose (many-token BF16 path)
   int32_t* ntile_base_dn = nullptr;
   int* bad = nullptr;
+  int* bad_flag = nullptr;      // device flag of the hash-table check
   int64_t max_ntiles_r = 0;
   CUtensorMap tm_w13q, tm_w2q, tm_w2qw, tm_xq, tm_hq, tm_w13sh, tm_w2sh, tm_w2shw;
   // shared experts alone (MXFP4 layers, few tokens): split-K partial sums
   float* sh_parts_gu = nullptr;  // [S][ks_gu][T][2I]
   float* sh_parts_dn = nullptr;  // [S][ks_dn][T][H]
   int ks_gu = 1, ks_dn = 1;
+
+  // hash-routed layers: the vocabulary table [hash_vocab, k] (library copy), or none
+  int32_t* hash_table = nullptr;
+  int32_t hash_vocab = 0;
 
   uint64_t timeout_ns = 2000000000ull;
   std::vector<void*> allocs;
@@ -167,6 +172,8 @@ struct moe_handle {
   void release() {
     for (void* p : allocs) cudaFree(p);
     allocs.clear();
+    if (hash_table != nullptr) cudaFree(hash_table);
+    hash_table = nullptr;
     for (cudaEvent_t e : ev) cudaEventDestroy(e);
     ev.clear();
   }
@@ -344,6 +351,7 @@ moe_status moe_create(const moe_config* cfg, const moe_weights* w, moe_stream_t 
   ok = ok && h->alloc(&h->h, h->R * I * 2, ws);
   ok = ok && h->alloc(&h->o, h->R * H * 4, ws);
   ok = ok && h->alloc(&h->status, 16, ws);
+  ok = ok && h->alloc(&h->bad_flag, 16, ws);
   ok = ok && h->alloc(&h->x_stage, Tm * H * 2, ws);
   ok = ok && h->alloc(&h->y_stage, Tm * H * 2, ws);
   if (!ok) {
@@ -422,8 +430,12 @@ moe_status moe_create(const moe_config* cfg, const moe_weights* w, moe_stream_t 
   return MOE_OK;
 }
 
-moe_status moe_forward(moe_handle* h, const void* x, int32_t T, void* y, int32_t* topk_idx, float* topk_w,
-                       moe_stream_t stream) {
+namespace {
+
+// One layer invocation; token_ids != nullptr selects the hash routing of the
+// handle's table instead of the learned router and top-k.
+moe_status forward_impl(moe_handle* h, const void* x, const int32_t* token_ids, int32_t T, void* y,
+                        int32_t* topk_idx, float* topk_w, moe_stream_t stream) {
   if (h == nullptr) return MOE_ERR_INVALID_ARG;
   if (T < 0 || T > h->cfg.max_tokens) return MOE_ERR_INVALID_ARG;
   if (T == 0) {
@@ -461,7 +473,12 @@ moe_status moe_forward(moe_handle* h, const void* x, int32_t T, void* y, int32_t
   if (!make_tmap_bf16(&tm_x, x, static_cast<uint64_t>(T), static_cast<uint64_t>(H), 32)) return MOE_ERR_CUDA;
 
   // 1-2. router logits (+ bias), scores, top-k, weights
-  if (T <= kSmallRouterMaxTokens) {
+  if (token_ids != nullptr) {
+    h->prof_mark(kKHashRoute, s);
+    MOE_TRY_CUDA(launch_hash_route(x, h->wg, h->bias, h->hash_table, token_ids, T, H, E, k, h->hash_vocab,
+                                   c.route_scale, h->idx, h->wts, h->status, s));
+    h->prof_done(s);
+  } else if (T <= kSmallRouterMaxTokens) {
     h->prof_mark(kKRouterLogits, s);
     MOE_TRY_CUDA(launch_router_small(x, h->wg, h->zpart, T, H, E, s));
     h->prof_done(s);
@@ -490,7 +507,7 @@ moe_status moe_forward(moe_handle* h, const void* x, int32_t T, void* y, int32_t
     MOE_TRY_CUDA(launch_gemm_down(h->tm_wg, tm_x, a, kBnLarge, nt < h->num_sms ? nt : h->num_sms, s));
     h->prof_done(s);
   }
-  if (T > kSmallRouterMaxTokens) {
+  if (token_ids == nullptr && T > kSmallRouterMaxTokens) {
     // scores, top-k with exact refinement of the near-tie candidates, weights
     h->prof_mark(kKTopk, s);
     if (T <= kTopkCtaMaxTokens) {
@@ -752,6 +769,54 @@ moe_status moe_forward(moe_handle* h, const void* x, int32_t T, void* y, int32_t
   if (topk_w) MOE_TRY_CUDA(cudaMemcpyAsync(topk_w, h->wts, static_cast<size_t>(nslots) * 4, cudaMemcpyDefault, s));
   h->last_T = T;
   return MOE_OK;
+}
+
+}  // namespace
+
+moe_status moe_forward(moe_handle* h, const void* x, int32_t T, void* y, int32_t* topk_idx, float* topk_w,
+                       moe_stream_t stream) {
+  return forward_impl(h, x, nullptr, T, y, topk_idx, topk_w, stream);
+}
+
+moe_status moe_set_hash_table(moe_handle* h, const int32_t* table, int32_t vocab, moe_stream_t stream) {
+  if (h == nullptr || table == nullptr || vocab <= 0) return MOE_ERR_INVALID_ARG;
+  int cur = -1;
+  if (cudaGetDevice(&cur) != cudaSuccess || cur != h->device) return MOE_ERR_INVALID_ARG;
+  if (!device_pointer_on(table, h->device)) return MOE_ERR_INVALID_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const size_t bytes = static_cast<size_t>(vocab) * h->cfg.top_k * 4;
+  int32_t* copy = nullptr;
+  if (cudaMalloc(&copy, bytes) != cudaSuccess) {
+    cudaGetLastError();
+    return MOE_ERR_OOM;
+  }
+  int bad = 0;
+  bool err = cudaMemcpyAsync(copy, table, bytes, cudaMemcpyDeviceToDevice, s) != cudaSuccess;
+  err |= cudaMemsetAsync(h->bad_flag, 0, sizeof(int), s) != cudaSuccess;
+  err |= launch_hash_table_check(copy, vocab, h->cfg.top_k, h->cfg.n_routed, h->bad_flag, s) != cudaSuccess;
+  err |= cudaMemcpyAsync(&bad, h->bad_flag, sizeof(int), cudaMemcpyDeviceToHost, s) != cudaSuccess;
+  err |= cudaStreamSynchronize(s) != cudaSuccess;
+  if (err || bad) {
+    cudaGetLastError();
+    cudaFree(copy);
+    return err ? MOE_ERR_CUDA : MOE_ERR_INVALID_ARG;
+  }
+  if (h->hash_table != nullptr) cudaFree(h->hash_table);
+  h->hash_table = copy;
+  h->hash_vocab = vocab;
+  return MOE_OK;
+}
+
+moe_status moe_forward_hashed(moe_handle* h, const void* x, const int32_t* token_ids, int32_t T, void* y,
+                              int32_t* topk_idx, float* topk_w, moe_stream_t stream) {
+  if (h == nullptr || h->hash_table == nullptr) return MOE_ERR_INVALID_ARG;
+  if (T > 0) {
+    if (token_ids == nullptr) return MOE_ERR_INVALID_ARG;
+    int cur = -1;
+    if (cudaGetDevice(&cur) != cudaSuccess || cur != h->device) return MOE_ERR_INVALID_ARG;
+    if (!device_pointer_on(token_ids, h->device)) return MOE_ERR_INVALID_ARG;
+  }
+  return forward_impl(h, x, token_ids, T, y, topk_idx, topk_w, stream);
 }
 
 moe_status moe_forward_host(moe_handle* h, const void* x_host, int32_t T, void* y_host, int32_t* topk_idx_host,

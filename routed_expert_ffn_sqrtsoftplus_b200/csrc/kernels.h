@@ -65,6 +65,7 @@ enum KernelKind {
   kKGateUpMx,
   kKDownMx,
   kKSwigluReduce,
+  kKHashRoute,
   kKNumKinds
 };
 
@@ -88,6 +89,13 @@ cudaError_t launch_topk_small(const float* part, int nparts, const void* x, cons
 cudaError_t launch_topk_refine(const float* z, const void* x, const void* wg, const float* bias, int T, int H,
                                int E, int k, float route_scale, float delta, int32_t* idx, float* w, int* status,
                                cudaStream_t s);
+
+// Hash-routed layers: selection from table[ids[t]] [vocab, k], exact sqrtsoftplus weights.
+cudaError_t launch_hash_route(const void* x, const void* wg, const float* bias, const int32_t* table,
+                              const int32_t* ids, int T, int H, int E, int k, int vocab, float route_scale,
+                              int32_t* idx, float* w, int* status, cudaStream_t s);
+// Sets *bad when an entry lies outside [0, E) or a row repeats an expert.
+cudaError_t launch_hash_table_check(const int32_t* table, int vocab, int k, int E, int* bad, cudaStream_t s);
 
 // ---- permutation
 constexpr int kPermChunk = 1024;

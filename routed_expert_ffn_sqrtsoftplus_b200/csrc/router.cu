@@ -519,7 +519,93 @@ __global__ void __launch_bounds__(256)
                                   w_out + static_cast<size_t>(t) * k, status);
 }
 
+// Hash-routed layers (MAX DeepseekV41Config num_hash_layers): token t takes the
+// k experts of row ids[t] of the layer's table, in the table's order; their
+// weights are the sqrtsoftplus scores normalised over the k and scaled by
+// route_scale. One CTA per token: warp j re-scores experts j, j + 8, ... exactly
+// (fp32-exact BF16 products, fp64 sums, as the learned routing's refinement),
+// warp 0 normalises. An id outside [0, vocab) gives the placeholder experts
+// 0..k-1 with NaN weights and records a device error.
+__global__ void __launch_bounds__(256)
+    hash_route_kernel(const uint4* __restrict__ x, const uint4* __restrict__ wg, const float* __restrict__ bias,
+                      const int32_t* __restrict__ table, const int32_t* __restrict__ ids, int H, int E, int k,
+                      int vocab, float route_scale, int32_t* __restrict__ idx_out, float* __restrict__ w_out,
+                      int* status) {
+  __shared__ double sc[kMaxK];
+  __shared__ int ex[kMaxK];
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int t = blockIdx.x;
+  const int id = ids[t];
+  const bool ok = id >= 0 && id < vocab;
+  const int hv = H / 8;
+  const uint4* xrow = x + static_cast<size_t>(t) * hv;
+  for (int j = warp; j < k; j += 8) {
+    const int e = ok ? table[static_cast<size_t>(id) * k + j] : j;
+    const uint4* wrow = wg + static_cast<size_t>(e) * hv;
+    double acc[4] = {0.0, 0.0, 0.0, 0.0};
+    for (int c = lane, q = 0; c < hv; c += 32, ++q) {
+      float xf[8], wf[8];
+      bf16x8_to_f32(__ldg(xrow + c), xf);
+      bf16x8_to_f32(__ldg(wrow + c), wf);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) acc[q & 3] += static_cast<double>(xf[i] * wf[i]);
+    }
+    double a = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
+    if (lane == 0) {
+      sc[j] = sqrt(softplus_f64(a + (bias ? static_cast<double>(bias[e]) : 0.0)));
+      ex[j] = e;
+    }
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    if (!ok) report_status(status, kStatusDevice);
+    double sum = 0.0;
+    for (int j = 0; j < k; ++j) sum += sc[j];
+    for (int j = 0; j < k; ++j) {
+      idx_out[static_cast<size_t>(t) * k + j] = ex[j];
+      w_out[static_cast<size_t>(t) * k + j] =
+          ok ? static_cast<float>(route_scale * (sc[j] / sum)) : __int_as_float(0x7fc00000);
+    }
+  }
+}
+
+// Table check: every entry in [0, E) and no expert twice in a row.
+__global__ void __launch_bounds__(256)
+    hash_table_check_kernel(const int32_t* __restrict__ table, int vocab, int k, int E, int* bad) {
+  const int v = blockIdx.x * blockDim.x + threadIdx.x;
+  if (v >= vocab) return;
+  const int32_t* row = table + static_cast<size_t>(v) * k;
+  for (int j = 0; j < k; ++j) {
+    const int e = row[j];
+    if (e < 0 || e >= E) {
+      atomicOr(bad, 1);
+      return;
+    }
+    for (int i = 0; i < j; ++i)
+      if (row[i] == e) {
+        atomicOr(bad, 1);
+        return;
+      }
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_hash_route(const void* x, const void* wg, const float* bias, const int32_t* table,
+                              const int32_t* ids, int T, int H, int E, int k, int vocab, float route_scale,
+                              int32_t* idx, float* w, int* status, cudaStream_t s) {
+  if (k > kMaxK || T == 0) return T == 0 ? cudaSuccess : cudaErrorInvalidValue;
+  hash_route_kernel<<<T, 256, 0, s>>>(static_cast<const uint4*>(x), static_cast<const uint4*>(wg), bias, table, ids,
+                                      H, E, k, vocab, route_scale, idx, w, status);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_hash_table_check(const int32_t* table, int vocab, int k, int E, int* bad, cudaStream_t s) {
+  hash_table_check_kernel<<<(vocab + 255) / 256, 256, 0, s>>>(table, vocab, k, E, bad);
+  return cudaGetLastError();
+}
 
 cudaError_t router_set_attributes() {
   return cudaFuncSetAttribute(router_small_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmallTok * 1024 * 2);

@@ -125,6 +125,30 @@ def make_experts(wl: Workload, device="cpu", seed: Optional[int] = None):
     return dict(w1=w1, w3=w3, w2=w2, sh_w1=s1, sh_w3=s3, sh_w2=s2)
 
 
+VOCAB = 129280   # DeepSeek V4.1 vocabulary (MAX DeepseekV41Config vocab_size)
+
+
+def make_hash_table(wl: Workload, vocab: int = VOCAB, device="cpu", seed: Optional[int] = None):
+    """Vocabulary table of a hash-routed layer: int32 [vocab, k], each row k distinct
+    experts (the k largest of E seeded uniform draws), from its own seeded stream."""
+    gen = torch.Generator(device="cpu")
+    gen.manual_seed((wl.seed if seed is None else seed) * 7919 + 53)
+    out = torch.empty((vocab, wl.k), dtype=torch.int32)
+    for v0 in range(0, vocab, 16384):
+        v1 = min(vocab, v0 + 16384)
+        out[v0:v1] = torch.rand((v1 - v0, wl.E), generator=gen).topk(wl.k, dim=1).indices.to(torch.int32)
+    return out.to(device)
+
+
+def make_token_ids(wl: Workload, vocab: int = VOCAB, device="cpu", T: Optional[int] = None,
+                   seed: Optional[int] = None):
+    """Token ids uniform over the vocabulary, int32 [T], from their own seeded stream."""
+    T = wl.T if T is None else T
+    gen = torch.Generator(device="cpu")
+    gen.manual_seed((wl.seed if seed is None else seed) * 7919 + 59)
+    return torch.randint(0, vocab, (T,), generator=gen, dtype=torch.int64).to(torch.int32).to(device)
+
+
 def make_layer(wl: Workload, device="cpu", T: Optional[int] = None, seed: Optional[int] = None):
     """All inputs of one layer invocation: x, wg, bias and the expert weights."""
     x = make_tokens(wl, device, T=T, seed=seed)

@@ -216,3 +216,23 @@ def check_nan_token(layer, lay, T, bad, k, E, rs, limit, mx_q=None):
     layer.forward(lay["x"][:T].contiguous())
     torch.cuda.synchronize()
     assert layer.status() == moe.MOE_OK
+
+
+def compare_hashed(layer, tokens, ids, table, y_gpu, idx_gpu, w_gpu, k, rs, limit, mx_q=None):
+    """Hash-routed layer: indices equal to the table rows of the ids, weights and
+    outputs against the oracle's moe_forward_hashed on the same tokens."""
+    tokens = np.asarray(tokens)
+    x = f64(layer["x"][torch.as_tensor(tokens, device=layer["x"].device)])
+    bias = None if layer.get("bias") is None else f64(layer["bias"])
+    tab = table.cpu().numpy().astype(np.int64)
+    ids_np = np.asarray(ids, dtype=np.int64)[tokens]
+    assert np.array_equal(np.asarray(idx_gpu, dtype=np.int64), tab[ids_np]), "selection differs from the table"
+    ex = LayerExperts(layer, mx_q)
+    res = om.moe_forward_hashed(x, f64(layer["wg"]), ex, tab, ids_np, rs, limit, bias=bias)
+    dw = float(np.abs(np.asarray(w_gpu, dtype=np.float64) - res.route.w).max())
+    assert dw <= TOL_W, f"routing weights differ by {dw}"
+    yg = np.asarray(y_gpu, dtype=np.float64)
+    rms = float(np.sqrt(np.mean(res.y ** 2)))
+    err = float(np.abs(yg - res.y).max())
+    assert np.all(np.isfinite(yg)) and err <= TOL_Y * rms, f"max|dy| = {err:.3e} > {TOL_Y} * RMS {rms:.3e}"
+    return dict(max_abs_err=err, rms=rms, rel=err / rms, max_dw=dw, tokens=len(tokens))

@@ -109,6 +109,8 @@ def test_null_handle_calls(L):
     assert L.moe_set_wait_timeout(None, 10) == moe.MOE_ERR_INVALID_ARG
     assert L.moe_profile_begin(None, 1) == moe.MOE_ERR_INVALID_ARG
     assert L.moe_get_info(None, None) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_set_hash_table(None, FAKE, 10, None) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_forward_hashed(None, FAKE, FAKE, 1, FAKE, None, None, None) == moe.MOE_ERR_INVALID_ARG
     L.moe_destroy(None)  # no-op
 
 
@@ -118,6 +120,14 @@ def test_quantize_rejects_bad_shapes(L):
     assert L.moe_quantize_mxfp4(None, 4, 32, FAKE, FAKE, None) == moe.MOE_ERR_INVALID_ARG
     assert L.moe_quantize_mxfp4(FAKE + 2, 4, 32, FAKE, FAKE, None) == moe.MOE_ERR_INVALID_ARG
     assert L.moe_quantize_mxfp4(FAKE, 0, 32, FAKE, FAKE, None) == moe.MOE_OK
+
+
+def test_quantize_mxfp8_rejects_bad_shapes(L):
+    assert L.moe_quantize_mxfp8(FAKE, 4, 33, FAKE, FAKE, None) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_quantize_mxfp8(FAKE, -1, 32, FAKE, FAKE, None) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_quantize_mxfp8(None, 4, 32, FAKE, FAKE, None) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_quantize_mxfp8(FAKE, 4, 32, FAKE + 4, FAKE, None) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_quantize_mxfp8(FAKE, 0, 32, FAKE, FAKE, None) == moe.MOE_OK
 
 
 def test_binding_refuses_cpu_tensors(L):
