@@ -132,7 +132,9 @@ typedef struct {
  * weights and the workspace for cfg->max_tokens tokens, and enqueue the weight
  * repack on `stream` (the analogue of the MAX pipeline's one-time routed-expert
  * upload, DeepseekV41Model.load_model). On success *out owns all device memory
- * it allocated. On failure *out is NULL and nothing is leaked. Every weight
+ * it allocated. On failure *out is NULL and nothing is leaked. (For tests of
+ * that path: with the environment variable MOE_TEST_FAIL_ALLOC_AFTER=n set, the
+ * create makes its (n+1)-th device allocation fail.) Every weight
  * pointer must be device (or managed) memory of the current device, else
  * MOE_ERR_INVALID_ARG before anything is enqueued.
  */
@@ -261,6 +263,14 @@ typedef enum {
  * buffer's size for max_tokens. For tests and debugging.
  */
 MOE_API moe_status moe_inspect(moe_handle* h, int32_t what, void* dst, size_t bytes, moe_stream_t stream);
+
+/*
+ * Fill every per-forward scratch buffer of the handle with `byte_value` (0-255;
+ * 0xFF makes every float a NaN and every index -1) on `stream`, leaving the
+ * status word alone. A forward must give the same bits after this as before it:
+ * nothing it reads is left over from an earlier call. For tests and debugging.
+ */
+MOE_API moe_status moe_fill_workspace(moe_handle* h, int32_t byte_value, moe_stream_t stream);
 
 /* Limit, in nanoseconds, of every device-side wait of this handle's kernels
  * (default 2e9). A smaller value makes a stuck wait return sooner. */

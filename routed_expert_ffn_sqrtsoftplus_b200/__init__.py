@@ -34,7 +34,7 @@ EXPORTED = ("moe_create", "moe_forward", "moe_forward_host", "moe_get_status", "
             "moe_destroy", "moe_abi_version", "moe_quantize_mxfp4", "moe_inspect", "moe_set_wait_timeout",
             "moe_selftest_wait_timeout", "moe_get_info", "moe_profile_begin", "moe_profile_end",
             "moe_num_kernel_kinds", "moe_kernel_name", "moe_route_noalloc", "moe_quantize_mxfp8",
-            "moe_set_hash_table", "moe_forward_hashed")
+            "moe_set_hash_table", "moe_forward_hashed", "moe_fill_workspace")
 
 
 class MoEError(RuntimeError):
@@ -84,6 +84,7 @@ def lib() -> ctypes.CDLL:
             "moe_quantize_mxfp4": (I32, [P, I64, I32, P, P, P]),
             "moe_quantize_mxfp8": (I32, [P, I64, I32, P, P, P]),
             "moe_set_hash_table": (I32, [P, P, I32, P]),
+            "moe_fill_workspace": (I32, [P, I32, P]),
             "moe_forward_hashed": (I32, [P, P, P, I32, P, P, P, P]),
             "moe_inspect": (I32, [P, I32, P, ctypes.c_size_t, P]),
             "moe_set_wait_timeout": (I32, [P, U64]),
@@ -286,6 +287,10 @@ class MoELayer:
         nbytes = out.numel() * out.element_size()
         _check(lib().moe_inspect(self._h, what, _ptr(out), nbytes, _stream(stream)), "moe_inspect")
         return out
+
+    def fill_workspace(self, byte_value: int, stream=None):
+        """Overwrite every per-forward scratch buffer with one byte value (a debugging aid)."""
+        _check(lib().moe_fill_workspace(self._h, int(byte_value), _stream(stream)), "moe_fill_workspace")
 
     def status(self) -> int:
         return lib().moe_get_status(self._h)

@@ -6,7 +6,10 @@
 #include <cstdlib>
 #include <cstring>
 #include <new>
+#include <utility>
 #include <vector>
+
+#include <nvtx3/nvToolsExt.h>
 
 #include "../../include/moe.h"
 #include "common.cuh"
@@ -146,6 +149,9 @@ struct moe_handle {
 
   uint64_t timeout_ns = 2000000000ull;
   std::vector<void*> allocs;
+  std::vector<std::pair<void*, size_t>> ws_allocs;  // per-forward scratch (moe_fill_workspace)
+  int fail_after = -1;          // test hook: allocations allowed before one is made to fail (-1: off)
+  int nvtx_open = 0;            // NVTX kernel ranges pushed and not yet popped
   uint64_t weight_bytes = 0, workspace_bytes = 0;
   int last_T = 0;
 
@@ -159,6 +165,8 @@ struct moe_handle {
   bool alloc(T** p, size_t bytes, uint64_t* counter) {
     void* q = nullptr;
     if (bytes == 0) bytes = 16;
+    if (fail_after == 0) return false;
+    if (fail_after > 0) --fail_after;
     if (cudaMalloc(&q, bytes) != cudaSuccess) {
       cudaGetLastError();
       return false;
@@ -166,6 +174,7 @@ struct moe_handle {
     allocs.push_back(q);
     *p = static_cast<T*>(q);
     *counter += bytes;
+    if (counter == &workspace_bytes) ws_allocs.emplace_back(q, bytes);
     return true;
   }
 
@@ -179,11 +188,17 @@ struct moe_handle {
   }
 
   void prof_mark(int kind, cudaStream_t s) {
+    nvtxRangePushA(kKernelNames[kind]);
+    ++nvtx_open;
     if (!prof_on || ev_used + 2 > ev.size()) return;
     cudaEventRecord(ev[ev_used], s);
     ev_kind[ev_used / 2] = kind;
   }
   void prof_done(cudaStream_t s) {
+    if (nvtx_open > 0) {
+      nvtxRangePop();
+      --nvtx_open;
+    }
     if (!prof_on || ev_used + 2 > ev.size()) return;
     cudaEventRecord(ev[ev_used + 1], s);
     ev_used += 2;
@@ -281,6 +296,7 @@ moe_status moe_create(const moe_config* cfg, const moe_weights* w, moe_stream_t 
   moe_handle* h = new (std::nothrow) moe_handle();
   if (h == nullptr) return MOE_ERR_OOM;
   h->cfg = *cfg;
+  if (const char* f = std::getenv("MOE_TEST_FAIL_ALLOC_AFTER")) h->fail_after = std::atoi(f);
   h->mx = mx;
   h->a8 = a8;
   if (cudaGetDevice(&h->device) != cudaSuccess ||
@@ -450,6 +466,18 @@ moe_status forward_impl(moe_handle* h, const void* x, const int32_t* token_ids, 
     if (!device_pointer_on(x, h->device) || !device_pointer_on(y, h->device)) return MOE_ERR_INVALID_ARG;
   }
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  // NVTX: one range per forward and one per kernel launch (the kernel ranges of a
+  // launch that failed are closed here too)
+  struct ForwardRange {
+    moe_handle* h;
+    explicit ForwardRange(moe_handle* hh, bool hashed) : h(hh) {
+      nvtxRangePushA(hashed ? "moe_forward_hashed" : "moe_forward");
+    }
+    ~ForwardRange() {
+      for (; h->nvtx_open > 0; --h->nvtx_open) nvtxRangePop();
+      nvtxRangePop();
+    }
+  } range(h, token_ids != nullptr);
   const moe_config& c = h->cfg;
   const int H = c.hidden, I = c.inter, E = c.n_routed, S = c.n_shared, k = c.top_k;
   const int nslots = T * k;
@@ -926,6 +954,17 @@ moe_status moe_inspect(moe_handle* h, int32_t what, void* dst, size_t bytes, moe
   if (bytes > cap) return MOE_ERR_INVALID_ARG;
   if (bytes == 0) return MOE_OK;
   MOE_TRY_CUDA(cudaMemcpyAsync(dst, src, bytes, cudaMemcpyDefault, reinterpret_cast<cudaStream_t>(stream)));
+  return MOE_OK;
+}
+
+moe_status moe_fill_workspace(moe_handle* h, int32_t byte_value, moe_stream_t stream) {
+  if (h == nullptr || byte_value < 0 || byte_value > 255) return MOE_ERR_INVALID_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  for (const auto& a : h->ws_allocs) {
+    // the status word and the check flags keep their meaning
+    if (a.first == h->status || a.first == h->bad || a.first == h->bad_flag) continue;
+    MOE_TRY_CUDA(cudaMemsetAsync(a.first, byte_value, a.second, s));
+  }
   return MOE_OK;
 }
 

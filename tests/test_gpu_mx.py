@@ -137,6 +137,19 @@ def test_mx_nan_token_is_contained(tiny_mx, T, bad):
     parity.check_nan_token(layer, lay, T, bad, WL.k, WL.E, WL.route_scale, WL.swiglu_limit, mx_q=mxq)
 
 
+@pytest.mark.parametrize("T", [5, 40, 300])
+def test_mx_poisoned_workspace_gives_the_same_bits(tiny_mx, T):
+    lay, _, layer = tiny_mx
+    x = lay["x"][:T].contiguous()
+    y1 = layer.forward(x).clone()
+    torch.cuda.synchronize()
+    layer.fill_workspace(0xFF)
+    y2 = layer.forward(x)
+    torch.cuda.synchronize()
+    assert layer.status() == moe.MOE_OK
+    assert torch.equal(y1, y2)
+
+
 def test_mx_deterministic(tiny_mx):
     lay, _, layer = tiny_mx
     x = lay["x"][:300].contiguous()

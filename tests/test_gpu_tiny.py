@@ -333,3 +333,36 @@ def test_tile_lists_are_complete_and_longest_first(tiny, cuda_device, T, hot):
     finally:
         if made is not None:
             made.close()
+
+
+@pytest.mark.parametrize("T", [5, 40, 300, 700])
+def test_poisoned_workspace_gives_the_same_bits(tiny, T):
+    """Every scratch buffer filled with 0xFF bytes (NaN floats, -1 indices) between
+    two forwards of the same tokens: the outputs are bit-identical, so no forward
+    reads anything an earlier call left in the workspace."""
+    lay, layer = tiny
+    x = lay["x"][:T].contiguous()
+    y1, i1, w1 = _run(layer, x)
+    y1 = y1.clone()
+    layer.fill_workspace(0xFF)
+    y2, i2, w2 = _run(layer, x)
+    assert torch.equal(y1, y2) and torch.equal(i1, i2) and torch.equal(w1, w2)
+
+
+@pytest.mark.parametrize("n_ok", [0, 1, 4, 12, 24])
+def test_create_failing_allocation_leaks_nothing(tiny, cuda_device, n_ok, monkeypatch):
+    """moe_create whose (n_ok+1)-th device allocation fails returns MOE_ERR_OOM and
+    hands back every byte it took (free device memory is unchanged)."""
+    lay, _ = tiny
+    torch.cuda.synchronize()
+    free0, _ = torch.cuda.mem_get_info(cuda_device)
+    monkeypatch.setenv("MOE_TEST_FAIL_ALLOC_AFTER", str(n_ok))
+    with pytest.raises(moe.MoEError) as ei:
+        moe.MoELayer.from_layer(lay, top_k=WL.k, max_tokens=700)
+    assert ei.value.status == moe.MOE_ERR_OOM
+    torch.cuda.synchronize()
+    free1, _ = torch.cuda.mem_get_info(cuda_device)
+    assert abs(free1 - free0) <= 2 << 20, f"free memory moved by {free0 - free1} bytes"
+    monkeypatch.delenv("MOE_TEST_FAIL_ALLOC_AFTER")
+    ok = moe.MoELayer.from_layer(lay, top_k=WL.k, max_tokens=64)
+    ok.close()
