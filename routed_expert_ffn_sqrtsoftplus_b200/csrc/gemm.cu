@@ -44,6 +44,11 @@ constexpr int kBK = 64;           // K elements per stage (128 bytes of BF16 = o
 constexpr int kBBoxRows = 32;     // token rows per B TMA box
 constexpr int kBBoxBytes = kBBoxRows * 128;
 constexpr int kWarpTma = 0, kWarpMma = 1;
+// Weight boxes prefetched into L2 this many ring stages ahead of the loads (0 = none).
+#ifndef MOE_BF16_PREFETCH
+#define MOE_BF16_PREFETCH 0
+#endif
+constexpr int kPrefetch = MOE_BF16_PREFETCH;
 
 constexpr int pow2_at_least(int v, int lo) {
   int p = lo;
@@ -205,6 +210,24 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
       uint32_t phase = 0;
       long issued = 0;
       bool ok = true;
+      // L2 prefetch cursor: walks the same (tile, K block) sequence kPrefetch stages ahead
+      int pf_t = tfirst, pf_kb = 0, pf_row = 0, pf_kb0 = 0, pf_nkb = 0;
+      auto prefetch_next = [&]() {
+        if (pf_t >= ntiles) return;
+        if (pf_kb == 0) {
+          const Tile pt = load_tile<BN>(args, pf_t);
+          pf_row = (pt.group - args.group_base) * args.a_rows_per_group + pt.m_tile * C::kARows;
+          pf_kb0 = pt.kb0;
+          pf_nkb = pt.nkb;
+        }
+        if (pf_nkb > 0) tma_prefetch_2d(tmA, (pf_kb0 + pf_kb) * kBK, pf_row);
+        if (++pf_kb >= pf_nkb) {
+          pf_kb = 0;
+          pf_t += gridDim.x;
+        }
+      };
+      if constexpr (kPrefetch > 0)
+        for (int i = 0; i < kPrefetch; ++i) prefetch_next();
       for (int t = tfirst; ok && t < ntiles && !*abort_flag; t += gridDim.x) {
         const Tile tl = load_tile<BN>(args, t);
         const CUtensorMap* mb = (kGateUp && tl.group >= args.n_routed) ? tmBsh : tmB;
@@ -222,6 +245,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
           for (int j = 0; j < nb; ++j)
             tma_load_2d(sB + stage * C::kBBytes + j * kBBoxBytes, mb, &full[stage], kx, tl.b_row0 + j * kBBoxRows,
                         kCacheEvictLast);
+          if constexpr (kPrefetch > 0) prefetch_next();
           ++issued;
           if (++stage == kStages) {
             stage = 0;
