@@ -64,18 +64,18 @@ const char* kKernelNames[kKNumKinds] = {"router_logits", "router_gemm",  "topk_r
                                         "gemm_down",     "combine",      "quant_x",     "gemm_gateup_mx",
                                         "gemm_down_mx",  "swiglu_reduce", "hash_route"};
 
-// 2-D tensor map, 128-byte swizzle, box of box_cols x box_rows elements.
+// 2-D tensor map, box of box_cols x box_rows elements, 128-byte swizzle unless stated.
 bool make_tmap(CUtensorMap* m, const void* ptr, CUtensorMapDataType dt, uint64_t rows, uint64_t cols,
-               uint64_t row_bytes, uint32_t box_cols, uint32_t box_rows) {
+               uint64_t row_bytes, uint32_t box_cols, uint32_t box_rows,
+               CUtensorMapSwizzle swz = CU_TENSOR_MAP_SWIZZLE_128B) {
   EncodeTiledFn enc = get_encode_fn();
   if (enc == nullptr) return false;
   cuuint64_t dims[2] = {cols, rows};
   cuuint64_t strides[1] = {row_bytes};
   cuuint32_t box[2] = {box_cols, box_rows};
   cuuint32_t estr[2] = {1, 1};
-  return enc(m, dt, 2, const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  return enc(m, dt, 2, const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 }  // namespace
@@ -414,11 +414,22 @@ moe_status moe_create(const moe_config* cfg, const moe_weights* w, moe_stream_t 
     }
     // MXFP4: packed E2M1 pairs, unpacked by the TMA to one value per byte in shared
     // memory; MXFP8: E4M3 bytes as stored. Either way 128 values = 128 smem bytes per row.
-    const CUtensorMapDataType wdt = a8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B;
-    err |= !make_tmap(&h->tm_w13q, h->w13q, wdt, E * 2 * I, H, a8 ? H : H / 2, 128, 256);
-    err |= !make_tmap(&h->tm_w2q, h->w2q, wdt, E * H, I, a8 ? I : I / 2, 128, 128);
-    h->wide_ok = H % 256 == 0;
-    if (h->wide_ok) err |= !make_tmap(&h->tm_w2qw, h->w2q, wdt, E * H, I, a8 ? I : I / 2, 128, 256);
+    // (With packed staging the MXFP4 weights are plain bytes: 64 per row per K step,
+    // unswizzled, and the kernel's expander warps lay them out for the MMA.)
+    if (!a8 && kMxPacked) {
+      const CUtensorMapDataType u8 = CU_TENSOR_MAP_DATA_TYPE_UINT8;
+      const CUtensorMapSwizzle none = CU_TENSOR_MAP_SWIZZLE_NONE;
+      err |= !make_tmap(&h->tm_w13q, h->w13q, u8, E * 2 * I, H / 2, H / 2, 64, 256, none);
+      err |= !make_tmap(&h->tm_w2q, h->w2q, u8, E * H, I / 2, I / 2, 64, 128, none);
+      h->wide_ok = H % 256 == 0;
+      if (h->wide_ok) err |= !make_tmap(&h->tm_w2qw, h->w2q, u8, E * H, I / 2, I / 2, 64, 256, none);
+    } else {
+      const CUtensorMapDataType wdt = a8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B;
+      err |= !make_tmap(&h->tm_w13q, h->w13q, wdt, E * 2 * I, H, a8 ? H : H / 2, 128, 256);
+      err |= !make_tmap(&h->tm_w2q, h->w2q, wdt, E * H, I, a8 ? I : I / 2, 128, 128);
+      h->wide_ok = H % 256 == 0;
+      if (h->wide_ok) err |= !make_tmap(&h->tm_w2qw, h->w2q, wdt, E * H, I, a8 ? I : I / 2, 128, 256);
+    }
     err |= !make_tmap(&h->tm_xq, h->xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, Tm * k, H, H, 128, 32);
     err |= !make_tmap(&h->tm_hq, h->hq, CU_TENSOR_MAP_DATA_TYPE_UINT8, Tm * k, I, I, 128, 32);
   }

@@ -33,7 +33,14 @@ namespace {
 
 constexpr int kEpiWarps = 8;  // two per TMEM lane quarter
 constexpr int kEpiGroups = kEpiWarps / 4;
-constexpr int kThreads = 64 + 32 * kEpiWarps;
+// Packed staging of MXFP4 weights (MOE_MX_PACKED, kernels.h): the ring holds the
+// packed E2M1 bytes as stored (half the shared memory per HBM byte of the TMA
+// unpacking), and kExpWarps expander warps copy each stage into the 16-byte-
+// aligned layout the MMA reads, in kXBufs buffers of their own.
+constexpr int kExpWarps = kMxPacked ? 4 : 0;
+constexpr int kXBufs = MOE_MX_PACKED_BUFS;
+static_assert(kXBufs == 1 || kXBufs == 2, "expanded buffers");
+constexpr int kThreads = 64 + 32 * (kEpiWarps + kExpWarps);
 constexpr int kBK = 128;          // K values per stage
 constexpr int kBBoxRows = 32;
 constexpr int kBBoxBytes = kBBoxRows * 128;
@@ -60,6 +67,9 @@ struct MxCfg {
   static constexpr int kARows = kTwoA ? 256 : 128;
   static constexpr int kABytes = kARows * 128;          // one byte per value in shared memory
   static constexpr int kATx = kAF8 ? kABytes : kARows * 64;  // bytes the TMA moves from HBM
+  static constexpr bool kPack = kMxPacked && !kAF8;     // packed staging (E2M1 only)
+  static constexpr int kStageABytes = kPack ? kATx : kABytes;  // A bytes of one ring stage
+  static constexpr int kNX = kPack ? kXBufs : 0;        // expanded A buffers
   static constexpr int kBBytes = BN * 128;
   static constexpr int kSfaBytes = kTwoA ? 2 * kAtomBytes : kAtomBytes;
   static constexpr int kSfBytes = kSfaBytes + kAtomBytes;
@@ -67,10 +77,11 @@ struct MxCfg {
   static constexpr int kSfCols = kTwoA ? 12 : 8;         // 4 TMEM columns per atom
   static constexpr int kSfColBase = 2 * kAccCols;
   static constexpr int kTmemCols = pow2_at_least(kSfColBase + kStages * kSfCols, 32);
-  static constexpr int kBarrierBytes = 256;
-  static constexpr int kSmemBytes = 1024 + kStages * (kABytes + kBBytes + kSfBytes) + kBarrierBytes;
+  static constexpr int kBarrierBytes = 512;
+  static constexpr int kSmemBytes =
+      1024 + kNX * kABytes + kStages * (kStageABytes + kBBytes + kSfBytes) + kBarrierBytes;
   static_assert(kTmemCols <= 512, "TMEM");
-  static_assert((2 * kStages + 5) * 8 + 8 <= kBarrierBytes, "barriers");
+  static_assert((2 * kStages + 5 + 2 * kNX) * 8 + 8 <= kBarrierBytes, "barriers");
   static_assert(BN % kBBoxRows == 0 && BN <= 128, "BN");
   static_assert(kSmemBytes <= 227 * 1024, "shared memory");
 };
@@ -115,8 +126,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   using C = MxCfg<kGateUp, kWide, BN, kStages, kAF8>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sA = smem;
-  uint8_t* sB = sA + kStages * C::kABytes;
+  uint8_t* sX = smem;                                   // expanded A buffers (packed staging)
+  uint8_t* sA = sX + C::kNX * C::kABytes;
+  uint8_t* sB = sA + kStages * C::kStageABytes;
   uint8_t* sSF = sB + kStages * C::kBBytes;
   uint64_t* bars = reinterpret_cast<uint64_t*>(sSF + kStages * C::kSfBytes);
   uint64_t* full = bars;
@@ -124,7 +136,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* tfull = bars + 2 * kStages;
   uint64_t* tempty = bars + 2 * kStages + 2;
   uint64_t* drain = bars + 2 * kStages + 4;
-  uint32_t* tmem_base_smem = reinterpret_cast<uint32_t*>(bars + 2 * kStages + 5);
+  uint64_t* xfull = bars + 2 * kStages + 5;             // expanded buffer written
+  uint64_t* xempty = xfull + C::kNX;                    // expanded buffer consumed by the MMAs
+  uint32_t* tmem_base_smem = reinterpret_cast<uint32_t*>(xempty + C::kNX);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_base_smem + 1);
 
   const int warp = threadIdx.x / 32;
@@ -140,6 +154,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&tempty[i], kEpiWarps);
     }
     mbar_init(drain, 1);
+    for (int i = 0; i < C::kNX; ++i) {
+      mbar_init(&xfull[i], kExpWarps);
+      mbar_init(&xempty[i], 1);
+    }
     *abort_flag = 0;
     fence_mbarrier_init();
   }
@@ -199,7 +217,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
           mbar_arrive_expect_tx(&full[stage], bytes);
-          tma_load_2d(sA + stage * C::kABytes, &tmA, &full[stage], kb * kBK, a_row, kCacheEvictFirst);
+          // packed staging: the A map is over bytes (kBK / 2 per K step); otherwise over values
+          tma_load_2d(sA + stage * C::kStageABytes, &tmA, &full[stage], C::kPack ? kb * (kBK / 2) : kb * kBK, a_row,
+                      kCacheEvictFirst);
           for (int j = 0; j < nb; ++j)
             tma_load_2d(sB + stage * C::kBBytes + j * kBBoxBytes, &tmB, &full[stage], kb * kBK,
                         tl.row0 + j * kBBoxRows, kCacheEvictLast);
@@ -240,6 +260,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t phase = 0;
       int acc = 0;
       uint32_t acc_phase = 0;
+      int xb = 0;
+      uint32_t xph = 0;
       for (int t = tfirst; t < tend && !*abort_flag; t += gridDim.x) {
         const Tile tl = load_tile<BN>(args, t);
         const uint32_t n_mma = max(16, (tl.nrows + 15) & ~15);
@@ -248,12 +270,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t d = tmem_base + acc * C::kAccCols;
         bool ok = true;
         for (int kb = 0; kb < args.num_kb; ++kb) {
-          if (!wait_or_abort(&full[stage], phase, args, abort_flag)) {
+          if (!wait_or_abort(&full[stage], phase, args, abort_flag) ||
+              (C::kPack && !wait_or_abort(&xfull[xb], xph, args, abort_flag))) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t a_addr = smem_u32(sA + stage * C::kABytes);
+          const uint32_t a_addr = C::kPack ? smem_u32(sX + xb * C::kABytes) : smem_u32(sA + stage * C::kABytes);
           const uint32_t b_addr = smem_u32(sB + stage * C::kBBytes);
           const uint32_t sf_addr = smem_u32(sSF + stage * C::kSfBytes);
           const uint32_t sf_cols = tmem_base + C::kSfColBase + stage * C::kSfCols;
@@ -278,6 +301,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             stage = 0;
             phase ^= 1;
           }
+          if constexpr (C::kPack) {
+            umma_commit(&xempty[xb]);
+            if (++xb == C::kNX) {
+              xb = 0;
+              xph ^= 1;
+            }
+          }
         }
         if (!ok) break;
         umma_commit(&tfull[acc]);
@@ -289,6 +319,50 @@ __global__ void __launch_bounds__(kThreads, 1)
       umma_commit(drain);
       const uint64_t t0 = globaltimer_ns();
       while (!mbar_try_wait(drain, 0) && globaltimer_ns() - t0 < args.timeout_ns) {
+      }
+    }
+  } else if (warp >= 2 + kEpiWarps) {
+    // ------------------------------------------------------------ expanders (packed staging)
+    // Each stage's packed A rows (64 bytes = 128 E2M1 values) become the layout the
+    // 16U4_ALIGN16B TMA would have written: 8 packed bytes at the start of each
+    // 16-byte chunk, chunk c of row r at position c ^ (r % 8) of the row's 128
+    // bytes (128-byte swizzle, 8-row atoms of 1024 bytes).
+    if constexpr (C::kPack) {
+      const int et = (warp - 2 - kEpiWarps) * 32 + lane;  // 0 .. 32 * kExpWarps - 1
+      int stage = 0;
+      uint32_t phase = 0;
+      int xb = 0;
+      uint32_t xph = 0;
+      bool ok = true;
+      for (int t = tfirst; ok && t < tend; t += gridDim.x) {
+        for (int kb = 0; kb < args.num_kb; ++kb) {
+          if (lane == 0)
+            ok = wait_or_abort(&full[stage], phase, args, abort_flag) &&
+                 wait_or_abort(&xempty[xb], xph ^ 1, args, abort_flag);
+          ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+          if (!ok) break;
+          const uint8_t* src = sA + stage * C::kStageABytes;
+          uint8_t* dst = sX + xb * C::kABytes;
+#pragma unroll 4
+          for (int p = et; p < C::kARows * 4; p += 32 * kExpWarps) {
+            const int r = p >> 2, q = p & 3;
+            const uint4 v = *reinterpret_cast<const uint4*>(src + r * 64 + q * 16);
+            uint8_t* row = dst + (r >> 3) * 1024 + (r & 7) * 128;
+            *reinterpret_cast<uint2*>(row + (((2 * q) ^ (r & 7)) << 4)) = make_uint2(v.x, v.y);
+            *reinterpret_cast<uint2*>(row + (((2 * q + 1) ^ (r & 7)) << 4)) = make_uint2(v.z, v.w);
+          }
+          fence_proxy_async_smem();  // the tensor core reads what these generic stores wrote
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&xfull[xb]);
+          if (++stage == kStages) {
+            stage = 0;
+            phase ^= 1;
+          }
+          if (++xb == C::kNX) {
+            xb = 0;
+            xph ^= 1;
+          }
+        }
       }
     }
   } else {
@@ -404,23 +478,26 @@ cudaError_t launch(const CUtensorMap& tmA, const CUtensorMap& tmB, const MxGemmA
 }
 
 // Ring depths: as many stages as fit in 227 KB.
-constexpr int mx_ring_fit(int a_bytes, int b_bytes, int sf_bytes) {
-  return (227 * 1024 - 1024 - 256) / (a_bytes + b_bytes + sf_bytes);
+constexpr int mx_ring_fit(int a_bytes, int b_bytes, int sf_bytes, int fixed) {
+  return (227 * 1024 - 1024 - 512 - fixed) / (a_bytes + b_bytes + sf_bytes);
 }
-template <int BN>
-constexpr int kTwoAStages = mx_ring_fit(256 * 128, BN * 128, 3 * kAtomBytes);  // 32: 6, 64: 5, 96: 4
-template <int BN>
-constexpr int kOneAStages = mx_ring_fit(128 * 128, BN * 128, 2 * kAtomBytes);  // 32: 10, 64: 9, 96: 7
+// Ring stages for a token-tile width, one or two 128-row weight MMAs, packed staging or not:
+//   unpacked  two A: 32: 6, 64: 5, 96: 4    one A: 32: 10, 64: 9, 96: 7
+//   packed    two A (2 expanded buffers): 32: 7, 64: 6, 96: 5
+template <int BN, bool kTwo, bool kPack>
+constexpr int kStagesFor =
+    kPack ? mx_ring_fit((kTwo ? 256 : 128) * 64, BN * 128, (kTwo ? 3 : 2) * kAtomBytes, kXBufs * (kTwo ? 256 : 128) * 128)
+          : mx_ring_fit((kTwo ? 256 : 128) * 128, BN * 128, (kTwo ? 3 : 2) * kAtomBytes, 0);
 constexpr bool kExtraWidth = kBnMxLarge != 32 && kBnMxLarge != 64;
 
 template <bool kGateUp, bool kWide, bool kAF8>
 cudaError_t set_attrs() {
   constexpr bool two = kGateUp || kWide;
   cudaError_t e;
-  if ((e = set_attr<kGateUp, kWide, 32, two ? kTwoAStages<32> : kOneAStages<32>, kAF8>()) != cudaSuccess) return e;
-  if ((e = set_attr<kGateUp, kWide, 64, two ? kTwoAStages<64> : kOneAStages<64>, kAF8>()) != cudaSuccess) return e;
+  if ((e = set_attr<kGateUp, kWide, 32, kStagesFor<32, two, kMxPacked && !kAF8>, kAF8>()) != cudaSuccess) return e;
+  if ((e = set_attr<kGateUp, kWide, 64, kStagesFor<64, two, kMxPacked && !kAF8>, kAF8>()) != cudaSuccess) return e;
   if constexpr (kExtraWidth)
-    if ((e = set_attr<kGateUp, kWide, kBnMxLarge, two ? kTwoAStages<kBnMxLarge> : kOneAStages<kBnMxLarge>,
+    if ((e = set_attr<kGateUp, kWide, kBnMxLarge, kStagesFor<kBnMxLarge, two, kMxPacked && !kAF8>,
                       kAF8>()) != cudaSuccess)
       return e;
   return cudaSuccess;
@@ -431,12 +508,12 @@ cudaError_t launch_any(const CUtensorMap& tmA, const CUtensorMap& tmB, const MxG
                        cudaStream_t s) {
   constexpr bool two = kGateUp || kWide;
   if (bn == 32)
-    return launch<kGateUp, kWide, 32, two ? kTwoAStages<32> : kOneAStages<32>, kAF8>(tmA, tmB, a, grid, s);
+    return launch<kGateUp, kWide, 32, kStagesFor<32, two, kMxPacked && !kAF8>, kAF8>(tmA, tmB, a, grid, s);
   if (bn == 64)
-    return launch<kGateUp, kWide, 64, two ? kTwoAStages<64> : kOneAStages<64>, kAF8>(tmA, tmB, a, grid, s);
+    return launch<kGateUp, kWide, 64, kStagesFor<64, two, kMxPacked && !kAF8>, kAF8>(tmA, tmB, a, grid, s);
   if constexpr (kExtraWidth)
     if (bn == kBnMxLarge)
-      return launch<kGateUp, kWide, kBnMxLarge, two ? kTwoAStages<kBnMxLarge> : kOneAStages<kBnMxLarge>, kAF8>(
+      return launch<kGateUp, kWide, kBnMxLarge, kStagesFor<kBnMxLarge, two, kMxPacked && !kAF8>, kAF8>(
           tmA, tmB, a, grid, s);
   return cudaErrorInvalidValue;
 }

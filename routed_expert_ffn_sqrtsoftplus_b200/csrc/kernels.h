@@ -166,6 +166,15 @@ cudaError_t gemm_set_attributes();
 #define MOE_BN_MX_LARGE 96
 #endif
 constexpr int kBnMxLarge = MOE_BN_MX_LARGE;
+// MXFP4 weights staged packed in the ring and expanded by warps (1), or unpacked
+// by the 16U4_ALIGN16B TMA type (0); expanded buffers of the packed form.
+#ifndef MOE_MX_PACKED
+#define MOE_MX_PACKED 0
+#endif
+#ifndef MOE_MX_PACKED_BUFS
+#define MOE_MX_PACKED_BUFS 2
+#endif
+constexpr bool kMxPacked = MOE_MX_PACKED != 0;
 static_assert(kBnMxLarge % 32 == 0 && kBnMxLarge >= 32 && kBnMxLarge <= 128, "large MX token tile");
 struct MxGemmArgs {
   const int4* tiles;            // {group | m_tile << 16, token tile id, first row, rows}
