@@ -326,7 +326,7 @@ moe_status moe_create(const moe_config* cfg, const moe_weights* w, moe_stream_t 
   if (!mx) {
     ok = ok && h->alloc(&h->w13, (E + S) * 2 * I * H * 2, wb);
     ok = ok && h->alloc(&h->w2, (E + S) * H * I * 2, wb);
-    ok = ok && h->alloc(&h->xp, Tm * k * H * 2, ws);
+    if (!kGatherX) ok = ok && h->alloc(&h->xp, Tm * k * H * 2, ws);
   } else {
     ok = ok && h->alloc(&h->w13q, E * 2 * I * (a8 ? H : H / 2), wb);
     ok = ok && h->alloc(&h->w2q, E * H * (a8 ? I : I / 2), wb);
@@ -392,7 +392,7 @@ moe_status moe_create(const moe_config* cfg, const moe_weights* w, moe_stream_t 
     err |= !make_tmap_bf16(&h->tm_w2, h->w2, (E + S) * H, I, 128);
     h->wide_ok = H % 256 == 0;
     if (h->wide_ok) err |= !make_tmap_bf16(&h->tm_w2w, h->w2, (E + S) * H, I, 256);
-    err |= !make_tmap_bf16(&h->tm_xp, h->xp, Tm * k, H, 32);
+    if (!kGatherX) err |= !make_tmap_bf16(&h->tm_xp, h->xp, Tm * k, H, 32);
   } else {
     err |= cudaMemsetAsync(h->bad, 0, 16, s) != cudaSuccess;
     err |= launch_repack_w13_bytes(w->w1, w->w3, nullptr, nullptr, static_cast<int>(E), 0, static_cast<int>(I),
@@ -605,11 +605,23 @@ moe_status forward_impl(moe_handle* h, const void* x, const int32_t* token_ids, 
   }
 
   if (!h->mx) {
-    h->prof_mark(kKGather, s);
-    MOE_TRY_CUDA(launch_gather_rows(x, h->perm, nslots, k, H, h->xp, s));
-    h->prof_done(s);
-    // 4. gate/up grouped GEMM with the clamped SwiGLU epilogue (routed and shared groups)
+    // 4. gate/up grouped GEMM with the clamped SwiGLU epilogue (routed and shared
+    // groups). The routed token rows come straight from x through the permutation
+    // (tile::gather4 on a one-row-box map of x), or from a gathered copy.
+    CUtensorMap tm_xg;
+    if (kGatherX) {
+      if (!make_tmap_bf16(&tm_xg, x, static_cast<uint64_t>(T), static_cast<uint64_t>(H), 1)) return MOE_ERR_CUDA;
+    } else {
+      h->prof_mark(kKGather, s);
+      MOE_TRY_CUDA(launch_gather_rows(x, h->perm, nslots, k, H, h->xp, s));
+      h->prof_done(s);
+    }
+    const CUtensorMap& tm_b = kGatherX ? tm_xg : h->tm_xp;
     GemmArgs a{};
+    if (kGatherX) {
+      a.gather_perm = h->perm;
+      a.gather_k = k;
+    }
     a.tiles = h->tiles_gu;
     a.ntiles = h->ntiles;
     a.num_kb = H / 64;
@@ -625,9 +637,9 @@ moe_status forward_impl(moe_handle* h, const void* x, const int32_t* token_ids, 
     h->prof_mark(kKGateUp, s);
     if (alt) {
       a.bn_select = h->bn_choice;
-      MOE_TRY_CUDA(launch_gemm_gateup_dual(h->tm_w13, h->tm_xp, tm_x, a, h->num_sms, s));
+      MOE_TRY_CUDA(launch_gemm_gateup_dual(h->tm_w13, tm_b, tm_x, a, h->num_sms, s));
     } else {
-      MOE_TRY_CUDA(launch_gemm_gateup(h->tm_w13, h->tm_xp, tm_x, a, bn_gu, h->num_sms, s));
+      MOE_TRY_CUDA(launch_gemm_gateup(h->tm_w13, tm_b, tm_x, a, bn_gu, h->num_sms, s));
     }
     h->prof_done(s);
     // 5. down grouped GEMM

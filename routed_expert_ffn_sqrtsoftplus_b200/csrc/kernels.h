@@ -47,7 +47,15 @@ struct GemmArgs {
   int* status;                  // device status word
   unsigned long long timeout_ns;
   const int* bn_select;         // dual-width launch: the token-tile width the permutation chose
+  const int32_t* gather_perm;   // gate/up: routed B rows are x rows perm[row] / gather_k, fetched by
+  int gather_k;                 //   tile::gather4 through tmB (a one-row box map of x); nullptr = B rows as stored
 };
+// The BF16 gate/up GEMM fetches the routed token rows straight from x through the
+// permutation (tile::gather4) instead of a gathered copy (1), or reads the copy (0).
+#ifndef MOE_GATHER_X
+#define MOE_GATHER_X 1
+#endif
+constexpr bool kGatherX = MOE_GATHER_X != 0;
 
 // Kernel kinds for profiling (order = moe_kernel_name()).
 enum KernelKind {
