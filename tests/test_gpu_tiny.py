@@ -349,10 +349,11 @@ def test_poisoned_workspace_gives_the_same_bits(tiny, T):
     assert torch.equal(y1, y2) and torch.equal(i1, i2) and torch.equal(w1, w2)
 
 
-@pytest.mark.parametrize("n_ok", [0, 1, 4, 12, 24])
+@pytest.mark.parametrize("n_ok", [0, 1, 4, 12, 20])
 def test_create_failing_allocation_leaks_nothing(tiny, cuda_device, n_ok, monkeypatch):
     """moe_create whose (n_ok+1)-th device allocation fails returns MOE_ERR_OOM and
-    hands back every byte it took (free device memory is unchanged)."""
+    hands back every byte it took (free device memory is unchanged). A BF16 layer
+    makes about two dozen allocations, so every n_ok here fails one."""
     lay, _ = tiny
     torch.cuda.synchronize()
     free0, _ = torch.cuda.mem_get_info(cuda_device)
@@ -363,6 +364,8 @@ def test_create_failing_allocation_leaks_nothing(tiny, cuda_device, n_ok, monkey
     torch.cuda.synchronize()
     free1, _ = torch.cuda.mem_get_info(cuda_device)
     assert abs(free1 - free0) <= 2 << 20, f"free memory moved by {free0 - free1} bytes"
-    monkeypatch.delenv("MOE_TEST_FAIL_ALLOC_AFTER")
+    # a budget above the allocation count changes nothing
+    monkeypatch.setenv("MOE_TEST_FAIL_ALLOC_AFTER", "1000")
     ok = moe.MoELayer.from_layer(lay, top_k=WL.k, max_tokens=64)
     ok.close()
+    monkeypatch.delenv("MOE_TEST_FAIL_ALLOC_AFTER")
