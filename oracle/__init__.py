@@ -10,9 +10,10 @@ brute force, library decoders); none is "parity unpinned".
 """
 from . import mx
 from .moe import (ExpertSource, MoEResult, Route, clamped_swiglu, dense_reference,
-                  expert_forward, hash_route, moe_forward, moe_forward_hashed,
+                  expert_forward, hash_route, moe_forward, moe_forward_hashed, moe_forward_partial,
                   permutation_reference, route, silu, softplus, sqrtsoftplus)
 
 __all__ = ["mx", "ExpertSource", "MoEResult", "Route", "clamped_swiglu",
-           "dense_reference", "expert_forward", "hash_route", "moe_forward", "moe_forward_hashed", "permutation_reference",
+           "dense_reference", "expert_forward", "hash_route", "moe_forward", "moe_forward_hashed", "moe_forward_partial",
+           "permutation_reference",
            "route", "silu", "softplus", "sqrtsoftplus"]

@@ -242,6 +242,34 @@ def moe_forward(x, wg, experts: ExpertSource, k, route_scale, limit, bias=None,
     return res
 
 
+def moe_forward_partial(x, wg, experts: ExpertSource, k, route_scale, limit, expert_begin, expert_end,
+                        include_shared, bias=None, mx_act: Optional[bool] = None):
+    """One rank's share of an expert-parallel layer (MAX DeepseekV41Config ep_config,
+    "only under data parallelism"; the DEP recipes on the DeepSeek-V4-Pro page).
+
+    The experts are split into windows [expert_begin, expert_end), one per rank;
+    every rank routes all tokens with the full router. A rank's partial output is
+    the weighted sum over the selected slots whose expert lies in its window, plus
+    the shared experts when include_shared (exactly one rank holds them). The
+    partial outputs of a partition of [0, E) sum to the layer's output.
+    """
+    x = np.asarray(x, dtype=np.float64)
+    if mx_act is None:
+        mx_act = experts.routed_is_mx
+    r = route(x, wg, k, route_scale, bias=bias)
+    y = np.zeros_like(x)
+    if include_shared:
+        for j in range(experts.n_shared):
+            y += expert_forward(x, *experts.shared(j), limit, mx_act=False)[0]
+    for e in np.unique(r.idx):
+        if not (expert_begin <= e < expert_end):
+            continue
+        tok, slot = np.nonzero(r.idx == e)
+        o, _ = expert_forward(x[tok], *experts.routed(int(e)), limit, mx_act=mx_act)
+        y[tok] += r.w[tok, slot][:, None] * o
+    return y
+
+
 def dense_reference(x, wg, experts: ExpertSource, route_scale, bias=None):
     """The k = E, L = inf special case written without any top-k code:
 
