@@ -39,7 +39,7 @@
 extern "C" {
 #endif
 
-#define MOE_ABI_VERSION 2
+#define MOE_ABI_VERSION 3
 
 #if defined(__GNUC__)
 #define MOE_API __attribute__((visibility("default")))
@@ -157,6 +157,34 @@ MOE_API moe_status moe_create(const moe_config* cfg, const moe_weights* w, moe_s
  */
 MOE_API moe_status moe_forward(moe_handle* h, const void* x, int32_t T, void* y, int32_t* topk_idx,
                        float* topk_w, moe_stream_t stream);
+
+/*
+ * Expert parallelism (MAX DeepseekV41Config ep_config, "only under data
+ * parallelism"; the DEP recipes on the DeepSeek-V4-Pro page). The routed
+ * experts are split into windows, one per rank; every rank keeps the whole
+ * router. A rank routes all the ranks' tokens (gathered), runs only the slots
+ * whose expert lies in its window, and produces a partial output; the partial
+ * outputs of a partition of [0, n_routed) sum to the layer's output. The
+ * collectives (all-gather of x, reduce-scatter of the partial outputs) are the
+ * caller's (the Python package's ExpertParallelLayer uses torch.distributed).
+ *
+ * moe_create_ep: as moe_create, holding routed experts [expert_begin,
+ * expert_begin + expert_count) of cfg->n_routed. router_w [n_routed, H] and
+ * router_bias [n_routed] are whole; w1 / w3 / w2 (and s1 / s3 / s2) hold the
+ * window's expert_count experts only. The shared experts are cfg->n_shared
+ * of them on this rank (give them to exactly one rank, 0 to the others).
+ *
+ * moe_forward_partial: y_partial fp32 [T, H] device = this instance's share:
+ * sum over the selected slots of its window of w_j f_j(x), plus its shared
+ * experts, summed in fp32 in slot order and not rounded. Works on any handle
+ * (a whole layer gives the full output in fp32). moe_forward and
+ * moe_forward_hashed reject a handle that holds a window of the experts
+ * (MOE_ERR_INVALID_ARG).
+ */
+MOE_API moe_status moe_create_ep(const moe_config* cfg, const moe_weights* w, int32_t expert_begin,
+                                 int32_t expert_count, moe_stream_t stream, moe_handle** out);
+MOE_API moe_status moe_forward_partial(moe_handle* h, const void* x, int32_t T, float* y_partial,
+                                       int32_t* topk_idx, float* topk_w, moe_stream_t stream);
 
 /*
  * Hash-routed layers (MAX DeepseekV41Config num_hash_layers; DeepSeek-V4-Pro has

@@ -34,7 +34,8 @@ EXPORTED = ("moe_create", "moe_forward", "moe_forward_host", "moe_get_status", "
             "moe_destroy", "moe_abi_version", "moe_quantize_mxfp4", "moe_inspect", "moe_set_wait_timeout",
             "moe_selftest_wait_timeout", "moe_get_info", "moe_profile_begin", "moe_profile_end",
             "moe_num_kernel_kinds", "moe_kernel_name", "moe_route_noalloc", "moe_quantize_mxfp8",
-            "moe_set_hash_table", "moe_forward_hashed", "moe_fill_workspace")
+            "moe_set_hash_table", "moe_forward_hashed", "moe_fill_workspace", "moe_create_ep",
+            "moe_forward_partial")
 
 
 class MoEError(RuntimeError):
@@ -85,6 +86,9 @@ def lib() -> ctypes.CDLL:
             "moe_quantize_mxfp8": (I32, [P, I64, I32, P, P, P]),
             "moe_set_hash_table": (I32, [P, P, I32, P]),
             "moe_fill_workspace": (I32, [P, I32, P]),
+            "moe_create_ep": (I32, [ctypes.POINTER(_Config), ctypes.POINTER(_Weights), I32, I32, P,
+                                    ctypes.POINTER(P)]),
+            "moe_forward_partial": (I32, [P, P, I32, P, P, P, P]),
             "moe_forward_hashed": (I32, [P, P, P, I32, P, P, P, P]),
             "moe_inspect": (I32, [P, I32, P, ctypes.c_size_t, P]),
             "moe_set_wait_timeout": (I32, [P, U64]),
@@ -175,22 +179,28 @@ class MoELayer:
                  sh_w2: Optional[torch.Tensor] = None, router_bias: Optional[torch.Tensor] = None,
                  s1: Optional[torch.Tensor] = None, s3: Optional[torch.Tensor] = None,
                  s2: Optional[torch.Tensor] = None, route_scale: float = 1.5, swiglu_limit: float = 10.0,
-                 expert_dtype: str = "bf16", stream=None):
+                 expert_dtype: str = "bf16", expert_begin: int = 0, expert_count: Optional[int] = None,
+                 stream=None):
+        """expert_begin / expert_count: hold only that window of the routed experts
+        (expert parallelism; w1 / w3 / w2 and s1 / s3 / s2 then hold expert_count
+        experts); such a layer computes partial outputs only (forward_partial)."""
         self._h = ctypes.c_void_p(None)
         L = lib()
         H, I, E, S = hidden, inter, n_routed, n_shared
+        Ec = E if expert_count is None else expert_count
         _need(router_w, "router_w", torch.bfloat16, (E, H))
         if router_bias is not None:
             _need(router_bias, "router_bias", torch.float32, (E,))
         if expert_dtype == "bf16":
-            _need(w1, "w1", torch.bfloat16, (E, I, H)); _need(w3, "w3", torch.bfloat16, (E, I, H))
-            _need(w2, "w2", torch.bfloat16, (E, H, I))
+            _need(w1, "w1", torch.bfloat16, (Ec, I, H)); _need(w3, "w3", torch.bfloat16, (Ec, I, H))
+            _need(w2, "w2", torch.bfloat16, (Ec, H, I))
             dt = MOE_DT_BF16
         elif expert_dtype in ("mxfp4", "mxfp8"):
             div = 2 if expert_dtype == "mxfp4" else 1
-            _need(w1, "w1", torch.uint8, (E, I, H // div)); _need(w3, "w3", torch.uint8, (E, I, H // div))
-            _need(w2, "w2", torch.uint8, (E, H, I // div))
-            for n, t, shp in (("s1", s1, (E, I, H // 32)), ("s3", s3, (E, I, H // 32)), ("s2", s2, (E, H, I // 32))):
+            _need(w1, "w1", torch.uint8, (Ec, I, H // div)); _need(w3, "w3", torch.uint8, (Ec, I, H // div))
+            _need(w2, "w2", torch.uint8, (Ec, H, I // div))
+            for n, t, shp in (("s1", s1, (Ec, I, H // 32)), ("s3", s3, (Ec, I, H // 32)),
+                              ("s2", s2, (Ec, H, I // 32))):
                 if t is None:
                     raise ValueError(f"{n} is required for {expert_dtype} experts")
                 _need(t, n, torch.uint8, shp)
@@ -204,7 +214,12 @@ class MoELayer:
         wts = _Weights(_ptr(router_w), _ptr(router_bias), _ptr(w1), _ptr(w3), _ptr(w2), _ptr(s1), _ptr(s3),
                        _ptr(s2), _ptr(sh_w1), _ptr(sh_w3), _ptr(sh_w2))
         st = _stream(stream)
-        _check(L.moe_create(ctypes.byref(self.cfg), ctypes.byref(wts), st, ctypes.byref(self._h)), "moe_create")
+        if expert_count is None and expert_begin == 0:
+            _check(L.moe_create(ctypes.byref(self.cfg), ctypes.byref(wts), st, ctypes.byref(self._h)), "moe_create")
+        else:
+            _check(L.moe_create_ep(ctypes.byref(self.cfg), ctypes.byref(wts), expert_begin, Ec, st,
+                                   ctypes.byref(self._h)), "moe_create_ep")
+        self.expert_begin, self.expert_count = expert_begin, Ec
         # The library copied the weights on `st`; wait so the caller may free its tensors.
         torch.cuda.synchronize()
         self.hidden, self.inter, self.n_routed, self.n_shared, self.top_k = H, I, E, S, top_k
@@ -232,6 +247,21 @@ class MoELayer:
         return out
 
     __call__ = forward
+
+    def forward_partial(self, x: torch.Tensor, out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+        """This layer's share of an expert-parallel layer, fp32 [T, H]: the selected
+        slots whose expert lies in its window (plus the shared experts it holds)."""
+        T = x.shape[0]
+        _need(x, "x", torch.bfloat16, (T, self.hidden))
+        if out is None:
+            out = torch.empty((T, self.hidden), dtype=torch.float32, device=x.device)
+        _need(out, "out", torch.float32, (T, self.hidden))
+        for n, t in (("x", x), ("out", out)):
+            if t.device != self.device:
+                raise ValueError(f"{n} is on {t.device}, the layer on {self.device}")
+        _check(lib().moe_forward_partial(self._h, _ptr(x), T, _ptr(out), None, None, _stream(stream)),
+               "moe_forward_partial")
+        return out
 
     def set_hash_table(self, table: torch.Tensor, stream=None):
         """Vocabulary table int32 [vocab, top_k] of a hash-routed layer (copied by the library)."""
@@ -331,20 +361,23 @@ class MoELayer:
 
     @classmethod
     def from_layer(cls, layer: dict, *, top_k: int, max_tokens: int, route_scale: float = 1.5,
-                   swiglu_limit: float = 10.0, mx: Optional[dict] = None, stream=None) -> "MoELayer":
+                   swiglu_limit: float = 10.0, mx: Optional[dict] = None, expert_window=None,
+                   with_shared: bool = True, stream=None) -> "MoELayer":
         """Build from a dict of tensors (x ignored): wg, bias, w1, w3, w2, sh_w1, sh_w3, sh_w2.
 
         With ``mx`` = dict(w1, s1, w3, s3, w2, s2) of MXFP4 (packed, w1 [E, I, H/2]) or
         MXFP8 (w1 [E, I, H]) tensors the routed experts are stored in that format.
         """
         E, I, H = layer["w1"].shape
-        S = layer["sh_w1"].shape[0] if layer.get("sh_w1") is not None else 0
+        S = layer["sh_w1"].shape[0] if (with_shared and layer.get("sh_w1") is not None) else 0
+        sh = {n: (layer.get(n) if S > 0 else None) for n in ("sh_w1", "sh_w3", "sh_w2")}
+        b, c = (0, None) if expert_window is None else expert_window
+        cut = (lambda t: t) if expert_window is None else (lambda t: t[b:b + c].contiguous())
         kw = dict(hidden=H, inter=I, n_routed=E, n_shared=S, top_k=top_k, max_tokens=max_tokens,
-                  router_w=layer["wg"], router_bias=layer.get("bias"), sh_w1=layer.get("sh_w1"),
-                  sh_w3=layer.get("sh_w3"), sh_w2=layer.get("sh_w2"), route_scale=route_scale,
-                  swiglu_limit=swiglu_limit, stream=stream)
+                  router_w=layer["wg"], router_bias=layer.get("bias"), route_scale=route_scale,
+                  swiglu_limit=swiglu_limit, expert_begin=b, expert_count=c, stream=stream, **sh)
         if mx is None:
-            return cls(w1=layer["w1"], w3=layer["w3"], w2=layer["w2"], expert_dtype="bf16", **kw)
+            return cls(w1=cut(layer["w1"]), w3=cut(layer["w3"]), w2=cut(layer["w2"]), expert_dtype="bf16", **kw)
         fmt = "mxfp8" if mx["w1"].shape[-1] == H else "mxfp4"
-        return cls(w1=mx["w1"], w3=mx["w3"], w2=mx["w2"], s1=mx["s1"], s3=mx["s3"], s2=mx["s2"],
-                   expert_dtype=fmt, **kw)
+        return cls(w1=cut(mx["w1"]), w3=cut(mx["w3"]), w2=cut(mx["w2"]), s1=cut(mx["s1"]), s3=cut(mx["s3"]),
+                   s2=cut(mx["s2"]), expert_dtype=fmt, **kw)

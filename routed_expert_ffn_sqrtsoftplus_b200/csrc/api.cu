@@ -121,6 +121,7 @@ struct moe_handle {
   // MXFP4 routed experts (expert_dtype == MOE_DT_MXFP4)
   bool mx = false;              // routed experts block-scaled (MXFP4 or MXFP8)
   bool a8 = false;              // ... and MXFP8 (E4M3 weights, one byte per value)
+  int e_begin = 0, e_local = 0; // routed experts held: [e_begin, e_begin + e_local) of cfg.n_routed
   uint8_t* w13q = nullptr;      // packed E2M1, gate/up tile order
   uint8_t* w2q = nullptr;       // packed E2M1
   uint8_t* sfa13 = nullptr;     // scale atoms of W1|W3
@@ -263,12 +264,20 @@ const char* moe_kernel_name(int32_t kind) {
   return kKernelNames[kind];
 }
 
-moe_status moe_create(const moe_config* cfg, const moe_weights* w, moe_stream_t stream, moe_handle** out) {
+}  // extern "C"
+
+namespace {
+
+// A layer instance holding the routed experts [e_begin, e_begin + e_count) of the
+// router's n_routed (all of them for moe_create; a window for moe_create_ep).
+moe_status create_impl(const moe_config* cfg, const moe_weights* w, int32_t e_begin, int32_t e_count,
+                       moe_stream_t stream, moe_handle** out) {
   if (out == nullptr) return MOE_ERR_INVALID_ARG;
   *out = nullptr;
   if (cfg == nullptr || w == nullptr) return MOE_ERR_INVALID_ARG;
   moe_status st = validate_config(cfg);
   if (st != MOE_OK) return st;
+  if (e_begin < 0 || e_count < 1 || e_begin > cfg->n_routed - e_count) return MOE_ERR_INVALID_ARG;
   const bool mx = cfg->expert_dtype == MOE_DT_MXFP4 || cfg->expert_dtype == MOE_DT_MXFP8;
   const bool a8 = cfg->expert_dtype == MOE_DT_MXFP8;
   const void* req[] = {w->router_w, w->w1, w->w3, w->w2};
@@ -299,6 +308,8 @@ moe_status moe_create(const moe_config* cfg, const moe_weights* w, moe_stream_t 
   if (const char* f = std::getenv("MOE_TEST_FAIL_ALLOC_AFTER")) h->fail_after = std::atoi(f);
   h->mx = mx;
   h->a8 = a8;
+  h->e_begin = e_begin;
+  h->e_local = e_count;
   if (cudaGetDevice(&h->device) != cudaSuccess ||
       cudaDeviceGetAttribute(&h->num_sms, cudaDevAttrMultiProcessorCount, h->device) != cudaSuccess ||
       gemm_set_attributes() != cudaSuccess || gemm_mx_set_attributes() != cudaSuccess ||
@@ -307,16 +318,17 @@ moe_status moe_create(const moe_config* cfg, const moe_weights* w, moe_stream_t 
     delete h;
     return MOE_ERR_CUDA;
   }
-  const int64_t H = cfg->hidden, I = cfg->inter, E = cfg->n_routed, S = cfg->n_shared, k = cfg->top_k,
-                Tm = cfg->max_tokens;
-  h->G = static_cast<int>(E + S);
+  // E: the router's experts; El: the routed experts this instance holds
+  const int64_t H = cfg->hidden, I = cfg->inter, E = cfg->n_routed, El = e_count, S = cfg->n_shared,
+                k = cfg->top_k, Tm = cfg->max_tokens;
+  h->G = static_cast<int>(El + S);
   h->R = Tm * k + S * Tm;
   h->nchunks_max = static_cast<int>((Tm * k + kPermChunk - 1) / kPermChunk);
   h->m_tiles_gu = static_cast<int>(I / 128);
   h->m_tiles_dn = static_cast<int>(H / 128);
   h->max_tiles_gu = h->m_tiles_gu * (h->G + (h->R + 31) / 32);
   h->max_tiles_dn = h->m_tiles_dn * (h->G + (h->R + 31) / 32);
-  h->max_ntiles_r = E + (Tm * k + 31) / 32;
+  h->max_ntiles_r = El + (Tm * k + 31) / 32;
 
   bool ok = true;
   uint64_t* wb = &h->weight_bytes;
@@ -324,14 +336,14 @@ moe_status moe_create(const moe_config* cfg, const moe_weights* w, moe_stream_t 
   ok = ok && h->alloc(&h->wg, E * H * 2, wb);
   if (w->router_bias) ok = ok && h->alloc(&h->bias, E * 4, wb);
   if (!mx) {
-    ok = ok && h->alloc(&h->w13, (E + S) * 2 * I * H * 2, wb);
-    ok = ok && h->alloc(&h->w2, (E + S) * H * I * 2, wb);
+    ok = ok && h->alloc(&h->w13, (El + S) * 2 * I * H * 2, wb);
+    ok = ok && h->alloc(&h->w2, (El + S) * H * I * 2, wb);
     if (!kGatherX) ok = ok && h->alloc(&h->xp, Tm * k * H * 2, ws);
   } else {
-    ok = ok && h->alloc(&h->w13q, E * 2 * I * (a8 ? H : H / 2), wb);
-    ok = ok && h->alloc(&h->w2q, E * H * (a8 ? I : I / 2), wb);
-    ok = ok && h->alloc(&h->sfa13, E * (I / 128) * (H / 128) * 1024, wb);
-    ok = ok && h->alloc(&h->sfa2, E * (H / 128) * (I / 128) * 512, wb);
+    ok = ok && h->alloc(&h->w13q, El * 2 * I * (a8 ? H : H / 2), wb);
+    ok = ok && h->alloc(&h->w2q, El * H * (a8 ? I : I / 2), wb);
+    ok = ok && h->alloc(&h->sfa13, El * (I / 128) * (H / 128) * 1024, wb);
+    ok = ok && h->alloc(&h->sfa2, El * (H / 128) * (I / 128) * 512, wb);
     if (S > 0) {
       ok = ok && h->alloc(&h->w13sh, S * 2 * I * H * 2, wb);
       ok = ok && h->alloc(&h->w2sh, S * H * I * 2, wb);
@@ -340,8 +352,8 @@ moe_status moe_create(const moe_config* cfg, const moe_weights* w, moe_stream_t 
     ok = ok && h->alloc(&h->hq, Tm * k * I, ws);
     ok = ok && h->alloc(&h->sfb_gu, h->max_ntiles_r * (H / 128) * 512, ws);
     ok = ok && h->alloc(&h->sfb_dn, h->max_ntiles_r * (I / 128) * 512, ws);
-    ok = ok && h->alloc(&h->ntile_base_gu, (E + 1) * 4, ws);
-    ok = ok && h->alloc(&h->ntile_base_dn, (E + 1) * 4, ws);
+    ok = ok && h->alloc(&h->ntile_base_gu, (El + 1) * 4, ws);
+    ok = ok && h->alloc(&h->ntile_base_dn, (El + 1) * 4, ws);
     ok = ok && h->alloc(&h->bad, 16, ws);
     if (S > 0) {
       const int64_t tsmall = Tm < kSmallRouterMaxTokens ? Tm : kSmallRouterMaxTokens;
@@ -355,9 +367,9 @@ moe_status moe_create(const moe_config* cfg, const moe_weights* w, moe_stream_t 
   ok = ok && h->alloc(&h->zpart, (H / 128) * (Tm < kSmallRouterMaxTokens ? Tm : kSmallRouterMaxTokens) * E * 4, ws);
   ok = ok && h->alloc(&h->idx, Tm * k * 4, ws);
   ok = ok && h->alloc(&h->wts, Tm * k * 4, ws);
-  ok = ok && h->alloc(&h->chunk_cnt, static_cast<size_t>(h->nchunks_max) * E * 4, ws);
-  ok = ok && h->alloc(&h->cnt, (E + S) * 4, ws);
-  ok = ok && h->alloc(&h->off, (E + S + 1) * 4, ws);
+  ok = ok && h->alloc(&h->chunk_cnt, static_cast<size_t>(h->nchunks_max) * El * 4, ws);
+  ok = ok && h->alloc(&h->cnt, (El + S) * 4, ws);
+  ok = ok && h->alloc(&h->off, (El + S + 1) * 4, ws);
   ok = ok && h->alloc(&h->perm, Tm * k * 4, ws);
   ok = ok && h->alloc(&h->inv, Tm * k * 4, ws);
   ok = ok && h->alloc(&h->bn_choice, 16, ws);
@@ -382,25 +394,25 @@ moe_status moe_create(const moe_config* cfg, const moe_weights* w, moe_stream_t 
   err |= cudaMemcpyAsync(h->wg, w->router_w, E * H * 2, cudaMemcpyDeviceToDevice, s) != cudaSuccess;
   if (w->router_bias) err |= cudaMemcpyAsync(h->bias, w->router_bias, E * 4, cudaMemcpyDeviceToDevice, s) != cudaSuccess;
   if (!mx) {
-    err |= launch_repack_w13(w->w1, w->w3, w->sh_w1, w->sh_w3, static_cast<int>(E), static_cast<int>(S),
+    err |= launch_repack_w13(w->w1, w->w3, w->sh_w1, w->sh_w3, static_cast<int>(El), static_cast<int>(S),
                              static_cast<int>(I), static_cast<int>(H), h->w13, s) != cudaSuccess;
-    err |= cudaMemcpyAsync(h->w2, w->w2, E * H * I * 2, cudaMemcpyDeviceToDevice, s) != cudaSuccess;
+    err |= cudaMemcpyAsync(h->w2, w->w2, El * H * I * 2, cudaMemcpyDeviceToDevice, s) != cudaSuccess;
     if (S > 0)
-      err |= cudaMemcpyAsync(static_cast<uint8_t*>(h->w2) + E * H * I * 2, w->sh_w2, S * H * I * 2,
+      err |= cudaMemcpyAsync(static_cast<uint8_t*>(h->w2) + El * H * I * 2, w->sh_w2, S * H * I * 2,
                              cudaMemcpyDeviceToDevice, s) != cudaSuccess;
-    err |= !make_tmap_bf16(&h->tm_w13, h->w13, (E + S) * 2 * I, H, 256);
-    err |= !make_tmap_bf16(&h->tm_w2, h->w2, (E + S) * H, I, 128);
+    err |= !make_tmap_bf16(&h->tm_w13, h->w13, (El + S) * 2 * I, H, 256);
+    err |= !make_tmap_bf16(&h->tm_w2, h->w2, (El + S) * H, I, 128);
     h->wide_ok = H % 256 == 0;
-    if (h->wide_ok) err |= !make_tmap_bf16(&h->tm_w2w, h->w2, (E + S) * H, I, 256);
+    if (h->wide_ok) err |= !make_tmap_bf16(&h->tm_w2w, h->w2, (El + S) * H, I, 256);
     if (!kGatherX) err |= !make_tmap_bf16(&h->tm_xp, h->xp, Tm * k, H, 32);
   } else {
     err |= cudaMemsetAsync(h->bad, 0, 16, s) != cudaSuccess;
-    err |= launch_repack_w13_bytes(w->w1, w->w3, nullptr, nullptr, static_cast<int>(E), 0, static_cast<int>(I),
+    err |= launch_repack_w13_bytes(w->w1, w->w3, nullptr, nullptr, static_cast<int>(El), 0, static_cast<int>(I),
                                    static_cast<int>(a8 ? H : H / 2), h->w13q, s) != cudaSuccess;
-    err |= cudaMemcpyAsync(h->w2q, w->w2, E * H * (a8 ? I : I / 2), cudaMemcpyDeviceToDevice, s) != cudaSuccess;
-    err |= launch_sf_atoms(w->s1, w->s3, static_cast<int>(E), static_cast<int>(I), static_cast<int>(H), h->sfa13,
+    err |= cudaMemcpyAsync(h->w2q, w->w2, El * H * (a8 ? I : I / 2), cudaMemcpyDeviceToDevice, s) != cudaSuccess;
+    err |= launch_sf_atoms(w->s1, w->s3, static_cast<int>(El), static_cast<int>(I), static_cast<int>(H), h->sfa13,
                            h->bad, s) != cudaSuccess;
-    err |= launch_sf_atoms(w->s2, nullptr, static_cast<int>(E), static_cast<int>(H), static_cast<int>(I), h->sfa2,
+    err |= launch_sf_atoms(w->s2, nullptr, static_cast<int>(El), static_cast<int>(H), static_cast<int>(I), h->sfa2,
                            h->bad, s) != cudaSuccess;
     if (S > 0) {
       err |= launch_repack_w13(nullptr, nullptr, w->sh_w1, w->sh_w3, 0, static_cast<int>(S), static_cast<int>(I),
@@ -419,16 +431,16 @@ moe_status moe_create(const moe_config* cfg, const moe_weights* w, moe_stream_t 
     if (!a8 && kMxPacked) {
       const CUtensorMapDataType u8 = CU_TENSOR_MAP_DATA_TYPE_UINT8;
       const CUtensorMapSwizzle none = CU_TENSOR_MAP_SWIZZLE_NONE;
-      err |= !make_tmap(&h->tm_w13q, h->w13q, u8, E * 2 * I, H / 2, H / 2, 64, 256, none);
-      err |= !make_tmap(&h->tm_w2q, h->w2q, u8, E * H, I / 2, I / 2, 64, 128, none);
+      err |= !make_tmap(&h->tm_w13q, h->w13q, u8, El * 2 * I, H / 2, H / 2, 64, 256, none);
+      err |= !make_tmap(&h->tm_w2q, h->w2q, u8, El * H, I / 2, I / 2, 64, 128, none);
       h->wide_ok = H % 256 == 0;
-      if (h->wide_ok) err |= !make_tmap(&h->tm_w2qw, h->w2q, u8, E * H, I / 2, I / 2, 64, 256, none);
+      if (h->wide_ok) err |= !make_tmap(&h->tm_w2qw, h->w2q, u8, El * H, I / 2, I / 2, 64, 256, none);
     } else {
       const CUtensorMapDataType wdt = a8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B;
-      err |= !make_tmap(&h->tm_w13q, h->w13q, wdt, E * 2 * I, H, a8 ? H : H / 2, 128, 256);
-      err |= !make_tmap(&h->tm_w2q, h->w2q, wdt, E * H, I, a8 ? I : I / 2, 128, 128);
+      err |= !make_tmap(&h->tm_w13q, h->w13q, wdt, El * 2 * I, H, a8 ? H : H / 2, 128, 256);
+      err |= !make_tmap(&h->tm_w2q, h->w2q, wdt, El * H, I, a8 ? I : I / 2, 128, 128);
       h->wide_ok = H % 256 == 0;
-      if (h->wide_ok) err |= !make_tmap(&h->tm_w2qw, h->w2q, wdt, E * H, I, a8 ? I : I / 2, 128, 256);
+      if (h->wide_ok) err |= !make_tmap(&h->tm_w2qw, h->w2q, wdt, El * H, I, a8 ? I : I / 2, 128, 256);
     }
     err |= !make_tmap(&h->tm_xq, h->xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, Tm * k, H, H, 128, 32);
     err |= !make_tmap(&h->tm_hq, h->hq, CU_TENSOR_MAP_DATA_TYPE_UINT8, Tm * k, I, I, 128, 32);
@@ -457,11 +469,28 @@ moe_status moe_create(const moe_config* cfg, const moe_weights* w, moe_stream_t 
   return MOE_OK;
 }
 
+}  // namespace
+
+extern "C" {
+
+moe_status moe_create(const moe_config* cfg, const moe_weights* w, moe_stream_t stream, moe_handle** out) {
+  return create_impl(cfg, w, 0, cfg != nullptr ? cfg->n_routed : 0, stream, out);
+}
+
+moe_status moe_create_ep(const moe_config* cfg, const moe_weights* w, int32_t expert_begin, int32_t expert_count,
+                         moe_stream_t stream, moe_handle** out) {
+  return create_impl(cfg, w, expert_begin, expert_count, stream, out);
+}
+
+}  // extern "C"
+
 namespace {
 
 // One layer invocation; token_ids != nullptr selects the hash routing of the
 // handle's table instead of the learned router and top-k.
-moe_status forward_impl(moe_handle* h, const void* x, const int32_t* token_ids, int32_t T, void* y,
+// y_f32: y is fp32 [T, H] and receives this instance's partial output (its expert
+// window's slots, plus the shared experts it holds), else BF16 [T, H].
+moe_status forward_impl(moe_handle* h, const void* x, const int32_t* token_ids, int32_t T, void* y, bool y_f32,
                         int32_t* topk_idx, float* topk_w, moe_stream_t stream) {
   if (h == nullptr) return MOE_ERR_INVALID_ARG;
   if (T < 0 || T > h->cfg.max_tokens) return MOE_ERR_INVALID_ARG;
@@ -490,7 +519,10 @@ moe_status forward_impl(moe_handle* h, const void* x, const int32_t* token_ids, 
     }
   } range(h, token_ids != nullptr);
   const moe_config& c = h->cfg;
+  // E: the router's experts; El: the routed expert groups this instance holds,
+  // experts [eb, eb + El)
   const int H = c.hidden, I = c.inter, E = c.n_routed, S = c.n_shared, k = c.top_k;
+  const int El = h->e_local, eb = h->e_begin;
   const int nslots = T * k;
   const int nchunks = (nslots + kPermChunk - 1) / kPermChunk;
   // Token tiles. Few tokens: 32-row tiles and deep smem rings (weight streaming).
@@ -564,13 +596,15 @@ moe_status forward_impl(moe_handle* h, const void* x, const int32_t* token_ids, 
   // 3. permutation and tile lists
   if (nchunks > 1) {
     h->prof_mark(kKPermCount, s);
-    MOE_TRY_CUDA(launch_perm_count(h->idx, nslots, E, h->chunk_cnt, h->status, s));
+    MOE_TRY_CUDA(launch_perm_count(h->idx, nslots, El, eb, E, h->chunk_cnt, h->status, s));
     h->prof_done(s);
   }
   ScanArgs sa{};
   sa.chunk_cnt = h->chunk_cnt;
   sa.nchunks = nchunks;
-  sa.E = E;
+  sa.E = El;
+  sa.e_begin = eb;
+  sa.e_global = E;
   sa.S = S;
   sa.T = T;
   sa.k = k;
@@ -600,7 +634,7 @@ moe_status forward_impl(moe_handle* h, const void* x, const int32_t* token_ids, 
     MOE_TRY_CUDA(launch_perm_scan(sa, s));
     h->prof_done(s);
     h->prof_mark(kKPermScatter, s);
-    MOE_TRY_CUDA(launch_perm_scatter(h->idx, nslots, E, h->chunk_cnt, h->perm, h->inv, s));
+    MOE_TRY_CUDA(launch_perm_scatter(h->idx, nslots, El, eb, h->chunk_cnt, h->perm, h->inv, s));
     h->prof_done(s);
   }
 
@@ -626,7 +660,7 @@ moe_status forward_impl(moe_handle* h, const void* x, const int32_t* token_ids, 
     a.ntiles = h->ntiles;
     a.num_kb = H / 64;
     a.a_rows_per_group = 2 * I;
-    a.n_routed = E;
+    a.n_routed = El;
     a.out = h->h;
     a.out_ld = I;
     a.out_rows = static_cast<int>(h->R);
@@ -648,7 +682,7 @@ moe_status forward_impl(moe_handle* h, const void* x, const int32_t* token_ids, 
     d.ntiles = h->ntiles + 1;
     d.num_kb = I / 64;
     d.a_rows_per_group = H;
-    d.n_routed = E;
+    d.n_routed = El;
     d.out = h->o;
     d.out_ld = H;
     d.out_rows = static_cast<int>(h->R);
@@ -667,8 +701,8 @@ moe_status forward_impl(moe_handle* h, const void* x, const int32_t* token_ids, 
   } else {
     // MXFP8 token rows of the routed slots
     h->prof_mark(kKQuantX, s);
-    MOE_TRY_CUDA(launch_quant_gather_mx(x, h->perm, h->idx, h->off, h->ntile_base_gu, nslots, k, H, bn_mx, h->xq,
-                                        h->sfb_gu, s));
+    MOE_TRY_CUDA(launch_quant_gather_mx(x, h->perm, h->idx, h->off, h->ntile_base_gu, nslots, k, H, bn_mx, eb,
+                                        h->xq, h->sfb_gu, s));
     h->prof_done(s);
     // 4a. routed gate/up on block-scaled MMAs (tiles after the shared ones)
     MxGemmArgs g{};
@@ -733,10 +767,10 @@ moe_status forward_impl(moe_handle* h, const void* x, const int32_t* token_ids, 
       GemmArgs a{};
       a.tiles = h->tiles_gu;
       a.ntiles = h->ntiles + 2;
-      a.group_base = E;
+      a.group_base = El;
       a.num_kb = H / 64;
       a.a_rows_per_group = 2 * I;
-      a.n_routed = E;
+      a.n_routed = El;
       a.out = h->h;
       a.out_ld = I;
       a.out_rows = static_cast<int>(h->R);
@@ -795,10 +829,10 @@ moe_status forward_impl(moe_handle* h, const void* x, const int32_t* token_ids, 
       GemmArgs a{};
       a.tiles = h->tiles_dn;
       a.ntiles = h->ntiles + 3;
-      a.group_base = E;
+      a.group_base = El;
       a.num_kb = I / 64;
       a.a_rows_per_group = H;
-      a.n_routed = E;
+      a.n_routed = El;
       a.out = h->o;
       a.out_ld = H;
       a.out_rows = static_cast<int>(h->R);
@@ -813,8 +847,8 @@ moe_status forward_impl(moe_handle* h, const void* x, const int32_t* token_ids, 
   // 6. weighted combine with the shared experts
   h->prof_mark(kKCombine, s);
   const bool parts = h->mx && S > 0 && T <= kSmallRouterMaxTokens;
-  MOE_TRY_CUDA(launch_combine(h->o, h->inv, h->wts, T, H, k, S, y, parts ? h->sh_parts_dn : nullptr,
-                              parts ? h->ks_dn : 0, s));
+  MOE_TRY_CUDA(launch_combine(h->o, h->inv, h->idx, eb, El, h->wts, T, H, k, S, y, y_f32,
+                              parts ? h->sh_parts_dn : nullptr, parts ? h->ks_dn : 0, s));
   h->prof_done(s);
   if (topk_idx) MOE_TRY_CUDA(cudaMemcpyAsync(topk_idx, h->idx, static_cast<size_t>(nslots) * 4, cudaMemcpyDefault, s));
   if (topk_w) MOE_TRY_CUDA(cudaMemcpyAsync(topk_w, h->wts, static_cast<size_t>(nslots) * 4, cudaMemcpyDefault, s));
@@ -824,9 +858,17 @@ moe_status forward_impl(moe_handle* h, const void* x, const int32_t* token_ids, 
 
 }  // namespace
 
+extern "C" {
+
 moe_status moe_forward(moe_handle* h, const void* x, int32_t T, void* y, int32_t* topk_idx, float* topk_w,
                        moe_stream_t stream) {
-  return forward_impl(h, x, nullptr, T, y, topk_idx, topk_w, stream);
+  if (h != nullptr && h->e_local != h->cfg.n_routed) return MOE_ERR_INVALID_ARG;  // an expert window: partial only
+  return forward_impl(h, x, nullptr, T, y, false, topk_idx, topk_w, stream);
+}
+
+moe_status moe_forward_partial(moe_handle* h, const void* x, int32_t T, float* y_partial, int32_t* topk_idx,
+                               float* topk_w, moe_stream_t stream) {
+  return forward_impl(h, x, nullptr, T, y_partial, true, topk_idx, topk_w, stream);
 }
 
 moe_status moe_set_hash_table(moe_handle* h, const int32_t* table, int32_t vocab, moe_stream_t stream) {
@@ -867,7 +909,8 @@ moe_status moe_forward_hashed(moe_handle* h, const void* x, const int32_t* token
     if (cudaGetDevice(&cur) != cudaSuccess || cur != h->device) return MOE_ERR_INVALID_ARG;
     if (!device_pointer_on(token_ids, h->device)) return MOE_ERR_INVALID_ARG;
   }
-  return forward_impl(h, x, token_ids, T, y, topk_idx, topk_w, stream);
+  if (h->e_local != h->cfg.n_routed) return MOE_ERR_INVALID_ARG;
+  return forward_impl(h, x, token_ids, T, y, false, topk_idx, topk_w, stream);
 }
 
 moe_status moe_forward_host(moe_handle* h, const void* x_host, int32_t T, void* y_host, int32_t* topk_idx_host,

@@ -107,11 +107,14 @@ cudaError_t launch_hash_table_check(const int32_t* table, int vocab, int k, int 
 
 // ---- permutation
 constexpr int kPermChunk = 1024;
-cudaError_t launch_perm_count(const int32_t* idx, int nslots, int E, int32_t* chunk_cnt, int* status,
-                              cudaStream_t s);
+// Expert window: this instance holds routed experts [e_begin, e_begin + E) of e_global
+// (the whole layer: e_begin 0, E = e_global); slots of other experts are skipped.
+cudaError_t launch_perm_count(const int32_t* idx, int nslots, int E, int e_begin, int e_global, int32_t* chunk_cnt,
+                              int* status, cudaStream_t s);
 struct ScanArgs {
   int32_t* chunk_cnt;
-  int nchunks, E, S, T, k;
+  int nchunks, E, S, T, k;     // E: routed groups of this instance (its expert window)
+  int e_begin, e_global;        // the window's first expert and the router's expert count
   int32_t* cnt;
   int32_t* off;
   int4* tiles_gu;
@@ -130,8 +133,8 @@ cudaError_t launch_perm_scan(const ScanArgs& a, cudaStream_t s);
 // count + scan + scatter in one launch when all slots fit one chunk
 cudaError_t launch_perm_fused(const ScanArgs& a, const int32_t* idx, int nslots, int32_t* perm, int32_t* inv,
                               int* status, cudaStream_t s);
-cudaError_t launch_perm_scatter(const int32_t* idx, int nslots, int E, const int32_t* chunk_base, int32_t* perm,
-                                int32_t* inv, cudaStream_t s);
+cudaError_t launch_perm_scatter(const int32_t* idx, int nslots, int E, int e_begin, const int32_t* chunk_base,
+                                int32_t* perm, int32_t* inv, cudaStream_t s);
 cudaError_t launch_gather_rows(const void* x, const int32_t* perm, int nrows, int k, int H, void* xp,
                                cudaStream_t s);
 
@@ -216,8 +219,8 @@ cudaError_t launch_gemm_mx_down(const CUtensorMap& tmA, const CUtensorMap& tmB, 
 // x rows of the routed slots -> MXFP8: xq[row] = E4M3 codes of x[perm[row] / k], scale
 // atoms by gate/up token tile.
 cudaError_t launch_quant_gather_mx(const void* x, const int32_t* perm, const int32_t* idx, const int32_t* off,
-                                   const int32_t* ntile_base_gu, int nrows, int k, int H, int bn_gu, uint8_t* xq,
-                                   uint8_t* sfb, cudaStream_t s);
+                                   const int32_t* ntile_base_gu, int nrows, int k, int H, int bn_gu, int e_begin,
+                                   uint8_t* xq, uint8_t* sfb, cudaStream_t s);
 // Weight scales [groups, rows, K/32] -> atoms [groups][rows/128][K/128][parts * 512]; for
 // gate/up the two parts are W1 and W3 of the same 128 rows. Codes 0xFF raise *bad.
 cudaError_t launch_sf_atoms(const uint8_t* s_a, const uint8_t* s_b, int groups, int rows, int K, uint8_t* dst,
@@ -230,8 +233,11 @@ cudaError_t launch_repack_w13_bytes(const void* w1, const void* w3, const void* 
 // ---- combine
 // sh_parts: when not null, the shared experts' outputs are the sum of n_parts fp32
 // slices [n_parts][S][T][H] (split-K partial sums) instead of O's shared rows.
-cudaError_t launch_combine(const float* O, const int32_t* inv, const float* w, int T, int H, int k, int S,
-                           void* y, const float* sh_parts, int n_parts, cudaStream_t s);
+// Only the slots whose expert (idx) lies in [e_begin, e_begin + e_count) are summed;
+// y is BF16, or fp32 when y_f32 (an expert-parallel partial output).
+cudaError_t launch_combine(const float* O, const int32_t* inv, const int32_t* idx, int e_begin, int e_count,
+                           const float* w, int T, int H, int k, int S, void* y, bool y_f32, const float* sh_parts,
+                           int n_parts, cudaStream_t s);
 // h[row0 + t] = clamped SwiGLU of the sum over n_parts slices of fp32 G | U rows [n_parts][T][2I].
 cudaError_t launch_swiglu_reduce(const float* parts, int n_parts, int T, int I, float limit, void* h,
                                  cudaStream_t s);

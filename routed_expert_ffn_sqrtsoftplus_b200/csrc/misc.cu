@@ -9,10 +9,14 @@ namespace {
 
 // y[t] = sum_shared O[T*k + j*T + t] + sum_j w[t, j] * O[inv[t*k + j]]
 // (shared experts have weight 1; the routed sum runs in slot order j = 0..k-1,
-// accumulated in fp32 and rounded once to BF16).
+// accumulated in fp32 and rounded once to BF16). Only slots whose expert lies in
+// this instance's window [e_begin, e_begin + e_count) count (all of them for a
+// whole layer); with y_f32 the sum is written in fp32 (an expert-parallel
+// partial output, summed over the instances afterwards).
 __global__ void __launch_bounds__(128)
-    combine_kernel(const float4* __restrict__ O, const int32_t* __restrict__ inv, const float* __restrict__ w, int T,
-                   int H4, int k, int S, uint2* __restrict__ y, const float4* __restrict__ sh_parts, int n_parts) {
+    combine_kernel(const float4* __restrict__ O, const int32_t* __restrict__ inv, const int32_t* __restrict__ idx,
+                   int e_begin, int e_count, const float* __restrict__ w, int T, int H4, int k, int S,
+                   void* __restrict__ y, int y_f32, const float4* __restrict__ sh_parts, int n_parts) {
   const int t = blockIdx.x;
   const int c = blockIdx.y * blockDim.x + threadIdx.x;
   if (c >= H4) return;
@@ -42,6 +46,8 @@ __global__ void __launch_bounds__(128)
     }
   }
   for (int j = 0; j < k; ++j) {
+    const int e = __ldg(idx + static_cast<size_t>(t) * k + j) - e_begin;
+    if (e < 0 || e >= e_count) continue;  // another instance's expert
     const int row = __ldg(inv + static_cast<size_t>(t) * k + j);
     // every slot's row is below T*k; the check keeps a corrupted row index from
     // reading outside O
@@ -53,12 +59,16 @@ __global__ void __launch_bounds__(128)
     acc.z = fmaf(wj, v.z, acc.z);
     acc.w = fmaf(wj, v.w, acc.w);
   }
+  if (y_f32) {
+    static_cast<float4*>(y)[static_cast<size_t>(t) * H4 + c] = acc;
+    return;
+  }
   __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y);
   __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z, acc.w);
   uint2 out;
   out.x = *reinterpret_cast<uint32_t*>(&lo);
   out.y = *reinterpret_cast<uint32_t*>(&hi);
-  y[static_cast<size_t>(t) * H4 + c] = out;
+  static_cast<uint2*>(y)[static_cast<size_t>(t) * H4 + c] = out;
 }
 
 // h[t, i] = silu(min(G, L)) * clamp(U, -L, L) with G, U the sums of the split-K
@@ -229,13 +239,14 @@ __global__ void wait_timeout_probe_kernel(int* status, unsigned long long timeou
 
 }  // namespace
 
-cudaError_t launch_combine(const float* O, const int32_t* inv, const float* w, int T, int H, int k, int S, void* y,
-                           const float* sh_parts, int n_parts, cudaStream_t s) {
+cudaError_t launch_combine(const float* O, const int32_t* inv, const int32_t* idx, int e_begin, int e_count,
+                           const float* w, int T, int H, int k, int S, void* y, bool y_f32, const float* sh_parts,
+                           int n_parts, cudaStream_t s) {
   if (T == 0) return cudaSuccess;
   const int H4 = H / 4;
   const dim3 grid(T, (H4 + 127) / 128);
-  combine_kernel<<<grid, 128, 0, s>>>(reinterpret_cast<const float4*>(O), inv, w, T, H4, k, S,
-                                      static_cast<uint2*>(y), reinterpret_cast<const float4*>(sh_parts), n_parts);
+  combine_kernel<<<grid, 128, 0, s>>>(reinterpret_cast<const float4*>(O), inv, idx, e_begin, e_count, w, T, H4, k,
+                                      S, y, y_f32 ? 1 : 0, reinterpret_cast<const float4*>(sh_parts), n_parts);
   return cudaGetLastError();
 }
 

@@ -21,20 +21,24 @@ constexpr int kMaxGroups = 1024;      // routed experts of the histogram and sca
 constexpr int kMaxScanGroups = 544;   // routed (<= 512) + shared (<= 4) groups of the scan kernel
 constexpr int kMaxSegs = 2 * kMaxScanGroups;  // tile-list segments (shared, full, partial)
 
+// Expert windows (expert parallelism): this layer instance holds routed experts
+// [e_begin, e_begin + E) of e_global; a slot whose expert lies outside the window
+// belongs to another instance and is skipped, one outside [0, e_global) is an error.
 __global__ void __launch_bounds__(256)
-    perm_count_kernel(const int32_t* __restrict__ idx, int nslots, int E, int32_t* __restrict__ chunk_cnt,
-                      int* status) {
+    perm_count_kernel(const int32_t* __restrict__ idx, int nslots, int E, int e_begin, int e_global,
+                      int32_t* __restrict__ chunk_cnt, int* status) {
   __shared__ int hist[kMaxGroups];
   for (int e = threadIdx.x; e < E; e += blockDim.x) hist[e] = 0;
   __syncthreads();
   const int base = blockIdx.x * kPermChunk;
   const int end = min(nslots, base + kPermChunk);
   for (int s = base + threadIdx.x; s < end; s += blockDim.x) {
-    const int e = idx[s];
-    if (e >= 0 && e < E)
-      atomicAdd(&hist[e], 1);
-    else
+    const int g = idx[s];
+    const int e = g - e_begin;
+    if (g < 0 || g >= e_global)
       report_status(status, kStatusDevice);
+    else if (e >= 0 && e < E)
+      atomicAdd(&hist[e], 1);
   }
   __syncthreads();
   for (int e = threadIdx.x; e < E; e += blockDim.x) chunk_cnt[static_cast<size_t>(blockIdx.x) * E + e] = hist[e];
@@ -92,11 +96,12 @@ __global__ void __launch_bounds__(1024) perm_scan_kernel(ScanArgs a, int fused, 
     for (int g = tid; g < a.E; g += blockDim.x) cnt_s[g] = 0;
     __syncthreads();
     for (int s = tid; s < nslots; s += blockDim.x) {
-      const int e = idx[s];
-      if (e >= 0 && e < a.E)
-        atomicAdd(&cnt_s[e], 1);
-      else
+      const int g = idx[s];
+      const int e = g - a.e_begin;
+      if (g < 0 || g >= a.e_global)
         report_status(status, kStatusDevice);
+      else if (e >= 0 && e < a.E)
+        atomicAdd(&cnt_s[e], 1);
     }
     __syncthreads();
     for (int g = a.E + tid; g < G; g += blockDim.x) cnt_s[g] = a.T;
@@ -252,7 +257,7 @@ __global__ void __launch_bounds__(1024) perm_scan_kernel(ScanArgs a, int fused, 
     __syncwarp();
     for (int b = 0; b < nslots; b += 32) {
       const int s = b + lane;
-      const int e = s < nslots ? idx[s] : -1;
+      const int e = s < nslots ? idx[s] - a.e_begin : -1;
       const bool valid = e >= 0 && e < a.E;
       const unsigned peers = __match_any_sync(0xffffffffu, valid ? e : -1);
       const int rank = __popc(peers & ((1u << lane) - 1u));
@@ -271,8 +276,9 @@ __global__ void __launch_bounds__(1024) perm_scan_kernel(ScanArgs a, int fused, 
 // One warp per chunk walks its slots in order, 32 at a time; peers with the
 // same expert get consecutive positions in lane order.
 __global__ void __launch_bounds__(32)
-    perm_scatter_kernel(const int32_t* __restrict__ idx, int nslots, int E, const int32_t* __restrict__ chunk_base,
-                        int32_t* __restrict__ perm, int32_t* __restrict__ inv) {
+    perm_scatter_kernel(const int32_t* __restrict__ idx, int nslots, int E, int e_begin,
+                        const int32_t* __restrict__ chunk_base, int32_t* __restrict__ perm,
+                        int32_t* __restrict__ inv) {
   __shared__ int ctr[kMaxGroups];
   const int lane = threadIdx.x;
   for (int e = lane; e < E; e += 32) ctr[e] = chunk_base[static_cast<size_t>(blockIdx.x) * E + e];
@@ -281,7 +287,7 @@ __global__ void __launch_bounds__(32)
   const int end = min(nslots, base + kPermChunk);
   for (int b = base; b < end; b += 32) {
     const int s = b + lane;
-    const int e = s < end ? idx[s] : -1;
+    const int e = s < end ? idx[s] - e_begin : -1;
     const bool valid = e >= 0 && e < E;
     const unsigned peers = __match_any_sync(0xffffffffu, valid ? e : -1);
     const int rank = __popc(peers & ((1u << lane) - 1u));
@@ -316,14 +322,14 @@ __global__ void __launch_bounds__(256)
 __global__ void __launch_bounds__(256)
     quant_gather_mx_kernel(const uint4* __restrict__ x, const int32_t* __restrict__ perm,
                            const int32_t* __restrict__ idx, const int32_t* __restrict__ off,
-                           const int32_t* __restrict__ ntile_base, int nrows, int k, int H, int bn,
+                           const int32_t* __restrict__ ntile_base, int nrows, int k, int H, int bn, int e_begin,
                            uint4* __restrict__ xq, uint8_t* __restrict__ sfb) {
   const int row = blockIdx.x * 8 + threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
   if (row >= nrows) return;
   const int slot = perm[row];
   const int t = slot / k;
-  const int g = idx[slot];
+  const int g = idx[slot] - e_begin;
   const int j = row - off[g];
   const int ntile = ntile_base[g] + j / bn;
   const int n = j % bn;
@@ -368,20 +374,20 @@ __global__ void __launch_bounds__(256)
 }  // namespace
 
 cudaError_t launch_quant_gather_mx(const void* x, const int32_t* perm, const int32_t* idx, const int32_t* off,
-                                   const int32_t* ntile_base_gu, int nrows, int k, int H, int bn_gu, uint8_t* xq,
-                                   uint8_t* sfb, cudaStream_t s) {
+                                   const int32_t* ntile_base_gu, int nrows, int k, int H, int bn_gu, int e_begin,
+                                   uint8_t* xq, uint8_t* sfb, cudaStream_t s) {
   if (nrows == 0) return cudaSuccess;
   quant_gather_mx_kernel<<<(nrows + 7) / 8, 256, 0, s>>>(static_cast<const uint4*>(x), perm, idx, off,
-                                                          ntile_base_gu, nrows, k, H, bn_gu,
+                                                          ntile_base_gu, nrows, k, H, bn_gu, e_begin,
                                                           reinterpret_cast<uint4*>(xq), sfb);
   return cudaGetLastError();
 }
 
-cudaError_t launch_perm_count(const int32_t* idx, int nslots, int E, int32_t* chunk_cnt, int* status,
-                              cudaStream_t s) {
+cudaError_t launch_perm_count(const int32_t* idx, int nslots, int E, int e_begin, int e_global, int32_t* chunk_cnt,
+                              int* status, cudaStream_t s) {
   if (E > kMaxGroups) return cudaErrorInvalidValue;
   const int nchunks = (nslots + kPermChunk - 1) / kPermChunk;
-  perm_count_kernel<<<nchunks, 256, 0, s>>>(idx, nslots, E, chunk_cnt, status);
+  perm_count_kernel<<<nchunks, 256, 0, s>>>(idx, nslots, E, e_begin, e_global, chunk_cnt, status);
   return cudaGetLastError();
 }
 
@@ -398,10 +404,10 @@ cudaError_t launch_perm_fused(const ScanArgs& a, const int32_t* idx, int nslots,
   return cudaGetLastError();
 }
 
-cudaError_t launch_perm_scatter(const int32_t* idx, int nslots, int E, const int32_t* chunk_base, int32_t* perm,
-                                int32_t* inv, cudaStream_t s) {
+cudaError_t launch_perm_scatter(const int32_t* idx, int nslots, int E, int e_begin, const int32_t* chunk_base,
+                                int32_t* perm, int32_t* inv, cudaStream_t s) {
   const int nchunks = (nslots + kPermChunk - 1) / kPermChunk;
-  perm_scatter_kernel<<<nchunks, 32, 0, s>>>(idx, nslots, E, chunk_base, perm, inv);
+  perm_scatter_kernel<<<nchunks, 32, 0, s>>>(idx, nslots, E, e_begin, chunk_base, perm, inv);
   return cudaGetLastError();
 }
 

@@ -43,7 +43,7 @@ def test_exports_are_exactly_the_header(L):
 
 
 def test_abi_version_and_strings(L):
-    assert L.moe_abi_version() == 2
+    assert L.moe_abi_version() == 3
     assert L.moe_status_string(moe.MOE_OK) == b"MOE_OK"
     assert L.moe_status_string(moe.MOE_ERR_TIMEOUT) == b"MOE_ERR_TIMEOUT"
     assert L.moe_num_kernel_kinds() == len(moe.kernel_names())
