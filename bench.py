@@ -283,26 +283,18 @@ def cpu_cores():
 
 # ----------------------------------------------------------------------------- main arms
 def read_stream_peak(dev, gib: float = 4.0, reps: int = 5):
-    """Read-only streaming bandwidth of this GPU in GB/s: the best of a few library
-    reductions over a buffer far larger than L2, timed with CUDA events. The weight
-    streams of the GEMMs only read, so this is the ceiling they can approach; the
-    copy bandwidth of MEASURED_PEAKS.json counts a read and a write per byte."""
-    n = int(gib * (1 << 30)) // 4
-    buf = torch.ones(n, dtype=torch.int32, device=dev)
-    best = 0.0
-    for op in (lambda t: t.max(), lambda t: t.sum(dtype=torch.int64)):
-        op(buf)
-        torch.cuda.synchronize()
-        for _ in range(reps):
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record()
-            op(buf)
-            e1.record()
-            torch.cuda.synchronize()
-            best = max(best, n * 4 / (e0.elapsed_time(e1) / 1e3) / 1e9)
-    del buf
-    torch.cuda.empty_cache()
-    return best
+    """Read-only streaming bandwidth of this GPU in GB/s (moe_read_bandwidth: one CTA
+    per SM keeps six 32 KiB bulk copies in flight over a 4 GiB buffer, far larger
+    than L2, and computes nothing). The GEMMs' weight streams only read, so this
+    is the ceiling they can approach; the copy bandwidth of MEASURED_PEAKS.json
+    counts a read and a write per byte."""
+    import routed_expert_ffn_sqrtsoftplus_b200 as moe
+    buf = torch.ones(int(gib * (1 << 30)) // 4, dtype=torch.int32, device=dev)
+    try:
+        return moe.read_bandwidth(buf, reps)
+    finally:
+        del buf
+        torch.cuda.empty_cache()
 
 
 def kernel_roofline(kern, prof, alg, hbm, tc, src, read_gbs, wl_name):
@@ -380,17 +372,18 @@ def measure(wl, steps, warmup, world, local, read_gbs=None, flush_l2=False, e2e_
 
     # ---- L2 flushed: a buffer twice the L2 size written before every timed step
     if flush_l2:
+        # every step's flush, events and forward enqueued back to back (the host never
+        # waits in between, so no step waits for its launches); the step time is the
+        # sum of the per-step event intervals, which exclude the flushes
         junk = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
-        tot = 0.0
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
         for i in range(steps):
             junk.fill_(float(i))
-            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            a.record(stream)
+            evs[i][0].record(stream)
             layer.forward(x, out=y)
-            b.record(stream)
-            b.synchronize()
-            tot += a.elapsed_time(b)
-        tot = max_over_ranks(tot, world)
+            evs[i][1].record(stream)
+        torch.cuda.synchronize()
+        tot = max_over_ranks(sum(a.elapsed_time(b) for a, b in evs), world)
         del junk
         res["l2_flushed"] = {"value": weak_scaling_value(world, T, steps, tot), "ms_per_step": tot / steps,
                              "flush": f"{2 * L2_BYTES >> 20} MiB written before each step, outside its events"}

@@ -300,6 +300,17 @@ MOE_API moe_status moe_inspect(moe_handle* h, int32_t what, void* dst, size_t by
  */
 MOE_API moe_status moe_fill_workspace(moe_handle* h, int32_t byte_value, moe_stream_t stream);
 
+/*
+ * Read-only streaming bandwidth of the current device, in GB/s (the roofline
+ * denominator of the weight-streaming kernels, which read without writing):
+ * one CTA per SM keeps six 32 KiB bulk copies (global -> shared memory) in
+ * flight over the whole of buf, reps times after one warm-up pass, timed with
+ * CUDA events on `stream`; synchronises. buf: device memory of at least 1 MiB,
+ * 16-byte aligned (far larger than L2 for a DRAM figure); bytes beyond a whole
+ * number of 32 KiB chunks are not read. Allocates a 4-byte status word.
+ */
+MOE_API moe_status moe_read_bandwidth(const void* buf, size_t bytes, int32_t reps, moe_stream_t stream, double* gbs);
+
 /* Limit, in nanoseconds, of every device-side wait of this handle's kernels
  * (default 2e9). A smaller value makes a stuck wait return sooner. */
 MOE_API moe_status moe_set_wait_timeout(moe_handle* h, uint64_t timeout_ns);

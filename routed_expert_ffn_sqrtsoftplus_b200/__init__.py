@@ -35,7 +35,7 @@ EXPORTED = ("moe_create", "moe_forward", "moe_forward_host", "moe_get_status", "
             "moe_selftest_wait_timeout", "moe_get_info", "moe_profile_begin", "moe_profile_end",
             "moe_num_kernel_kinds", "moe_kernel_name", "moe_route_noalloc", "moe_quantize_mxfp8",
             "moe_set_hash_table", "moe_forward_hashed", "moe_fill_workspace", "moe_create_ep",
-            "moe_forward_partial")
+            "moe_forward_partial", "moe_read_bandwidth")
 
 
 class MoEError(RuntimeError):
@@ -89,6 +89,7 @@ def lib() -> ctypes.CDLL:
             "moe_create_ep": (I32, [ctypes.POINTER(_Config), ctypes.POINTER(_Weights), I32, I32, P,
                                     ctypes.POINTER(P)]),
             "moe_forward_partial": (I32, [P, P, I32, P, P, P, P]),
+            "moe_read_bandwidth": (I32, [P, ctypes.c_size_t, I32, P, ctypes.POINTER(ctypes.c_double)]),
             "moe_forward_hashed": (I32, [P, P, P, I32, P, P, P, P]),
             "moe_inspect": (I32, [P, I32, P, ctypes.c_size_t, P]),
             "moe_set_wait_timeout": (I32, [P, U64]),
@@ -168,6 +169,16 @@ def quantize_mxfp8(w: torch.Tensor, stream=None):
     _check(lib().moe_quantize_mxfp8(_ptr(w), rows, K, _ptr(codes), _ptr(scales), _stream(stream)),
            "moe_quantize_mxfp8")
     return codes, scales
+
+
+def read_bandwidth(buf: torch.Tensor, reps: int = 5, stream=None) -> float:
+    """Read-only streaming bandwidth (GB/s) of the device holding `buf` (a large CUDA tensor)."""
+    if buf.device.type != "cuda" or not buf.is_contiguous():
+        raise ValueError("buf must be a contiguous CUDA tensor")
+    g = ctypes.c_double(0.0)
+    _check(lib().moe_read_bandwidth(_ptr(buf), buf.numel() * buf.element_size(), reps, _stream(stream),
+                                    ctypes.byref(g)), "moe_read_bandwidth")
+    return g.value
 
 
 class MoELayer:

@@ -1034,6 +1034,40 @@ moe_status moe_fill_workspace(moe_handle* h, int32_t byte_value, moe_stream_t st
   return MOE_OK;
 }
 
+moe_status moe_read_bandwidth(const void* buf, size_t bytes, int32_t reps, moe_stream_t stream, double* gbs) {
+  if (buf == nullptr || gbs == nullptr || reps < 1 || bytes < (size_t(1) << 20) || !aligned16(buf))
+    return MOE_ERR_INVALID_ARG;
+  int dev = -1, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || !device_pointer_on(buf, dev)) return MOE_ERR_INVALID_ARG;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return MOE_ERR_CUDA;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const size_t used = bytes / (32 * 1024) * (32 * 1024);
+  int* status = nullptr;
+  cudaEvent_t e0 = nullptr, e1 = nullptr;
+  moe_status st = MOE_OK;
+  if (cudaMalloc(&status, sizeof(int)) != cudaSuccess || cudaEventCreate(&e0) != cudaSuccess ||
+      cudaEventCreate(&e1) != cudaSuccess || cudaMemsetAsync(status, 0, sizeof(int), s) != cudaSuccess ||
+      launch_stream_read(buf, used, sms, status, 2000000000ull, s) != cudaSuccess ||  // warm-up
+      cudaEventRecord(e0, s) != cudaSuccess) {
+    st = MOE_ERR_CUDA;
+  }
+  for (int i = 0; st == MOE_OK && i < reps; ++i)
+    if (launch_stream_read(buf, used, sms, status, 2000000000ull, s) != cudaSuccess) st = MOE_ERR_CUDA;
+  float ms = 0.f;
+  int v = 0;
+  if (st == MOE_OK && (cudaEventRecord(e1, s) != cudaSuccess || cudaEventSynchronize(e1) != cudaSuccess ||
+                       cudaEventElapsedTime(&ms, e0, e1) != cudaSuccess ||
+                       cudaMemcpy(&v, status, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess))
+    st = MOE_ERR_CUDA;
+  if (st == MOE_OK && v != 0) st = MOE_ERR_TIMEOUT;
+  if (st == MOE_OK) *gbs = static_cast<double>(used) * reps / (ms * 1e-3) / 1e9;
+  cudaGetLastError();
+  if (e0) cudaEventDestroy(e0);
+  if (e1) cudaEventDestroy(e1);
+  if (status) cudaFree(status);
+  return st;
+}
+
 moe_status moe_set_wait_timeout(moe_handle* h, uint64_t timeout_ns) {
   if (h == nullptr || timeout_ns == 0) return MOE_ERR_INVALID_ARG;
   h->timeout_ns = timeout_ns;

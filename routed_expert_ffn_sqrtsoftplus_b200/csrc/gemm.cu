@@ -205,86 +205,140 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
 
   if (warp == kWarpTma) {
     // ------------------------------------------------------------ TMA producer
-    // Lane 0 waits on the ring and issues the weight box (and the token boxes of
-    // rows stored in order); with gathered token rows every lane issues the
-    // tile::gather4 loads of its own four-row groups.
-    constexpr int kGpl = (BN / 4 + 31) / 32;  // four-row groups per lane
-    int stage = 0;
-    uint32_t phase = 0;
-    long issued = 0;
-    bool ok = true;
-    // L2 prefetch cursor (lane 0): walks the same (tile, K block) sequence kPrefetch stages ahead
-    int pf_t = tfirst, pf_kb = 0, pf_row = 0, pf_kb0 = 0, pf_nkb = 0;
-    auto prefetch_next = [&]() {
-      if (pf_t >= ntiles) return;
-      if (pf_kb == 0) {
-        const Tile pt = load_tile<BN>(args, pf_t);
-        pf_row = (pt.group - args.group_base) * args.a_rows_per_group + pt.m_tile * C::kARows;
-        pf_kb0 = pt.kb0;
-        pf_nkb = pt.nkb;
-      }
-      if (pf_nkb > 0) tma_prefetch_2d(tmA, (pf_kb0 + pf_kb) * kBK, pf_row);
-      if (++pf_kb >= pf_nkb) {
-        pf_kb = 0;
-        pf_t += gridDim.x;
-      }
-    };
-    if constexpr (kPrefetch > 0)
-      if (lane == 0)
-        for (int i = 0; i < kPrefetch; ++i) prefetch_next();
-    for (int t = tfirst; ok && t < ntiles; t += gridDim.x) {
-      if (__shfl_sync(0xffffffffu, lane == 0 ? *abort_flag : 0, 0)) break;
-      const Tile tl = load_tile<BN>(args, t);
-      const bool gather = kGateUp && args.gather_perm != nullptr && tl.group < args.n_routed;
-      const CUtensorMap* mb = (kGateUp && tl.group >= args.n_routed) ? tmBsh : tmB;
-      const int a_row = (tl.group - args.group_base) * args.a_rows_per_group + tl.m_tile * C::kARows;
-      const int nb = (tl.nrows + kBBoxRows - 1) / kBBoxRows;
-      const int n4 = (tl.nrows + 3) / 4;
-      // token rows of this lane's four-row groups (the tile's last row repeated past its end)
-      int tok[kGpl][4];
-#pragma unroll
-      for (int u = 0; u < kGpl; ++u)
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int r = min(4 * (lane + 32 * u) + i, tl.nrows - 1);
-          tok[u][i] = (gather && r >= 0) ? args.gather_perm[tl.b_row0 + r] / args.gather_k : 0;
-        }
-      const uint32_t bytes = C::kABytes + (gather ? n4 * 4 * 128 : nb * kBBoxBytes);
-      for (int kb = 0; kb < tl.nkb; ++kb) {
-        int go = 1;
-        if (lane == 0) go = wait_or_abort(&empty[stage], phase ^ 1, args, abort_flag) ? 1 : 0;
-        if (!__shfl_sync(0xffffffffu, go, 0)) {
-          ok = false;
-          break;
-        }
-        const int kx = (tl.kb0 + kb) * kBK;
-        if (lane == 0) {
-          mbar_arrive_expect_tx(&full[stage], bytes);
-          tma_load_2d(sA + stage * C::kABytes, tmA, &full[stage], kx, a_row, kCacheEvictFirst);
-          if (!gather)
+    if constexpr (!kGatherX) {
+      // lane 0 waits on the ring and issues the weight box and the token boxes
+      if (lane == 0) {
+        int stage = 0;
+        uint32_t phase = 0;
+        long issued = 0;
+        bool ok = true;
+        // L2 prefetch cursor: walks the same (tile, K block) sequence kPrefetch stages ahead
+        int pf_t = tfirst, pf_kb = 0, pf_row = 0, pf_kb0 = 0, pf_nkb = 0;
+        auto prefetch_next = [&]() {
+          if (pf_t >= ntiles) return;
+          if (pf_kb == 0) {
+            const Tile pt = load_tile<BN>(args, pf_t);
+            pf_row = (pt.group - args.group_base) * args.a_rows_per_group + pt.m_tile * C::kARows;
+            pf_kb0 = pt.kb0;
+            pf_nkb = pt.nkb;
+          }
+          if (pf_nkb > 0) tma_prefetch_2d(tmA, (pf_kb0 + pf_kb) * kBK, pf_row);
+          if (++pf_kb >= pf_nkb) {
+            pf_kb = 0;
+            pf_t += gridDim.x;
+          }
+        };
+        if constexpr (kPrefetch > 0)
+          for (int i = 0; i < kPrefetch; ++i) prefetch_next();
+        for (int t = tfirst; ok && t < ntiles && !*abort_flag; t += gridDim.x) {
+          const Tile tl = load_tile<BN>(args, t);
+          const CUtensorMap* mb = (kGateUp && tl.group >= args.n_routed) ? tmBsh : tmB;
+          const int a_row = (tl.group - args.group_base) * args.a_rows_per_group + tl.m_tile * C::kARows;
+          const int nb = (tl.nrows + kBBoxRows - 1) / kBBoxRows;
+          const uint32_t bytes = C::kABytes + nb * kBBoxBytes;
+          for (int kb = 0; kb < tl.nkb; ++kb) {
+            if (!wait_or_abort(&empty[stage], phase ^ 1, args, abort_flag)) {
+              ok = false;
+              break;
+            }
+            mbar_arrive_expect_tx(&full[stage], bytes);
+            const int kx = (tl.kb0 + kb) * kBK;
+            tma_load_2d(sA + stage * C::kABytes, tmA, &full[stage], kx, a_row, kCacheEvictFirst);
             for (int j = 0; j < nb; ++j)
               tma_load_2d(sB + stage * C::kBBytes + j * kBBoxBytes, mb, &full[stage], kx, tl.b_row0 + j * kBBoxRows,
                           kCacheEvictLast);
-          if constexpr (kPrefetch > 0) prefetch_next();
-        }
-        __syncwarp();
-        if (gather) {
-#pragma unroll
-          for (int u = 0; u < kGpl; ++u) {
-            const int g = lane + 32 * u;
-            if (g < n4)
-              tma_gather4(sB + stage * C::kBBytes + g * 4 * 128, tmB, &full[stage], kx, tok[u][0], tok[u][1],
-                          tok[u][2], tok[u][3]);
+            if constexpr (kPrefetch > 0) prefetch_next();
+            ++issued;
+            if (++stage == kStages) {
+              stage = 0;
+              phase ^= 1;
+            }
           }
         }
-        ++issued;
-        if (++stage == kStages) {
-          stage = 0;
-          phase ^= 1;
+        if (*abort_flag) drain_ring(full, kStages, issued, args.timeout_ns);
+      }
+    } else {
+      // Lane 0 waits on the ring and issues the weight box (and the token boxes of
+      // rows stored in order); with gathered token rows every lane issues the
+      // tile::gather4 loads of its own four-row groups.
+      constexpr int kGpl = (BN / 4 + 31) / 32;  // four-row groups per lane
+      int stage = 0;
+      uint32_t phase = 0;
+      long issued = 0;
+      bool ok = true;
+      // L2 prefetch cursor (lane 0): walks the same (tile, K block) sequence kPrefetch stages ahead
+      int pf_t = tfirst, pf_kb = 0, pf_row = 0, pf_kb0 = 0, pf_nkb = 0;
+      auto prefetch_next = [&]() {
+        if (pf_t >= ntiles) return;
+        if (pf_kb == 0) {
+          const Tile pt = load_tile<BN>(args, pf_t);
+          pf_row = (pt.group - args.group_base) * args.a_rows_per_group + pt.m_tile * C::kARows;
+          pf_kb0 = pt.kb0;
+          pf_nkb = pt.nkb;
+        }
+        if (pf_nkb > 0) tma_prefetch_2d(tmA, (pf_kb0 + pf_kb) * kBK, pf_row);
+        if (++pf_kb >= pf_nkb) {
+          pf_kb = 0;
+          pf_t += gridDim.x;
+        }
+      };
+      if constexpr (kPrefetch > 0)
+        if (lane == 0)
+          for (int i = 0; i < kPrefetch; ++i) prefetch_next();
+      for (int t = tfirst; ok && t < ntiles; t += gridDim.x) {
+        if (__shfl_sync(0xffffffffu, lane == 0 ? *abort_flag : 0, 0)) break;
+        const Tile tl = load_tile<BN>(args, t);
+        const bool gather = kGateUp && args.gather_perm != nullptr && tl.group < args.n_routed;
+        const CUtensorMap* mb = (kGateUp && tl.group >= args.n_routed) ? tmBsh : tmB;
+        const int a_row = (tl.group - args.group_base) * args.a_rows_per_group + tl.m_tile * C::kARows;
+        const int nb = (tl.nrows + kBBoxRows - 1) / kBBoxRows;
+        const int n4 = (tl.nrows + 3) / 4;
+        // token rows of this lane's four-row groups (the tile's last row repeated past its end)
+        int tok[kGpl][4];
+  #pragma unroll
+        for (int u = 0; u < kGpl; ++u)
+  #pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int r = min(4 * (lane + 32 * u) + i, tl.nrows - 1);
+            tok[u][i] = (gather && r >= 0) ? args.gather_perm[tl.b_row0 + r] / args.gather_k : 0;
+          }
+        const uint32_t bytes = C::kABytes + (gather ? n4 * 4 * 128 : nb * kBBoxBytes);
+        for (int kb = 0; kb < tl.nkb; ++kb) {
+          int go = 1;
+          if (lane == 0) go = wait_or_abort(&empty[stage], phase ^ 1, args, abort_flag) ? 1 : 0;
+          if (!__shfl_sync(0xffffffffu, go, 0)) {
+            ok = false;
+            break;
+          }
+          const int kx = (tl.kb0 + kb) * kBK;
+          if (lane == 0) {
+            mbar_arrive_expect_tx(&full[stage], bytes);
+            tma_load_2d(sA + stage * C::kABytes, tmA, &full[stage], kx, a_row, kCacheEvictFirst);
+            if (!gather)
+              for (int j = 0; j < nb; ++j)
+                tma_load_2d(sB + stage * C::kBBytes + j * kBBoxBytes, mb, &full[stage], kx, tl.b_row0 + j * kBBoxRows,
+                            kCacheEvictLast);
+            if constexpr (kPrefetch > 0) prefetch_next();
+          }
+          __syncwarp();
+          if (gather) {
+  #pragma unroll
+            for (int u = 0; u < kGpl; ++u) {
+              const int g = lane + 32 * u;
+              if (g < n4)
+                tma_gather4(sB + stage * C::kBBytes + g * 4 * 128, tmB, &full[stage], kx, tok[u][0], tok[u][1],
+                            tok[u][2], tok[u][3]);
+            }
+          }
+          ++issued;
+          if (++stage == kStages) {
+            stage = 0;
+            phase ^= 1;
+          }
         }
       }
+      if (lane == 0 && *abort_flag) drain_ring(full, kStages, issued, args.timeout_ns);
     }
-    if (lane == 0 && *abort_flag) drain_ring(full, kStages, issued, args.timeout_ns);
   } else if (warp == kWarpMma) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {

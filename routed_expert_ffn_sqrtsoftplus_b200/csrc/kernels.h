@@ -52,8 +52,11 @@ struct GemmArgs {
 };
 // The BF16 gate/up GEMM fetches the routed token rows straight from x through the
 // permutation (tile::gather4) instead of a gathered copy (1), or reads the copy (0).
+// Measured on B200: the gathers (a TMA instruction per four 128-byte rows, up to 64
+// per ring stage) made gate/up 1.7x slower at prefill than the copy kernel plus
+// 32-row boxes, so the copy is the default.
 #ifndef MOE_GATHER_X
-#define MOE_GATHER_X 1
+#define MOE_GATHER_X 0
 #endif
 constexpr bool kGatherX = MOE_GATHER_X != 0;
 
@@ -251,6 +254,10 @@ cudaError_t launch_quantize_mxfp8(const void* src, int64_t rows, int cols, uint8
 // ---- repack
 cudaError_t launch_repack_w13(const void* w1, const void* w3, const void* sh1, const void* sh3, int E, int S,
                               int I, int H, void* w13, cudaStream_t s);
+
+// ---- read-only streaming (roofline denominator): reads bytes / 32 KiB chunks of buf
+cudaError_t launch_stream_read(const void* buf, size_t bytes, int grid, int* status, unsigned long long timeout_ns,
+                               cudaStream_t s);
 
 // ---- self test
 cudaError_t launch_wait_timeout_probe(int* status, unsigned long long timeout_ns, cudaStream_t s);

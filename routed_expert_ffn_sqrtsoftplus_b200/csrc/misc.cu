@@ -223,6 +223,45 @@ __global__ void __launch_bounds__(256)
   scales[b] = static_cast<uint8_t>(code);
 }
 
+// Read-only streaming: one thread per CTA keeps kReadStages bulk copies of
+// kReadChunk bytes (global -> this CTA's shared memory) in flight over its
+// chunks (every gridDim-th one), the way the GEMMs' producers stream weights,
+// and computes nothing. Waits are bounded; a wait that runs out sets the status.
+constexpr int kReadStages = 6;
+constexpr int kReadChunk = 32 * 1024;
+
+__global__ void __launch_bounds__(32)
+    stream_read_kernel(const uint8_t* __restrict__ buf, long nchunks, int* status,
+                       unsigned long long timeout_ns) {
+  extern __shared__ __align__(1024) uint8_t ring[];
+  __shared__ uint64_t bar[kReadStages];
+  if (threadIdx.x != 0) return;
+  for (int i = 0; i < kReadStages; ++i) mbar_init(&bar[i], 1);
+  fence_mbarrier_init();
+  long next = blockIdx.x;
+  long issued = 0;
+  for (int i = 0; i < kReadStages && next < nchunks; ++i, next += gridDim.x, ++issued) {
+    mbar_arrive_expect_tx(&bar[i], kReadChunk);
+    bulk_load(ring + i * kReadChunk, buf + next * kReadChunk, kReadChunk, &bar[i], kCacheEvictFirst);
+  }
+  for (long done = 0; done < issued; ++done) {
+    const int st = static_cast<int>(done % kReadStages);
+    if (!mbar_wait(&bar[st], static_cast<uint32_t>((done / kReadStages) & 1), timeout_ns)) {
+      report_status(status, kStatusTimeout);
+      // let the copies still in flight land before the CTA exits
+      for (long j = done + 1; j < issued; ++j)
+        mbar_wait(&bar[j % kReadStages], static_cast<uint32_t>((j / kReadStages) & 1), timeout_ns);
+      return;
+    }
+    if (next < nchunks) {
+      mbar_arrive_expect_tx(&bar[st], kReadChunk);
+      bulk_load(ring + st * kReadChunk, buf + next * kReadChunk, kReadChunk, &bar[st], kCacheEvictFirst);
+      next += gridDim.x;
+      ++issued;
+    }
+  }
+}
+
 __global__ void wait_timeout_probe_kernel(int* status, unsigned long long timeout_ns) {
   __shared__ uint64_t bar;
   if (threadIdx.x == 0) {
@@ -297,6 +336,17 @@ cudaError_t launch_quantize_mxfp8(const void* src, int64_t rows, int cols, uint8
   if (nblocks == 0) return cudaSuccess;
   quantize_mxfp8_kernel<<<static_cast<unsigned>((nblocks + 255) / 256), 256, 0, s>>>(
       static_cast<const uint4*>(src), nblocks, reinterpret_cast<uint4*>(codes), scales);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_stream_read(const void* buf, size_t bytes, int grid, int* status, unsigned long long timeout_ns,
+                               cudaStream_t s) {
+  const long nchunks = static_cast<long>(bytes / kReadChunk);
+  if (nchunks == 0) return cudaSuccess;
+  const int smem = kReadStages * kReadChunk;
+  cudaError_t e = cudaFuncSetAttribute(stream_read_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  stream_read_kernel<<<grid, 32, smem, s>>>(static_cast<const uint8_t*>(buf), nchunks, status, timeout_ns);
   return cudaGetLastError();
 }
 
