@@ -20,6 +20,11 @@ namespace {
 constexpr int kMaxGroups = 1024;      // routed experts of the histogram and scatter kernels
 constexpr int kMaxScanGroups = 544;   // routed (<= 512) + shared (<= 4) groups of the scan kernel
 constexpr int kMaxSegs = 2 * kMaxScanGroups;  // tile-list segments (shared, full, partial)
+// Partial token tiles by row count, descending (1), or in group order (0).
+#ifndef MOE_TILE_ORDER_LPT
+#define MOE_TILE_ORDER_LPT 1
+#endif
+constexpr bool kTileOrderLongestFirst = MOE_TILE_ORDER_LPT != 0;
 
 // Expert windows (expert parallelism): this layer instance holds routed experts
 // [e_begin, e_begin + E) of e_global; a slot whose expert lies outside the window
@@ -165,7 +170,7 @@ __global__ void __launch_bounds__(1024) perm_scan_kernel(ScanArgs a, int fused, 
         int rank = 0;
         for (int h = 0; h < a.E; ++h) {
           const int rh = rem_s[h];
-          rank += (rh > rg) || (rh == rg && h < g);
+          rank += kTileOrderLongestFirst ? (rh > rg) || (rh == rg && h < g) : (rh > 0 && h < g);
         }
         part_g[list][rank] = g;
       }
