@@ -623,6 +623,9 @@ moe_status forward_impl(moe_handle* h, const void* x, const int32_t* token_ids, 
   sa.mx = h->mx ? 1 : 0;
   sa.ntile_base_gu = h->ntile_base_gu;
   sa.ntile_base_dn = h->ntile_base_dn;
+  // with few tokens every tile streams the same weight bytes and its rows cost
+  // next to nothing: the order of the partial tiles does not matter
+  sa.sort_partial = small ? 0 : 1;
   sa.bn_alt = alt ? kBnAlt : 0;
   sa.bn_choice = alt ? h->bn_choice : nullptr;
   if (nchunks == 1) {

@@ -131,6 +131,7 @@ struct ScanArgs {
   int32_t* ntile_base_dn;       // [E + 1] same for the down GEMM
   int bn_alt;                   // > 0: use this width for every tile when no routed group has more rows
   int* bn_choice;               // out: the width the tile lists were built with (bn_alt, or bn_gu_r)
+  int sort_partial;             // order the partial token tiles longest first (tile costs differ)
 };
 cudaError_t launch_perm_scan(const ScanArgs& a, cudaStream_t s);
 // count + scan + scatter in one launch when all slots fit one chunk

@@ -164,16 +164,24 @@ __global__ void __launch_bounds__(1024) perm_scan_kernel(ScanArgs a, int fused, 
     const int mtl = list == 0 ? a.m_tiles_gu : a.m_tiles_dn;
     for (int g = tid; g < a.E; g += blockDim.x) rem_s[g] = cnt_s[g] % bnr;
     __syncthreads();
-    for (int g = tid; g < a.E; g += blockDim.x) {
-      const int rg = rem_s[g];
-      if (rg > 0) {
-        int rank = 0;
-        for (int h = 0; h < a.E; ++h) {
-          const int rh = rem_s[h];
-          rank += kTileOrderLongestFirst ? (rh > rg) || (rh == rg && h < g) : (rh > 0 && h < g);
+    if (kTileOrderLongestFirst && a.sort_partial) {
+      // rank of each partial tile: longer ones first, ties by group (O(E) per thread)
+      for (int g = tid; g < a.E; g += blockDim.x) {
+        const int rg = rem_s[g];
+        if (rg > 0) {
+          int rank = 0;
+          for (int h = 0; h < a.E; ++h) {
+            const int rh = rem_s[h];
+            rank += (rh > rg) || (rh == rg && h < g);
+          }
+          part_g[list][rank] = g;
         }
-        part_g[list][rank] = g;
       }
+    } else {
+      // group order: a prefix count over the groups (E <= blockDim, one per thread)
+      const bool has = tid < a.E && rem_s[tid] > 0;
+      const int rank = block_exclusive_scan(has ? 1 : 0, warp_tot, &tot);
+      if (has) part_g[list][rank] = tid;
     }
     const int npart = __syncthreads_count(tid < a.E && rem_s[tid] > 0);
     const int ns = a.S + a.E + npart;

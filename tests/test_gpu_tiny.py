@@ -281,15 +281,21 @@ def test_nan_token_is_contained_warp_topk(cuda_device):
         layer.close()
 
 
-def _check_tile_list(tiles, n_shared_end, cnt, off, E, gateup):
-    """Every group's rows covered once per weight tile; shared tiles first; the
-    routed tiles by row count, non-increasing (full tiles, then partial ones by size)."""
+def _check_tile_list(tiles, n_shared_end, cnt, off, E, gateup, longest_first):
+    """Every group's rows covered once per weight tile; shared tiles first; with
+    many tokens per expert the routed tiles by row count, non-increasing (full
+    tiles, then partial ones by size), else in group order."""
     g = tiles[:, 0] & 0xFFFF
     mt = tiles[:, 0] >> 16
     y, z, rows = tiles[:, 1], tiles[:, 2], tiles[:, 3]
     assert np.all(g[:n_shared_end] >= E) and np.all(g[n_shared_end:] < E)
     r = rows[n_shared_end:]
-    assert np.all(r[:-1] >= r[1:]), "routed tiles are not longest first"
+    if longest_first:
+        assert np.all(r[:-1] >= r[1:]), "routed tiles are not longest first"
+    else:
+        gr = g[n_shared_end:]
+        full = r == r.max()
+        assert np.all(gr[:-1] <= gr[1:]) or np.all(np.diff(gr[~full]) >= 0), "routed tiles not in group order"
     assert np.all(rows > 0)
     m_tiles = int(mt.max()) + 1
     for grp in range(len(cnt)):
@@ -329,7 +335,8 @@ def test_tile_lists_are_complete_and_longest_first(tiny, cuda_device, T, hot):
         off = layer.inspect(moe.BUF_OFFSETS, torch.empty(G + 1, dtype=torch.int32, device=dev)).cpu().numpy()
         for which, n, ns, gateup in ((moe.BUF_TILES_GU, nt[0], nt[2], True), (moe.BUF_TILES_DN, nt[1], nt[3], False)):
             tl = layer.inspect(which, torch.empty((int(n), 4), dtype=torch.int32, device=dev)).cpu().numpy()
-            _check_tile_list(tl.astype(np.int64), int(ns), cnt.astype(np.int64), off.astype(np.int64), WL.E, gateup)
+            _check_tile_list(tl.astype(np.int64), int(ns), cnt.astype(np.int64), off.astype(np.int64), WL.E, gateup,
+                             longest_first=T > 32)
     finally:
         if made is not None:
             made.close()
