@@ -729,6 +729,8 @@ moe_status forward_impl(moe_handle* h, const void* x, const int32_t* token_ids, 
     g.dn_ntile_base = h->ntile_base_dn;
     g.status = h->status;
     g.timeout_ns = h->timeout_ns;
+    g.a_base = h->w13q;
+    g.a_row_bytes = h->a8 ? H : H / 2;
     h->prof_mark(kKGateUpMx, s);
     MOE_TRY_CUDA(launch_gemm_mx_gateup(h->tm_w13q, h->tm_xq, g, bn_mx, h->num_sms, s, h->a8));
     h->prof_done(s);
@@ -801,6 +803,8 @@ moe_status forward_impl(moe_handle* h, const void* x, const int32_t* token_ids, 
     d.m_limit = H;
     d.status = h->status;
     d.timeout_ns = h->timeout_ns;
+    d.a_base = h->w2q;
+    d.a_row_bytes = h->a8 ? I : I / 2;
     h->prof_mark(kKDownMx, s);
     MOE_TRY_CUDA(
         launch_gemm_mx_down(wide_mx ? h->tm_w2qw : h->tm_w2q, h->tm_hq, d, bn_mx, h->num_sms, s, wide_mx, h->a8));

@@ -50,6 +50,13 @@ constexpr int kAtomBytes = 512;   // scale factors of 128 rows x 4 blocks
 #define MOE_MX_PREFETCH 0
 #endif
 constexpr int kPrefetch = MOE_MX_PREFETCH;
+// At the start of each tile, prefetch into L2 this many quarters of the weights
+// of the CTA's next tile (contiguous in the repacked layout) with bulk prefetches
+// (0 = none).
+#ifndef MOE_MX_TILE_PREFETCH
+#define MOE_MX_TILE_PREFETCH 0
+#endif
+constexpr int kTilePrefetchQuarters = MOE_MX_TILE_PREFETCH;
 
 constexpr int pow2_at_least(int v, int lo) {
   int p = lo;
@@ -202,6 +209,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int t = tfirst; t < tend && !*abort_flag; t += gridDim.x) {
         const Tile tl = load_tile<BN>(args, t);
         const int a_row = tl.group * args.a_rows_per_group + tl.m_tile * C::kARows;
+        if constexpr (kTilePrefetchQuarters > 0) {
+          if (t + static_cast<int>(gridDim.x) < tend && args.a_base != nullptr) {
+            const Tile nt = load_tile<BN>(args, t + gridDim.x);
+            const uint8_t* src = args.a_base + (static_cast<size_t>(nt.group) * args.a_rows_per_group +
+                                                static_cast<size_t>(nt.m_tile) * C::kARows) * args.a_row_bytes;
+            const size_t total = static_cast<size_t>(C::kARows) * args.a_row_bytes * kTilePrefetchQuarters / 4;
+            for (size_t o = 0; o + 32768 <= total; o += 32768) bulk_prefetch_l2(src + o, 32768);
+          }
+        }
         const int nb = (tl.nrows + kBBoxRows - 1) / kBBoxRows;
         const uint32_t bytes = C::kATx + nb * kBBoxBytes + C::kSfBytes;
         // W1|W3 atoms: [group][m tile][k block][2 x 512 B]; W2 atoms: [group][128-row

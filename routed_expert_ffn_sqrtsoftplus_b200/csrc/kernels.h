@@ -212,6 +212,8 @@ struct MxGemmArgs {
   const int32_t* dn_ntile_base; // first down token tile of each group
   int* status;
   unsigned long long timeout_ns;
+  const uint8_t* a_base;        // the weights as stored: a tile's rows are contiguous, a_row_bytes each
+  int a_row_bytes;
 };
 cudaError_t gemm_mx_set_attributes();
 // a_fp8: the weights are MXFP8 (E4M3, one byte per value) instead of MXFP4
