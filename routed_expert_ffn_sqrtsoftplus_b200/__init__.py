@@ -383,6 +383,8 @@ class MoELayer:
         S = layer["sh_w1"].shape[0] if (with_shared and layer.get("sh_w1") is not None) else 0
         sh = {n: (layer.get(n) if S > 0 else None) for n in ("sh_w1", "sh_w3", "sh_w2")}
         b, c = (0, None) if expert_window is None else expert_window
+        if expert_window is not None and not (0 <= b and 1 <= c and b + c <= E):
+            raise ValueError(f"expert window {expert_window} is not inside [0, {E})")
         cut = (lambda t: t) if expert_window is None else (lambda t: t[b:b + c].contiguous())
         kw = dict(hidden=H, inter=I, n_routed=E, n_shared=S, top_k=top_k, max_tokens=max_tokens,
                   router_w=layer["wg"], router_bias=layer.get("bias"), route_scale=route_scale,

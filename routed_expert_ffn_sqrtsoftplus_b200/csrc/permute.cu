@@ -137,11 +137,14 @@ __global__ void __launch_bounds__(1024) perm_scan_kernel(ScanArgs a, int fused, 
   if (tid == 0 && a.bn_choice != nullptr) *a.bn_choice = alt ? a.bn_alt : a.bn_gu_r;
   // 2. scans (G <= 1024: one group per thread)
   {
+    // rows: the routed groups packed from 0 in group order; shared group j always
+    // at T*k + j*T (where the combine and the split shared GEMMs read it), also
+    // when an expert window holds fewer than T*k routed rows
     const int g = tid;
-    const int n = g < G ? cnt_s[g] : 0;
+    const int n = g < a.E ? cnt_s[g] : 0;
     int o = block_exclusive_scan(n, warp_tot, &tot);
-    if (g < G) off_s[g] = o;
-    if (tid == 0) off_s[G] = tot;
+    if (g < a.E) off_s[g] = o;
+    else if (g <= G) off_s[g] = a.T * a.k + (g - a.E) * a.T;
     // token-tile bases of the routed groups, in group order (MX scale atoms)
     const bool routed = g < a.E;
     int ng = block_exclusive_scan(routed ? (n + bn_gu_r - 1) / bn_gu_r : 0, warp_tot, &tot);

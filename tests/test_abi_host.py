@@ -101,6 +101,15 @@ def test_create_rejects_bad_pointers(L, wkw):
     assert L.moe_create(ctypes.byref(_cfg()), ctypes.byref(_w()), None, None) == moe.MOE_ERR_INVALID_ARG
 
 
+def test_create_ep_rejects_bad_windows(L):
+    h = ctypes.c_void_p()
+    E = _cfg().n_routed
+    for b, c in ((-1, 2), (0, 0), (E - 1, 2), (E, 1)):
+        assert L.moe_create_ep(ctypes.byref(_cfg()), ctypes.byref(_w()), b, c, None, ctypes.byref(h)) == \
+            moe.MOE_ERR_INVALID_ARG
+        assert not h.value
+
+
 def test_null_handle_calls(L):
     assert L.moe_forward(None, FAKE, 1, FAKE, None, None, None) == moe.MOE_ERR_INVALID_ARG
     assert L.moe_forward_host(None, FAKE, 1, FAKE, None, None, None) == moe.MOE_ERR_INVALID_ARG
