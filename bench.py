@@ -210,6 +210,9 @@ def algorithmic(wl, idx: np.ndarray, T: int):
     else:
         kern["gemm_gateup"] = (U * routed13 + S * shared13 + (rr + rs) * (H + I) * 2, (rr + rs) * 4 * H * I)
         kern["gemm_down"] = (U * routed2 + S * shared2 + (rr + rs) * (I * 2 + H * 4), (rr + rs) * 2 * H * I)
+        # few tokens: gate/up and down run as one launch
+        kern["gemm_fused"] = (kern["gemm_gateup"][0] + kern["gemm_down"][0],
+                              kern["gemm_gateup"][1] + kern["gemm_down"][1])
     return dict(U=U, step_bytes=step_bytes, step_flops=step_flops, kern=kern, rows=rr + rs)
 
 

@@ -62,7 +62,7 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 const char* kKernelNames[kKNumKinds] = {"router_logits", "router_gemm",  "topk_refine", "perm_count",
                                         "perm_scan",     "perm_scatter", "gather_rows", "gemm_gateup",
                                         "gemm_down",     "combine",      "quant_x",     "gemm_gateup_mx",
-                                        "gemm_down_mx",  "swiglu_reduce", "hash_route"};
+                                        "gemm_down_mx",  "swiglu_reduce", "hash_route",  "gemm_fused"};
 
 // 2-D tensor map, box of box_cols x box_rows elements, 128-byte swizzle unless stated.
 bool make_tmap(CUtensorMap* m, const void* ptr, CUtensorMapDataType dt, uint64_t rows, uint64_t cols,
@@ -137,6 +137,7 @@ struct moe_handle {
   int32_t* ntile_base_dn = nullptr;
   int* bad = nullptr;
   int* bad_flag = nullptr;      // device flag of the hash-table check
+  int* done = nullptr;          // per-group gate/up completion counters of the fused GEMM
   int64_t max_ntiles_r = 0;
   CUtensorMap tm_w13q, tm_w2q, tm_w2qw, tm_xq, tm_hq, tm_w13sh, tm_w2sh, tm_w2shw;
   // shared experts alone (MXFP4 layers, few tokens): split-K partial sums
@@ -380,6 +381,7 @@ moe_status create_impl(const moe_config* cfg, const moe_weights* w, int32_t e_be
   ok = ok && h->alloc(&h->o, h->R * H * 4, ws);
   ok = ok && h->alloc(&h->status, 16, ws);
   ok = ok && h->alloc(&h->bad_flag, 16, ws);
+  ok = ok && h->alloc(&h->done, (El + S) * 4, ws);
   ok = ok && h->alloc(&h->x_stage, Tm * H * 2, ws);
   ok = ok && h->alloc(&h->y_stage, Tm * H * 2, ws);
   if (!ok) {
@@ -626,6 +628,9 @@ moe_status forward_impl(moe_handle* h, const void* x, const int32_t* token_ids, 
   // with few tokens every tile streams the same weight bytes and its rows cost
   // next to nothing: the order of the partial tiles does not matter
   sa.sort_partial = small ? 0 : 1;
+  // few tokens, BF16: gate/up and down in one persistent launch
+  const bool fused = kFusedDecode && !kGatherX && !h->mx && wide_small;
+  sa.done = fused ? h->done : nullptr;
   sa.bn_alt = alt ? kBnAlt : 0;
   sa.bn_choice = alt ? h->bn_choice : nullptr;
   if (nchunks == 1) {
@@ -671,14 +676,16 @@ moe_status forward_impl(moe_handle* h, const void* x, const int32_t* token_ids, 
     a.limit = c.swiglu_limit;
     a.status = h->status;
     a.timeout_ns = h->timeout_ns;
-    h->prof_mark(kKGateUp, s);
-    if (alt) {
-      a.bn_select = h->bn_choice;
-      MOE_TRY_CUDA(launch_gemm_gateup_dual(h->tm_w13, tm_b, tm_x, a, h->num_sms, s));
-    } else {
-      MOE_TRY_CUDA(launch_gemm_gateup(h->tm_w13, tm_b, tm_x, a, bn_gu, h->num_sms, s));
+    if (!fused) {
+      h->prof_mark(kKGateUp, s);
+      if (alt) {
+        a.bn_select = h->bn_choice;
+        MOE_TRY_CUDA(launch_gemm_gateup_dual(h->tm_w13, tm_b, tm_x, a, h->num_sms, s));
+      } else {
+        MOE_TRY_CUDA(launch_gemm_gateup(h->tm_w13, tm_b, tm_x, a, bn_gu, h->num_sms, s));
+      }
+      h->prof_done(s);
     }
-    h->prof_done(s);
     // 5. down grouped GEMM
     GemmArgs d{};
     d.tiles = h->tiles_dn;
@@ -692,11 +699,22 @@ moe_status forward_impl(moe_handle* h, const void* x, const int32_t* token_ids, 
     d.m_limit = H;
     d.status = h->status;
     d.timeout_ns = h->timeout_ns;
-    h->prof_mark(kKDown, s);
-    if (alt) {
+    if (fused) {
+      // 4-5 together: the down tiles of a group start once its gate/up tiles are done
+      FusedArgs f{};
+      f.gu = a;
+      f.dn = d;
+      f.done = h->done;
+      f.cnt = h->cnt;
+      f.m_tiles_gu = h->m_tiles_gu;
+      h->prof_mark(kKGemmFused, s);
+      MOE_TRY_CUDA(launch_gemm_fused_small(h->tm_w13, tm_b, tm_x, h->tm_w2w, h->tm_h, f, h->num_sms, s));
+    } else if (alt) {
+      h->prof_mark(kKDown, s);
       d.bn_select = h->bn_choice;
       MOE_TRY_CUDA(launch_gemm_down_wide_dual(h->tm_w2w, h->tm_h, d, h->num_sms, s));
     } else {
+      h->prof_mark(kKDown, s);
       MOE_TRY_CUDA(launch_gemm_down(wide || wide_small ? h->tm_w2w : h->tm_w2, h->tm_h, d, bn_dn, h->num_sms, s,
                                     wide || wide_small));
     }

@@ -481,6 +481,267 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
   }
 }
 
+// Bounded wait until *p >= target (acquire); gives up when another role of the CTA
+// has aborted or the time runs out (then records MOE_ERR_TIMEOUT and aborts).
+__device__ __forceinline__ bool wait_count(const int* p, int target, const GemmArgs& a, volatile int* abort_flag) {
+  if (ld_acquire_gpu(p) >= target) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
+#pragma unroll 1
+    for (int i = 0; i < 32; ++i) {
+      if (ld_acquire_gpu(p) >= target) return true;
+      __nanosleep(100);
+    }
+    if (*abort_flag) return false;
+    if (globaltimer_ns() - t0 > a.timeout_ns) {
+      *abort_flag = 1;
+      report_status(a.status, kStatusTimeout);
+      return false;
+    }
+  }
+}
+
+// Gate/up and down of the few-token path in one persistent launch. Both halves
+// have the same geometry: two 128-row MMAs per K step sharing a BN-token tile (W1
+// and W3 rows of 128 expert-width rows; two 128-row halves of 256 W2 rows), so one
+// ring and one TMEM layout serve both. The combined tile index walks every gate/up
+// tile and then every down tile; a CTA takes every gridDim-th one, so it has
+// finished all its gate/up tiles before any down tile. A down tile of group g
+// waits until all of g's gate/up tiles have stored h: each epilogue warp of such a
+// tile adds 1 to done[g] after its stores, and g is ready at
+// m_tiles_gu * token tiles * kEpiWarps. All CTAs are resident (cooperative
+// launch), so every gate/up tile a down tile waits for is running or done.
+template <int BN, int kStages>
+__global__ void __launch_bounds__(kThreads, 1)
+    grouped_gemm_fused_kernel(const __grid_constant__ CUtensorMap tmA_gu, const __grid_constant__ CUtensorMap tmB_gu,
+                              const __grid_constant__ CUtensorMap tmBsh, const __grid_constant__ CUtensorMap tmA_dn,
+                              const __grid_constant__ CUtensorMap tmB_dn, const FusedArgs fa) {
+  using C = Cfg<true, 2, BN, kStages>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + kStages * C::kABytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sB + kStages * C::kBBytes);
+  uint64_t* full = bars;
+  uint64_t* empty = full + kStages;
+  uint64_t* tfull = empty + kStages;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_base_smem = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_base_smem + 1);
+  const GemmArgs& gu = fa.gu;
+  const GemmArgs& dn = fa.dn;
+
+  const int warp = threadIdx.x / 32;
+  const int lane = threadIdx.x % 32;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kStages; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&tfull[i], 1);
+      mbar_init(&tempty[i], kEpiWarps);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbarrier_init();
+  }
+  if (warp == kWarpTma && lane == 0) {
+    tma_prefetch_desc(&tmA_gu);
+    tma_prefetch_desc(&tmB_gu);
+    tma_prefetch_desc(&tmBsh);
+    tma_prefetch_desc(&tmA_dn);
+    tma_prefetch_desc(&tmB_dn);
+  }
+  if (warp == kWarpMma) {
+    tmem_alloc(tmem_base_smem, C::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_base_smem;
+
+  const int n_gu = *gu.ntiles;
+  const int n_all = n_gu + *dn.ntiles;
+  const int tfirst = static_cast<int>(blockIdx.x);
+  // the tile of combined index t: gate/up tiles first, then down tiles
+  auto tile_of = [&](int t, bool& is_dn) {
+    is_dn = t >= n_gu;
+    return load_tile<BN>(is_dn ? dn : gu, is_dn ? t - n_gu : t);
+  };
+
+  if (warp == kWarpTma) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      long issued = 0;
+      bool ok = true;
+      for (int t = tfirst; ok && t < n_all && !*abort_flag; t += gridDim.x) {
+        bool is_dn;
+        const Tile tl = tile_of(t, is_dn);
+        const GemmArgs& a = is_dn ? dn : gu;
+        const CUtensorMap* ma = is_dn ? &tmA_dn : &tmA_gu;
+        const CUtensorMap* mb = is_dn ? &tmB_dn : (tl.group >= gu.n_routed ? &tmBsh : &tmB_gu);
+        const int a_row = tl.group * a.a_rows_per_group + tl.m_tile * C::kARows;
+        if (is_dn) {
+          // the group's h rows: every gate/up tile of the group has stored them
+          const int g = tl.group;
+          const int target = fa.m_tiles_gu * ((fa.cnt[g] + BN - 1) / BN) * kEpiWarps;
+          if (!wait_count(fa.done + g, target, gu, abort_flag)) break;
+          fence_proxy_async_global();
+        }
+        const int nb = (tl.nrows + kBBoxRows - 1) / kBBoxRows;
+        const uint32_t bytes = C::kABytes + nb * kBBoxBytes;
+        for (int kb = 0; kb < tl.nkb; ++kb) {
+          if (!wait_or_abort(&empty[stage], phase ^ 1, gu, abort_flag)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&full[stage], bytes);
+          const int kx = kb * kBK;
+          tma_load_2d(sA + stage * C::kABytes, ma, &full[stage], kx, a_row, kCacheEvictFirst);
+          for (int j = 0; j < nb; ++j)
+            tma_load_2d(sB + stage * C::kBBytes + j * kBBoxBytes, mb, &full[stage], kx, tl.b_row0 + j * kBBoxRows,
+                        kCacheEvictLast);
+          ++issued;
+          if (++stage == kStages) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+      if (*abort_flag) drain_ring(full, kStages, issued, gu.timeout_ns);
+    }
+  } else if (warp == kWarpMma) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool ok = true;
+      for (int t = tfirst; ok && t < n_all && !*abort_flag; t += gridDim.x) {
+        bool is_dn;
+        const Tile tl = tile_of(t, is_dn);
+        const uint32_t n_mma = max(16, (tl.nrows + 15) & ~15);
+        const uint32_t idesc = idesc_bf16_f32(128, n_mma);
+        if (!wait_or_abort(&tempty[acc], acc_phase ^ 1, gu, abort_flag)) break;
+        tc_fence_after();
+        const uint32_t d = tmem_base + acc * C::kAccCols;
+        for (int kb = 0; kb < tl.nkb; ++kb) {
+          if (!wait_or_abort(&full[stage], phase, gu, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_addr = smem_u32(sA + stage * C::kABytes);
+          const uint32_t b_addr = smem_u32(sB + stage * C::kBBytes);
+#pragma unroll
+          for (int k = 0; k < kBK / 16; ++k) {
+            const uint64_t bdesc = sdesc_sw128(b_addr + k * 32);
+            const uint32_t accum = (kb | k) != 0;
+            umma_f16(d, sdesc_sw128(a_addr + k * 32), bdesc, idesc, accum);
+            umma_f16(d + BN, sdesc_sw128(a_addr + 128 * 128 + k * 32), bdesc, idesc, accum);
+          }
+          umma_commit(&empty[stage]);
+          if (++stage == kStages) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+        if (!ok) break;
+        umma_commit(&tfull[acc]);
+        if (++acc == C::kAccBufs) {
+          acc = 0;
+          acc_phase ^= 1;
+        }
+      }
+      umma_commit(drain);
+      const uint64_t t0 = globaltimer_ns();
+      while (!mbar_try_wait(drain, 0) && globaltimer_ns() - t0 < gu.timeout_ns) {
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue (warps 2..)
+    const int q = warp & 3;
+    const int cfirst = ((warp - 2) / 4) * 16;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int t = tfirst; t < n_all; t += gridDim.x) {
+      bool is_dn;
+      const Tile tl = tile_of(t, is_dn);
+      const GemmArgs& a = is_dn ? dn : gu;
+      const int n_mma = max(16, (tl.nrows + 15) & ~15);
+      bool ok = true;
+      if (lane == 0) ok = wait_or_abort(&tfull[acc], acc_phase, gu, abort_flag);
+      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+      if (!ok) break;
+      tc_fence_after();
+      const uint32_t tb = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * C::kAccCols;
+      const bool rows_ok = tl.out_row0 >= 0 && tl.out_row0 + tl.nrows <= a.out_rows;
+      if (!rows_ok && lane == 0 && q == 0) report_status(a.status, kStatusDevice);
+      for (int c0 = cfirst; c0 < n_mma; c0 += 16 * kEpiGroups) {
+        uint32_t g0[16], g1[16];
+        tmem_ld16(tb + c0, g0);
+        tmem_ld16(tb + BN + c0, g1);
+        tmem_ld_wait();
+        if (!is_dn) {
+          // h = silu(min(G, L)) * clamp(U, -L, L), BF16
+          const int m = tl.m_tile * 128 + q * 32 + lane;
+          const bool m_ok = m < a.m_limit && rows_ok;
+          __nv_bfloat16* out = static_cast<__nv_bfloat16*>(a.out);
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const int n = c0 + j;
+            if (n < tl.nrows && m_ok) {
+              const float hv = clamped_swiglu_f32(__uint_as_float(g0[j]), __uint_as_float(g1[j]), a.limit);
+              out[static_cast<size_t>(tl.out_row0 + n) * a.out_ld + m] = __float2bfloat16_rn(hv);
+            }
+          }
+        } else {
+          // fp32 O rows: columns m (first 128 W2 rows of the tile) and m + 128
+          const int m = tl.m_tile * 256 + q * 32 + lane;
+          float* out = static_cast<float*>(a.out);
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const int n = c0 + j;
+            if (n < tl.nrows && rows_ok) {
+              const size_t o = static_cast<size_t>(tl.out_row0 + n) * a.out_ld;
+              if (m < a.m_limit) out[o + m] = __uint_as_float(g0[j]);
+              if (m + 128 < a.m_limit) out[o + m + 128] = __uint_as_float(g1[j]);
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&tempty[acc]);
+        if (!is_dn) {
+          // this warp's h stores of the tile, visible GPU-wide (and to the TMA) before the count
+          __threadfence();
+          fence_proxy_async_global();
+          atomicAdd(fa.done + tl.group, 1);
+        }
+      }
+      if (++acc == C::kAccBufs) {
+        acc = 0;
+        acc_phase ^= 1;
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kWarpMma) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, C::kTmemCols);
+  }
+}
+
 template <bool kGateUp, int kAMmas, int BN, int kStages>
 __global__ void __launch_bounds__(kThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
@@ -580,8 +841,16 @@ constexpr int kBnAltT = kBnAlt > 0 ? kBnAlt : 64;  // an unused placeholder when
 
 }  // namespace
 
+// the fused few-token launch: 32-token tiles, the gate/up ring depth (both halves
+// have 256-row A boxes and 32-row B boxes)
+#define MOE_FUSED_SMALL 32, MOE_STAGES_GU_SMALL
+
 cudaError_t gemm_set_attributes() {
   cudaError_t e;
+  if ((e = cudaFuncSetAttribute(grouped_gemm_fused_kernel<MOE_FUSED_SMALL>,
+                                cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                Cfg<true, 2, MOE_FUSED_SMALL>::kSmemBytes)) != cudaSuccess)
+    return e;
   if ((e = set_attr<MOE_GU_SMALL>()) != cudaSuccess) return e;
   if ((e = set_attr<MOE_GU_MID>()) != cudaSuccess) return e;
   if ((e = set_attr<MOE_GU_LARGE>()) != cudaSuccess) return e;
@@ -630,6 +899,21 @@ cudaError_t launch_gemm_down_wide_dual(const CUtensorMap& tmA, const CUtensorMap
                                        cudaStream_t s) {
   if constexpr (kBnAlt > 0) return launch_dual<MOE_DN_WIDE_DUAL>(tmA, tmB, tmB, a, grid, s);
   return cudaErrorInvalidValue;
+}
+
+}  // namespace moe
+
+namespace moe {
+
+cudaError_t launch_gemm_fused_small(const CUtensorMap& tmA_gu, const CUtensorMap& tmB_gu, const CUtensorMap& tmBsh,
+                                   const CUtensorMap& tmA_dn, const CUtensorMap& tmB_dn, const FusedArgs& f,
+                                   int grid, cudaStream_t s) {
+  // cooperative: every CTA resident at once (a down tile waits for other CTAs' gate/up tiles)
+  void* args[] = {const_cast<CUtensorMap*>(&tmA_gu), const_cast<CUtensorMap*>(&tmB_gu),
+                  const_cast<CUtensorMap*>(&tmBsh),  const_cast<CUtensorMap*>(&tmA_dn),
+                  const_cast<CUtensorMap*>(&tmB_dn), const_cast<FusedArgs*>(&f)};
+  return cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(grouped_gemm_fused_kernel<MOE_FUSED_SMALL>),
+                                     dim3(grid), dim3(kThreads), args, Cfg<true, 2, MOE_FUSED_SMALL>::kSmemBytes, s);
 }
 
 }  // namespace moe

@@ -77,6 +77,7 @@ enum KernelKind {
   kKDownMx,
   kKSwigluReduce,
   kKHashRoute,
+  kKGemmFused,
   kKNumKinds
 };
 
@@ -132,6 +133,7 @@ struct ScanArgs {
   int bn_alt;                   // > 0: use this width for every tile when no routed group has more rows
   int* bn_choice;               // out: the width the tile lists were built with (bn_alt, or bn_gu_r)
   int sort_partial;             // order the partial token tiles longest first (tile costs differ)
+  int* done;                    // when not null: per-group counters of the fused GEMM, zeroed here
 };
 cudaError_t launch_perm_scan(const ScanArgs& a, cudaStream_t s);
 // count + scan + scatter in one launch when all slots fit one chunk
@@ -166,6 +168,23 @@ cudaError_t launch_gemm_gateup(const CUtensorMap& tmA, const CUtensorMap& tmB, c
 // the tile list's m tiles are then H / 256.
 cudaError_t launch_gemm_down(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmArgs& a, int bn, int grid,
                              cudaStream_t s, bool wide = false);
+// Gate/up and down of the few-token path (32-token tiles, 256 W2 rows per down
+// tile) in one persistent launch: the CTAs walk the gate/up tiles and then the down
+// tiles; a down tile of group g starts once every gate/up tile of g has stored its
+// h rows (done[g] counts the epilogue warps that finished one). Cooperative launch.
+struct FusedArgs {
+  GemmArgs gu, dn;
+  int* done;                    // per group, zeroed by the permutation kernel
+  const int32_t* cnt;           // rows per group
+  int m_tiles_gu;               // weight tiles per group of the gate/up GEMM
+};
+#ifndef MOE_FUSED_DECODE
+#define MOE_FUSED_DECODE 1
+#endif
+constexpr bool kFusedDecode = MOE_FUSED_DECODE != 0;
+cudaError_t launch_gemm_fused_small(const CUtensorMap& tmA_gu, const CUtensorMap& tmB_gu, const CUtensorMap& tmBsh,
+                                   const CUtensorMap& tmA_dn, const CUtensorMap& tmB_dn, const FusedArgs& f,
+                                   int grid, cudaStream_t s);
 // One launch for both many-token widths (kBnLarge and kBnAlt): a.bn_select holds
 // the permutation kernel's choice; wide W2 tiles for the down GEMM.
 cudaError_t launch_gemm_gateup_dual(const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap& tmBsh,

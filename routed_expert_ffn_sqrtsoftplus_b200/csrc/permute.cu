@@ -211,6 +211,7 @@ __global__ void __launch_bounds__(1024) perm_scan_kernel(ScanArgs a, int fused, 
   for (int g = tid; g <= G; g += blockDim.x) {
     a.off[g] = off_s[g];
     if (g < G) a.cnt[g] = cnt_s[g];
+    if (g < G && a.done != nullptr) a.done[g] = 0;
   }
   if (a.ntile_base_gu != nullptr)
     for (int g = tid; g <= a.E; g += blockDim.x) {
