@@ -376,7 +376,7 @@ moe_status create_impl(const moe_config* cfg, const moe_weights* w, int32_t e_be
   ok = ok && h->alloc(&h->bn_choice, 16, ws);
   ok = ok && h->alloc(&h->tiles_gu, h->max_tiles_gu * 16, ws);
   ok = ok && h->alloc(&h->tiles_dn, h->max_tiles_dn * 16, ws);
-  ok = ok && h->alloc(&h->ntiles, 16, ws);
+  ok = ok && h->alloc(&h->ntiles, 32, ws);   // 4 tile counts + the routed row count
   ok = ok && h->alloc(&h->h, h->R * I * 2, ws);
   ok = ok && h->alloc(&h->o, h->R * H * 4, ws);
   ok = ok && h->alloc(&h->status, 16, ws);
@@ -631,6 +631,7 @@ moe_status forward_impl(moe_handle* h, const void* x, const int32_t* token_ids, 
   // few tokens, BF16: gate/up and down in one persistent launch
   const bool fused = kFusedDecode && !kGatherX && !h->mx && wide_small;
   sa.done = fused ? h->done : nullptr;
+  sa.nrows_routed = h->ntiles + 4;
   sa.bn_alt = alt ? kBnAlt : 0;
   sa.bn_choice = alt ? h->bn_choice : nullptr;
   if (nchunks == 1) {
@@ -655,7 +656,7 @@ moe_status forward_impl(moe_handle* h, const void* x, const int32_t* token_ids, 
       if (!make_tmap_bf16(&tm_xg, x, static_cast<uint64_t>(T), static_cast<uint64_t>(H), 1)) return MOE_ERR_CUDA;
     } else {
       h->prof_mark(kKGather, s);
-      MOE_TRY_CUDA(launch_gather_rows(x, h->perm, nslots, k, H, h->xp, s));
+      MOE_TRY_CUDA(launch_gather_rows(x, h->perm, nslots, h->ntiles + 4, k, H, h->xp, s));
       h->prof_done(s);
     }
     const CUtensorMap& tm_b = kGatherX ? tm_xg : h->tm_xp;
@@ -722,8 +723,8 @@ moe_status forward_impl(moe_handle* h, const void* x, const int32_t* token_ids, 
   } else {
     // MXFP8 token rows of the routed slots
     h->prof_mark(kKQuantX, s);
-    MOE_TRY_CUDA(launch_quant_gather_mx(x, h->perm, h->idx, h->off, h->ntile_base_gu, nslots, k, H, bn_mx, eb,
-                                        h->xq, h->sfb_gu, s));
+    MOE_TRY_CUDA(launch_quant_gather_mx(x, h->perm, h->idx, h->off, h->ntile_base_gu, nslots, h->ntiles + 4, k, H,
+                                        bn_mx, eb, El, h->xq, h->sfb_gu, s));
     h->prof_done(s);
     // 4a. routed gate/up on block-scaled MMAs (tiles after the shared ones)
     MxGemmArgs g{};
@@ -1037,7 +1038,7 @@ moe_status moe_inspect(moe_handle* h, int32_t what, void* dst, size_t bytes, moe
       src = h->sfb_dn;
       cap = h->max_ntiles_r * (I / 128) * 512;
       break;
-    case MOE_BUF_NTILES: src = h->ntiles; cap = 16; break;
+    case MOE_BUF_NTILES: src = h->ntiles; cap = 20; break;
     case MOE_BUF_TILES_GU: src = h->tiles_gu; cap = h->max_tiles_gu * 16; break;
     case MOE_BUF_TILES_DN: src = h->tiles_dn; cap = h->max_tiles_dn * 16; break;
     default: return MOE_ERR_INVALID_ARG;

@@ -134,6 +134,7 @@ struct ScanArgs {
   int* bn_choice;               // out: the width the tile lists were built with (bn_alt, or bn_gu_r)
   int sort_partial;             // order the partial token tiles longest first (tile costs differ)
   int* done;                    // when not null: per-group counters of the fused GEMM, zeroed here
+  int32_t* nrows_routed;        // out: rows of the routed groups (T*k, or fewer in an expert window)
 };
 cudaError_t launch_perm_scan(const ScanArgs& a, cudaStream_t s);
 // count + scan + scatter in one launch when all slots fit one chunk
@@ -141,8 +142,9 @@ cudaError_t launch_perm_fused(const ScanArgs& a, const int32_t* idx, int nslots,
                               int* status, cudaStream_t s);
 cudaError_t launch_perm_scatter(const int32_t* idx, int nslots, int E, int e_begin, const int32_t* chunk_base,
                                 int32_t* perm, int32_t* inv, cudaStream_t s);
-cudaError_t launch_gather_rows(const void* x, const int32_t* perm, int nrows, int k, int H, void* xp,
-                               cudaStream_t s);
+// rows >= min(nrows, *nrows_dev) are not routed to this instance and are skipped
+cudaError_t launch_gather_rows(const void* x, const int32_t* perm, int nrows, const int32_t* nrows_dev, int k, int H,
+                               void* xp, cudaStream_t s);
 
 // ---- grouped GEMMs (tcgen05)
 // Token-tile width of the many-tokens-per-expert GEMMs (gate/up, down and the
@@ -244,8 +246,8 @@ cudaError_t launch_gemm_mx_down(const CUtensorMap& tmA, const CUtensorMap& tmB, 
 // x rows of the routed slots -> MXFP8: xq[row] = E4M3 codes of x[perm[row] / k], scale
 // atoms by gate/up token tile.
 cudaError_t launch_quant_gather_mx(const void* x, const int32_t* perm, const int32_t* idx, const int32_t* off,
-                                   const int32_t* ntile_base_gu, int nrows, int k, int H, int bn_gu, int e_begin,
-                                   uint8_t* xq, uint8_t* sfb, cudaStream_t s);
+                                   const int32_t* ntile_base_gu, int nrows, const int32_t* nrows_dev, int k, int H,
+                                   int bn_gu, int e_begin, int e_count, uint8_t* xq, uint8_t* sfb, cudaStream_t s);
 // Weight scales [groups, rows, K/32] -> atoms [groups][rows/128][K/128][parts * 512]; for
 // gate/up the two parts are W1 and W3 of the same 128 rows. Codes 0xFF raise *bad.
 cudaError_t launch_sf_atoms(const uint8_t* s_a, const uint8_t* s_b, int groups, int rows, int K, uint8_t* dst,

@@ -145,6 +145,7 @@ __global__ void __launch_bounds__(1024) perm_scan_kernel(ScanArgs a, int fused, 
     int o = block_exclusive_scan(n, warp_tot, &tot);
     if (g < a.E) off_s[g] = o;
     else if (g <= G) off_s[g] = a.T * a.k + (g - a.E) * a.T;
+    if (tid == 0 && a.nrows_routed != nullptr) *a.nrows_routed = tot;
     // token-tile bases of the routed groups, in group order (MX scale atoms)
     const bool routed = g < a.E;
     int ng = block_exclusive_scan(routed ? (n + bn_gu_r - 1) / bn_gu_r : 0, warp_tot, &tot);
@@ -322,10 +323,10 @@ __global__ void __launch_bounds__(32)
 
 // Xp[row] = x[perm[row] / k]: one warp per row, 16-byte vectors.
 __global__ void __launch_bounds__(256)
-    gather_rows_kernel(const uint4* __restrict__ x, const int32_t* __restrict__ perm, int nrows, int k, int hv,
-                       uint4* __restrict__ xp) {
+    gather_rows_kernel(const uint4* __restrict__ x, const int32_t* __restrict__ perm, int nrows,
+                       const int32_t* __restrict__ nrows_dev, int k, int hv, uint4* __restrict__ xp) {
   const int row = blockIdx.x * 8 + threadIdx.x / 32;
-  if (row >= nrows) return;
+  if (row >= nrows || row >= *nrows_dev) return;
   const int t = perm[row] / k;
   const uint4* src = x + static_cast<size_t>(t) * hv;
   uint4* dst = xp + static_cast<size_t>(row) * hv;
@@ -339,14 +340,16 @@ __global__ void __launch_bounds__(256)
 __global__ void __launch_bounds__(256)
     quant_gather_mx_kernel(const uint4* __restrict__ x, const int32_t* __restrict__ perm,
                            const int32_t* __restrict__ idx, const int32_t* __restrict__ off,
-                           const int32_t* __restrict__ ntile_base, int nrows, int k, int H, int bn, int e_begin,
-                           uint4* __restrict__ xq, uint8_t* __restrict__ sfb) {
+                           const int32_t* __restrict__ ntile_base, int nrows, const int32_t* __restrict__ nrows_dev,
+                           int k, int H, int bn, int e_begin, int e_count, uint4* __restrict__ xq,
+                           uint8_t* __restrict__ sfb) {
   const int row = blockIdx.x * 8 + threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
-  if (row >= nrows) return;
+  if (row >= nrows || row >= *nrows_dev) return;
   const int slot = perm[row];
   const int t = slot / k;
   const int g = idx[slot] - e_begin;
+  if (g < 0 || g >= e_count) return;  // never for a routed row of this instance
   const int j = row - off[g];
   const int ntile = ntile_base[g] + j / bn;
   const int n = j % bn;
@@ -391,12 +394,12 @@ __global__ void __launch_bounds__(256)
 }  // namespace
 
 cudaError_t launch_quant_gather_mx(const void* x, const int32_t* perm, const int32_t* idx, const int32_t* off,
-                                   const int32_t* ntile_base_gu, int nrows, int k, int H, int bn_gu, int e_begin,
-                                   uint8_t* xq, uint8_t* sfb, cudaStream_t s) {
+                                   const int32_t* ntile_base_gu, int nrows, const int32_t* nrows_dev, int k, int H,
+                                   int bn_gu, int e_begin, int e_count, uint8_t* xq, uint8_t* sfb, cudaStream_t s) {
   if (nrows == 0) return cudaSuccess;
   quant_gather_mx_kernel<<<(nrows + 7) / 8, 256, 0, s>>>(static_cast<const uint4*>(x), perm, idx, off,
-                                                          ntile_base_gu, nrows, k, H, bn_gu, e_begin,
-                                                          reinterpret_cast<uint4*>(xq), sfb);
+                                                          ntile_base_gu, nrows, nrows_dev, k, H, bn_gu, e_begin,
+                                                          e_count, reinterpret_cast<uint4*>(xq), sfb);
   return cudaGetLastError();
 }
 
@@ -428,10 +431,10 @@ cudaError_t launch_perm_scatter(const int32_t* idx, int nslots, int E, int e_beg
   return cudaGetLastError();
 }
 
-cudaError_t launch_gather_rows(const void* x, const int32_t* perm, int nrows, int k, int H, void* xp,
-                               cudaStream_t s) {
+cudaError_t launch_gather_rows(const void* x, const int32_t* perm, int nrows, const int32_t* nrows_dev, int k, int H,
+                               void* xp, cudaStream_t s) {
   if (nrows == 0) return cudaSuccess;
-  gather_rows_kernel<<<(nrows + 7) / 8, 256, 0, s>>>(static_cast<const uint4*>(x), perm, nrows, k, H / 8,
+  gather_rows_kernel<<<(nrows + 7) / 8, 256, 0, s>>>(static_cast<const uint4*>(x), perm, nrows, nrows_dev, k, H / 8,
                                                      static_cast<uint4*>(xp));
   return cudaGetLastError();
 }
