@@ -15,7 +15,7 @@ DeepSeek-V4-Pro config paragraph; distributions as stated per workload):
   flash_mxfp4_prefill T=4096, same
   flash_mxfp8_decode  T=32,   same layer, routed experts to be stored as MXFP8
                       (E4M3 + E8M0 per 32)
-  flash_mxfp8_prefill T=8192, same
+  flash_mxfp8_prefill T=4096, same (the MXFP4 prefill batch)
   pro_skewed          T=2048, H=7168, I=3072, 384 + 1, top-6, with a Zipf
                       per-expert logit bias b_e = 2 ln(1/rank_e) over a seeded
                       random expert permutation (a few experts get most tokens)
@@ -67,7 +67,7 @@ WORKLOADS = {
                                     expert_dtype="mxfp4", seed=1003),
     "flash_mxfp8_decode": Workload("flash_mxfp8_decode", T=32, H=5120, I=2304, E=384,
                                    expert_dtype="mxfp8", seed=1006),
-    "flash_mxfp8_prefill": Workload("flash_mxfp8_prefill", T=8192, H=5120, I=2304, E=384,
+    "flash_mxfp8_prefill": Workload("flash_mxfp8_prefill", T=4096, H=5120, I=2304, E=384,
                                     expert_dtype="mxfp8", seed=1006),
     "pro_skewed": Workload("pro_skewed", T=2048, H=7168, I=3072, E=384, zipf_bias=True, seed=1004),
     "dspark": Workload("dspark", T=256, H=5120, I=2304, E=128, k=3, seed=1005),
