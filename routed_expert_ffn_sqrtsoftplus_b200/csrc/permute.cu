@@ -91,6 +91,7 @@ __global__ void __launch_bounds__(1024) perm_scan_kernel(ScanArgs a, int fused, 
   __shared__ int part_g[2][kMaxScanGroups];      // routed group of each partial-tile segment
   __shared__ int rem_s[kMaxScanGroups];          // rows of each routed group's partial token tile
   __shared__ int nseg_s[2];
+  __shared__ int slot_e[kPermChunk];             // fused: each slot's group (-1: not this instance's)
   __shared__ int warp_tot[32];
   __shared__ int tot;
   __shared__ int maxc_s;
@@ -103,10 +104,10 @@ __global__ void __launch_bounds__(1024) perm_scan_kernel(ScanArgs a, int fused, 
     for (int s = tid; s < nslots; s += blockDim.x) {
       const int g = idx[s];
       const int e = g - a.e_begin;
-      if (g < 0 || g >= a.e_global)
-        report_status(status, kStatusDevice);
-      else if (e >= 0 && e < a.E)
-        atomicAdd(&cnt_s[e], 1);
+      const bool mine = g >= 0 && g < a.e_global && e >= 0 && e < a.E;
+      if (g < 0 || g >= a.e_global) report_status(status, kStatusDevice);
+      if (mine) atomicAdd(&cnt_s[e], 1);
+      slot_e[s] = mine ? e : -1;  // kept for the scatter below (no second pass over global memory)
     }
     __syncthreads();
     for (int g = a.E + tid; g < G; g += blockDim.x) cnt_s[g] = a.T;
@@ -275,8 +276,8 @@ __global__ void __launch_bounds__(1024) perm_scan_kernel(ScanArgs a, int fused, 
     __syncwarp();
     for (int b = 0; b < nslots; b += 32) {
       const int s = b + lane;
-      const int e = s < nslots ? idx[s] - a.e_begin : -1;
-      const bool valid = e >= 0 && e < a.E;
+      const int e = s < nslots ? slot_e[s] : -1;
+      const bool valid = e >= 0;
       const unsigned peers = __match_any_sync(0xffffffffu, valid ? e : -1);
       const int rank = __popc(peers & ((1u << lane) - 1u));
       if (valid) {
