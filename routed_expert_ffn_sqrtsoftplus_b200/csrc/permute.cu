@@ -25,6 +25,13 @@ constexpr int kMaxSegs = 2 * kMaxScanGroups;  // tile-list segments (shared, ful
 #define MOE_TILE_ORDER_LPT 1
 #endif
 constexpr bool kTileOrderLongestFirst = MOE_TILE_ORDER_LPT != 0;
+// Full and partial routed token tiles spread evenly over the list (1), so that the
+// compute-heavy full tiles of hot experts run beside the weight-streaming partial
+// tiles of cold ones, or full tiles first (0).
+#ifndef MOE_TILE_ORDER_MIX
+#define MOE_TILE_ORDER_MIX 0
+#endif
+constexpr bool kTileOrderMix = MOE_TILE_ORDER_MIX != 0;
 
 // Expert windows (expert parallelism): this layer instance holds routed experts
 // [e_begin, e_begin + E) of e_global; a slot whose expert lies outside the window
@@ -232,13 +239,24 @@ __global__ void __launch_bounds__(1024) perm_scan_kernel(ScanArgs a, int fused, 
     const int bnr = list == 0 ? bn_gu_r : bn_dn_r, bns = list == 0 ? bn_gu_s : bn_dn_s;
     int4* out = list == 0 ? a.tiles_gu : a.tiles_dn;
     const int total = pre[ns];
+    // mixed order: routed position r takes full tile floor(r NF / N) when that count
+    // steps up at r, else the next partial tile (each of the N = NF + NP once)
+    const int sh_end = pre[a.S], full_end = pre[a.S + a.E];
+    const long long NF = full_end - sh_end, NR = total - sh_end;
+    const bool mix = kTileOrderMix && a.sort_partial && NF > 0 && NR > NF;
     for (int t = tid; t < total; t += blockDim.x) {
-      int lo = 0, hi = ns - 1;
-      while (lo < hi) {  // last segment with pre <= t
-        const int mid = (lo + hi + 1) >> 1;
-        if (pre[mid] <= t) lo = mid; else hi = mid - 1;
+      int pos = t;
+      if (mix && t >= sh_end) {
+        const long long r = t - sh_end;
+        const long long f0 = r * NF / NR, f1 = (r + 1) * NF / NR;
+        pos = f1 > f0 ? sh_end + static_cast<int>(f0) : full_end + static_cast<int>(r - f0);
       }
-      const int local = t - pre[lo];
+      int lo = 0, hi = ns - 1;
+      while (lo < hi) {  // last segment with pre <= pos
+        const int mid = (lo + hi + 1) >> 1;
+        if (pre[mid] <= pos) lo = mid; else hi = mid - 1;
+      }
+      const int local = pos - pre[lo];
       int g, mt, nt;
       if (lo < a.S) {
         g = a.E + lo;

@@ -283,15 +283,20 @@ def test_nan_token_is_contained_warp_topk(cuda_device):
 
 def _check_tile_list(tiles, n_shared_end, cnt, off, E, gateup, longest_first):
     """Every group's rows covered once per weight tile; shared tiles first; with
-    many tokens per expert the routed tiles by row count, non-increasing (full
-    tiles, then partial ones by size), else in group order."""
+    many tokens per expert the partial (last) token tiles of the routed groups by
+    row count, non-increasing (the full tiles come before them or spread among
+    them, by the build's order), else the routed tiles in group order."""
     g = tiles[:, 0] & 0xFFFF
     mt = tiles[:, 0] >> 16
     y, z, rows = tiles[:, 1], tiles[:, 2], tiles[:, 3]
     assert np.all(g[:n_shared_end] >= E) and np.all(g[n_shared_end:] < E)
     r = rows[n_shared_end:]
     if longest_first:
-        assert np.all(r[:-1] >= r[1:]), "routed tiles are not longest first"
+        gr = g[n_shared_end:]
+        last = (z[n_shared_end:] - off[gr] + r) == cnt[gr]     # the group's last token tile
+        full = r == r.max()
+        part = r[last & ~full]
+        assert np.all(part[:-1] >= part[1:]), "partial tiles are not longest first"
     else:
         gr = g[n_shared_end:]
         full = r == r.max()
