@@ -57,19 +57,6 @@ constexpr int kPrefetch = MOE_MX_PREFETCH;
 #define MOE_MX_TILE_PREFETCH 0
 #endif
 constexpr int kTilePrefetchQuarters = MOE_MX_TILE_PREFETCH;
-// The 32 lanes of the producer warp prefetch the weight rows of the K step this
-// many ring stages ahead of the TMA loads into L2 with plain prefetch instructions
-// (0 = none): more HBM bytes in flight per SM than the ring holds, without the
-// TMA unit. kLsuPrefetchStep: bytes between two prefetches along a row.
-#ifndef MOE_MX_LSU_PREFETCH
-#define MOE_MX_LSU_PREFETCH 0
-#endif
-#ifndef MOE_MX_LSU_STEP
-#define MOE_MX_LSU_STEP 128
-#endif
-constexpr int kLsuPrefetch = MOE_MX_LSU_PREFETCH;
-constexpr int kLsuStep = MOE_MX_LSU_STEP;
-static_assert(kLsuStep == 32 || kLsuStep == 64 || kLsuStep == 128, "prefetch step");
 
 constexpr int pow2_at_least(int v, int lo) {
   int p = lo;
@@ -197,88 +184,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int tend = *args.ntiles;
   const int tfirst = (args.tile_begin ? *args.tile_begin : 0) + static_cast<int>(blockIdx.x);
 
-  if (warp == 0 && kLsuPrefetch > 0) {
-    // ------------------------------------------------------------ TMA producer, warp-wide:
-    // lane 0 waits and issues the copies, all lanes prefetch rows kLsuPrefetch stages ahead
-    int stage = 0;
-    uint32_t phase = 0;
-    long issued = 0;
-    const int rb = C::kATx / C::kARows;                  // HBM bytes of one row per K step
-    int pf_t = tfirst, pf_kb = 0;
-    const uint8_t* pf_src = nullptr;
-    auto lsu_prefetch = [&]() {
-      if (pf_t >= tend || args.a_base == nullptr) return;
-      if (pf_kb == 0) {
-        const Tile pt = load_tile<BN>(args, pf_t);
-        pf_src = args.a_base + (static_cast<size_t>(pt.group) * args.a_rows_per_group +
-                                static_cast<size_t>(pt.m_tile) * C::kARows) * args.a_row_bytes;
-      }
-      const int b0 = pf_kb * rb;                         // this K step's bytes [b0, b0 + rb) of each row
-#pragma unroll 1
-      for (int b = (b0 + kLsuStep - 1) / kLsuStep * kLsuStep; b < b0 + rb; b += kLsuStep)
-#pragma unroll 4
-        for (int r = lane; r < C::kARows; r += 32) prefetch_l2_line(pf_src + static_cast<size_t>(r) * args.a_row_bytes + b);
-      if (++pf_kb == args.num_kb) {
-        pf_kb = 0;
-        pf_t += gridDim.x;
-      }
-    };
-    for (int i = 0; i < kLsuPrefetch; ++i) lsu_prefetch();
-    bool ok = true;
-    for (int t = tfirst; ok && t < tend; t += gridDim.x) {
-      if (__shfl_sync(0xffffffffu, lane == 0 ? *abort_flag : 0, 0)) break;
-      const Tile tl = load_tile<BN>(args, t);
-      const int a_row = tl.group * args.a_rows_per_group + tl.m_tile * C::kARows;
-      const int nb = (tl.nrows + kBBoxRows - 1) / kBBoxRows;
-      const uint32_t bytes = C::kATx + nb * kBBoxBytes + C::kSfBytes;
-      const uint8_t* sfa_src =
-          kWide ? args.sfa + (static_cast<size_t>(tl.group) * args.m_tiles + 2 * tl.m_tile) * args.num_kb * kAtomBytes
-                : args.sfa + (static_cast<size_t>(tl.group) * args.m_tiles + tl.m_tile) * args.num_kb * C::kSfaBytes;
-      const uint8_t* sfb_src = args.sfb + static_cast<size_t>(tl.ntile) * args.num_kb * kAtomBytes;
-      for (int kb = 0; kb < args.num_kb; ++kb) {
-        bool w = true;
-        if (lane == 0) w = wait_or_abort(&empty[stage], phase ^ 1, args, abort_flag);
-        if (!__shfl_sync(0xffffffffu, w ? 1 : 0, 0)) {
-          ok = false;
-          break;
-        }
-        if (lane == 0) {
-          mbar_arrive_expect_tx(&full[stage], bytes);
-          tma_load_2d(sA + stage * C::kStageABytes, &tmA, &full[stage], C::kPack ? kb * (kBK / 2) : kb * kBK, a_row,
-                      kCacheEvictFirst);
-          for (int j = 0; j < nb; ++j)
-            tma_load_2d(sB + stage * C::kBBytes + j * kBBoxBytes, &tmB, &full[stage], kb * kBK,
-                        tl.row0 + j * kBBoxRows, kCacheEvictLast);
-          uint8_t* sf = sSF + stage * C::kSfBytes;
-          if (kWide) {
-            bulk_load(sf, sfa_src + static_cast<size_t>(kb) * kAtomBytes, kAtomBytes, &full[stage], kCacheEvictFirst);
-            bulk_load(sf + kAtomBytes, sfa_src + static_cast<size_t>(args.num_kb + kb) * kAtomBytes, kAtomBytes,
-                      &full[stage], kCacheEvictFirst);
-          } else {
-            bulk_load(sf, sfa_src + static_cast<size_t>(kb) * C::kSfaBytes, C::kSfaBytes, &full[stage],
-                      kCacheEvictFirst);
-          }
-          bulk_load(sf + C::kSfaBytes, sfb_src + static_cast<size_t>(kb) * kAtomBytes, kAtomBytes, &full[stage],
-                    kCacheEvictLast);
-        }
-        lsu_prefetch();
-        ++issued;
-        if (++stage == kStages) {
-          stage = 0;
-          phase ^= 1;
-        }
-      }
-    }
-    if (lane == 0 && *abort_flag) {
-      for (long i = issued - 1; i >= 0 && i >= issued - kStages; --i) {
-        const int s = static_cast<int>(i % kStages);
-        const uint32_t par = static_cast<uint32_t>((i / kStages) & 1);
-        const uint64_t t0 = globaltimer_ns();
-        while (!mbar_try_wait(&full[s], par) && globaltimer_ns() - t0 < args.timeout_ns) {
-        }
-      }
-    }
-  } else if (warp == 0) {
+  if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       int stage = 0;

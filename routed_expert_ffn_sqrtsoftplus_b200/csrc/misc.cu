@@ -13,15 +13,31 @@ namespace {
 // this instance's window [e_begin, e_begin + e_count) count (all of them for a
 // whole layer); with y_f32 the sum is written in fp32 (an expert-parallel
 // partial output, summed over the instances afterwards).
+constexpr int kCombineMaxK = 32;   // top_k <= 32
+constexpr int kCombineBatch = 8;   // O rows loaded before their products are summed
+
 __global__ void __launch_bounds__(128)
     combine_kernel(const float4* __restrict__ O, const int32_t* __restrict__ inv, const int32_t* __restrict__ idx,
                    int e_begin, int e_count, const float* __restrict__ w, int T, int H4, int k, int S,
                    void* __restrict__ y, int y_f32, const float4* __restrict__ sh_parts, int n_parts) {
+  // the token's slots, read once per block: O row (-1: another instance's expert, or
+  // a row index outside O, which only corrupted memory could give) and weight
+  __shared__ int row_s[kCombineMaxK];
+  __shared__ float w_s[kCombineMaxK];
   const int t = blockIdx.x;
+  const size_t routed_rows = static_cast<size_t>(T) * k;
+  if (static_cast<int>(threadIdx.x) < k) {
+    const size_t i = static_cast<size_t>(t) * k + threadIdx.x;
+    const int e = __ldg(idx + i) - e_begin;
+    const int row = __ldg(inv + i);
+    const bool use = e >= 0 && e < e_count && row >= 0 && static_cast<size_t>(row) < routed_rows;
+    row_s[threadIdx.x] = use ? row : -1;
+    w_s[threadIdx.x] = __ldg(w + i);
+  }
+  __syncthreads();
   const int c = blockIdx.y * blockDim.x + threadIdx.x;
   if (c >= H4) return;
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  const size_t routed_rows = static_cast<size_t>(T) * k;
   for (int j = 0; j < S; ++j) {
     if (sh_parts == nullptr) {
       const float4 v = __ldg(O + (routed_rows + static_cast<size_t>(j) * T + t) * H4 + c);
@@ -45,19 +61,24 @@ __global__ void __launch_bounds__(128)
       acc.w += sj.w;
     }
   }
-  for (int j = 0; j < k; ++j) {
-    const int e = __ldg(idx + static_cast<size_t>(t) * k + j) - e_begin;
-    if (e < 0 || e >= e_count) continue;  // another instance's expert
-    const int row = __ldg(inv + static_cast<size_t>(t) * k + j);
-    // every slot's row is below T*k; the check keeps a corrupted row index from
-    // reading outside O
-    if (row < 0 || static_cast<size_t>(row) >= routed_rows) continue;
-    const float wj = __ldg(w + static_cast<size_t>(t) * k + j);
-    const float4 v = __ldg(O + static_cast<size_t>(row) * H4 + c);
-    acc.x = fmaf(wj, v.x, acc.x);
-    acc.y = fmaf(wj, v.y, acc.y);
-    acc.z = fmaf(wj, v.z, acc.z);
-    acc.w = fmaf(wj, v.w, acc.w);
+  // routed slots in slot order; a batch of rows is in flight at once
+  for (int j0 = 0; j0 < k; j0 += kCombineBatch) {
+    float4 v[kCombineBatch];
+#pragma unroll
+    for (int u = 0; u < kCombineBatch; ++u) {
+      const int row = j0 + u < k ? row_s[j0 + u] : -1;
+      v[u] = row >= 0 ? __ldg(O + static_cast<size_t>(row) * H4 + c) : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int u = 0; u < kCombineBatch; ++u) {
+      if (j0 + u < k && row_s[j0 + u] >= 0) {
+        const float wj = w_s[j0 + u];
+        acc.x = fmaf(wj, v[u].x, acc.x);
+        acc.y = fmaf(wj, v[u].y, acc.y);
+        acc.z = fmaf(wj, v[u].z, acc.z);
+        acc.w = fmaf(wj, v[u].w, acc.w);
+      }
+    }
   }
   if (y_f32) {
     static_cast<float4*>(y)[static_cast<size_t>(t) * H4 + c] = acc;
@@ -282,6 +303,7 @@ cudaError_t launch_combine(const float* O, const int32_t* inv, const int32_t* id
                            const float* w, int T, int H, int k, int S, void* y, bool y_f32, const float* sh_parts,
                            int n_parts, cudaStream_t s) {
   if (T == 0) return cudaSuccess;
+  if (k > kCombineMaxK) return cudaErrorInvalidValue;
   const int H4 = H / 4;
   const dim3 grid(T, (H4 + 127) / 128);
   combine_kernel<<<grid, 128, 0, s>>>(reinterpret_cast<const float4*>(O), inv, idx, e_begin, e_count, w, T, H4, k,

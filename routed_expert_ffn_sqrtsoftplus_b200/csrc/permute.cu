@@ -349,7 +349,15 @@ __global__ void __launch_bounds__(256)
   const int t = perm[row] / k;
   const uint4* src = x + static_cast<size_t>(t) * hv;
   uint4* dst = xp + static_cast<size_t>(row) * hv;
-  for (int c = threadIdx.x % 32; c < hv; c += 32) dst[c] = __ldg(src + c);
+  int c = threadIdx.x % 32;
+  for (; c + 96 < hv; c += 128) {  // four 16-byte loads in flight per lane
+    const uint4 a = __ldg(src + c), b = __ldg(src + c + 32), d = __ldg(src + c + 64), e = __ldg(src + c + 96);
+    dst[c] = a;
+    dst[c + 32] = b;
+    dst[c + 64] = d;
+    dst[c + 96] = e;
+  }
+  for (; c < hv; c += 32) dst[c] = __ldg(src + c);
 }
 
 // MXFP8 quantisation of the routed token rows (OCP MX v1.0 rule, E4M3 with
