@@ -278,8 +278,10 @@ typedef enum {
                             Token tiles: each routed group's rows cut into tiles of 32 rows when
                             T <= 32, 96 rows when T * top_k >= 24 * n_routed, else 64 rows,
                             numbered group by group in expert order */
-  MOE_BUF_NTILES = 12,   /* int32 [5]: tiles in the gate/up and down lists, where their shared-expert
-                            tiles end, and the routed rows this instance holds */
+  MOE_BUF_NTILES = 12,   /* int32 [7]: tiles in the gate/up and down lists, where their shared-expert
+                            tiles end, the routed rows this instance holds, and where each list's
+                            thin tail begins (partial tiles of at most 32 rows, last in a list
+                            ordered longest first; the list's length when it is not ordered so) */
   MOE_BUF_TILES_GU = 13, /* int32 [n, 4] gate/up tile list: {group | m_tile << 16, B row or token-tile id,
                             first output row, rows} in the order the persistent CTAs take them */
   MOE_BUF_TILES_DN = 14  /* int32 [n, 4] the same for the down GEMM */

@@ -134,6 +134,7 @@ struct moe_handle {
   uint8_t* sfb_dn = nullptr;    // h scale atoms, down token tiles
   int32_t* ntile_base_gu = nullptr;
   int* bn_choice = nullptr;     // token-tile width the permutation chose (many-token BF16 path)
+  int* sched = nullptr;         // tile counters of the dual-width GEMMs (gate/up wide, thin; down wide, thin)
   int32_t* ntile_base_dn = nullptr;
   int* bad = nullptr;
   int* bad_flag = nullptr;      // device flag of the hash-table check
@@ -374,9 +375,10 @@ moe_status create_impl(const moe_config* cfg, const moe_weights* w, int32_t e_be
   ok = ok && h->alloc(&h->perm, Tm * k * 4, ws);
   ok = ok && h->alloc(&h->inv, Tm * k * 4, ws);
   ok = ok && h->alloc(&h->bn_choice, 16, ws);
+  ok = ok && h->alloc(&h->sched, 16, ws);
   ok = ok && h->alloc(&h->tiles_gu, h->max_tiles_gu * 16, ws);
   ok = ok && h->alloc(&h->tiles_dn, h->max_tiles_dn * 16, ws);
-  ok = ok && h->alloc(&h->ntiles, 32, ws);   // 4 tile counts + the routed row count
+  ok = ok && h->alloc(&h->ntiles, 32, ws);   // 4 tile counts, the routed row count, 2 thin-tile starts
   ok = ok && h->alloc(&h->h, h->R * I * 2, ws);
   ok = ok && h->alloc(&h->o, h->R * H * 4, ws);
   ok = ok && h->alloc(&h->status, 16, ws);
@@ -392,7 +394,7 @@ moe_status create_impl(const moe_config* cfg, const moe_weights* w, int32_t e_be
 
   bool err = false;
   err |= cudaMemsetAsync(h->status, 0, 16, s) != cudaSuccess;
-  err |= cudaMemsetAsync(h->ntiles, 0, 16, s) != cudaSuccess;
+  err |= cudaMemsetAsync(h->ntiles, 0, 32, s) != cudaSuccess;
   err |= cudaMemcpyAsync(h->wg, w->router_w, E * H * 2, cudaMemcpyDeviceToDevice, s) != cudaSuccess;
   if (w->router_bias) err |= cudaMemcpyAsync(h->bias, w->router_bias, E * 4, cudaMemcpyDeviceToDevice, s) != cudaSuccess;
   if (!mx) {
@@ -634,6 +636,7 @@ moe_status forward_impl(moe_handle* h, const void* x, const int32_t* token_ids, 
   sa.nrows_routed = h->ntiles + 4;
   sa.bn_alt = alt ? kBnAlt : 0;
   sa.bn_choice = alt ? h->bn_choice : nullptr;
+  sa.sched_zero = alt ? h->sched : nullptr;
   if (nchunks == 1) {
     h->prof_mark(kKPermScan, s);
     MOE_TRY_CUDA(launch_perm_fused(sa, h->idx, nslots, h->perm, h->inv, h->status, s));
@@ -681,6 +684,8 @@ moe_status forward_impl(moe_handle* h, const void* x, const int32_t* token_ids, 
       h->prof_mark(kKGateUp, s);
       if (alt) {
         a.bn_select = h->bn_choice;
+        a.thin_begin = h->ntiles + 5;
+        a.sched = h->sched;
         MOE_TRY_CUDA(launch_gemm_gateup_dual(h->tm_w13, tm_b, tm_x, a, h->num_sms, s));
       } else {
         MOE_TRY_CUDA(launch_gemm_gateup(h->tm_w13, tm_b, tm_x, a, bn_gu, h->num_sms, s));
@@ -713,6 +718,8 @@ moe_status forward_impl(moe_handle* h, const void* x, const int32_t* token_ids, 
     } else if (alt) {
       h->prof_mark(kKDown, s);
       d.bn_select = h->bn_choice;
+      d.thin_begin = h->ntiles + 6;
+      d.sched = h->sched + 2;
       MOE_TRY_CUDA(launch_gemm_down_wide_dual(h->tm_w2w, h->tm_h, d, h->num_sms, s));
     } else {
       h->prof_mark(kKDown, s);
@@ -1038,7 +1045,7 @@ moe_status moe_inspect(moe_handle* h, int32_t what, void* dst, size_t bytes, moe
       src = h->sfb_dn;
       cap = h->max_ntiles_r * (I / 128) * 512;
       break;
-    case MOE_BUF_NTILES: src = h->ntiles; cap = 20; break;
+    case MOE_BUF_NTILES: src = h->ntiles; cap = 28; break;
     case MOE_BUF_TILES_GU: src = h->tiles_gu; cap = h->max_tiles_gu * 16; break;
     case MOE_BUF_TILES_DN: src = h->tiles_dn; cap = h->max_tiles_dn * 16; break;
     default: return MOE_ERR_INVALID_ARG;

@@ -59,6 +59,10 @@ constexpr int pow2_at_least(int v, int lo) {
 // kAMmas 128-row MMAs per K step share one B tile: gate/up always has two (W1
 // and W3 rows of the same 128 expert-width rows); the down GEMM has one, or two
 // consecutive 128-row tiles of W2 ("wide") to double the work per B byte.
+// Tile indices in flight from the producer to the MMA thread and the epilogue
+// warps when the tiles come from a counter.
+constexpr int kTileQ = 4;
+
 template <bool kGateUp, int kAMmas, int BN, int kStages>
 struct Cfg {
   static constexpr int kARows = 128 * kAMmas;
@@ -73,7 +77,7 @@ struct Cfg {
   static_assert(!kGateUp || kAMmas == 2, "gate/up tiles pair W1 and W3 rows");
   static_assert(kTmemCols <= 512, "TMEM holds 512 columns");
   static_assert(BN % kBBoxRows == 0 && BN >= 32 && BN <= 256, "BN");
-  static_assert((2 * kStages + 5) * 8 + 8 <= kBarrierBytes, "barriers");
+  static_assert((2 * kStages + 5 + 2 * kTileQ) * 8 + 8 + 4 * kTileQ <= kBarrierBytes, "barriers");
   static_assert(kSmemBytes <= 227 * 1024, "shared memory");
 };
 
@@ -154,9 +158,31 @@ __device__ __forceinline__ void drain_ring(uint64_t* full, int depth, long issue
   }
 }
 
+// Before the ring's shared memory is reused: wait (bounded) until the MMAs have
+// released every stage, so no commit still has to arrive on an empty barrier.
+template <int kStages>
+__device__ __forceinline__ void release_ring(uint64_t* empty, int stage, uint32_t phase, const GemmArgs& a,
+                                             volatile int* abort_flag) {
+  for (int i = 0; i < kStages; ++i) {
+    if (!wait_or_abort(&empty[stage], phase ^ 1, a, abort_flag)) return;
+    if (++stage == kStages) {
+      stage = 0;
+      phase ^= 1;
+    }
+  }
+}
+
+// Runs tiles [tlo, thi) of the list: every gridDim-th from tlo + blockIdx.x, or,
+// with `counter`, tlo + the counter's next value until that reaches thi (the
+// producer takes the index and hands it to the MMA thread and the epilogue warps
+// through a small queue in shared memory). With `again` another body follows in
+// the same CTA: TMEM is freed without giving up the right to allocate it, and the
+// barriers are invalidated so that their shared memory can be reused. Returns
+// false when the CTA aborted (timeout).
 template <bool kGateUp, int kAMmas, int BN, int kStages>
-__device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensorMap* tmB, const CUtensorMap* tmBsh,
-                                          const GemmArgs& args, uint8_t* smem_raw) {
+__device__ __forceinline__ bool gemm_body(const CUtensorMap* tmA, const CUtensorMap* tmB, const CUtensorMap* tmBsh,
+                                          const GemmArgs& args, uint8_t* smem_raw, int tlo, int thi,
+                                          int* counter = nullptr, bool again = false) {
   using C = Cfg<kGateUp, kAMmas, BN, kStages>;
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
@@ -167,8 +193,12 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
   uint64_t* tfull = empty + kStages;
   uint64_t* tempty = tfull + 2;
   uint64_t* drain = tempty + 2;
-  uint32_t* tmem_base_smem = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* tq_full = drain + 1;       // tile queue: index written
+  uint64_t* tq_empty = tq_full + kTileQ;  // tile queue: index read by the MMA thread and every epilogue warp
+  constexpr int kNumBars = 2 * kStages + 5 + 2 * kTileQ;
+  uint32_t* tmem_base_smem = reinterpret_cast<uint32_t*>(tq_empty + kTileQ);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_base_smem + 1);
+  volatile int* tq = reinterpret_cast<volatile int*>(tmem_base_smem + 2);
 
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
@@ -183,6 +213,10 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
       mbar_init(&tempty[i], kEpiWarps);  // one arrive per epilogue warp
     }
     mbar_init(drain, 1);
+    for (int i = 0; i < kTileQ; ++i) {
+      mbar_init(&tq_full[i], 1);
+      mbar_init(&tq_empty[i], 1 + kEpiWarps);
+    }
     *abort_flag = 0;
     fence_mbarrier_init();
   }
@@ -193,15 +227,51 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
   }
   if (warp == kWarpMma) {
     tmem_alloc(tmem_base_smem, C::kTmemCols);
-    tmem_relinquish();
+    if (!again) tmem_relinquish();
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_base_smem;
 
-  const int ntiles = tile_count<BN>(args);
-  const int tfirst = tile_first(args) + static_cast<int>(blockIdx.x);
+  const int ntiles = thi;
+  const int tfirst = tlo + static_cast<int>(blockIdx.x);
+  const bool dyn = counter != nullptr;
+  // the tile after `prev` (-1: the first), or -1 when there is none
+  auto stride_next = [&](int prev) -> int {
+    const int t = prev < 0 ? tfirst : prev + static_cast<int>(gridDim.x);
+    return t < ntiles ? t : -1;
+  };
+  // producer (one thread): next tile, published to the queue when dynamic
+  int tq_ps = 0;
+  uint32_t tq_pp = 0;
+  auto produce = [&](int prev) -> int {
+    if (!dyn) return stride_next(prev);
+    int t = tlo + atomicAdd(counter, 1);
+    if (t >= ntiles) t = -1;
+    if (!wait_or_abort(&tq_empty[tq_ps], tq_pp ^ 1, args, abort_flag)) return -1;
+    tq[tq_ps] = t;
+    mbar_arrive(&tq_full[tq_ps]);
+    if (++tq_ps == kTileQ) {
+      tq_ps = 0;
+      tq_pp ^= 1;
+    }
+    return t;
+  };
+  // consumers (the MMA thread, lane 0 of each epilogue warp): the producer's sequence
+  int tq_cs = 0;
+  uint32_t tq_cp = 0;
+  auto consume = [&](int prev) -> int {
+    if (!dyn) return stride_next(prev);
+    if (!wait_or_abort(&tq_full[tq_cs], tq_cp, args, abort_flag)) return -1;
+    const int t = tq[tq_cs];
+    mbar_arrive(&tq_empty[tq_cs]);
+    if (++tq_cs == kTileQ) {
+      tq_cs = 0;
+      tq_cp ^= 1;
+    }
+    return t;
+  };
 
   if (warp == kWarpTma) {
     // ------------------------------------------------------------ TMA producer
@@ -229,8 +299,9 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
           }
         };
         if constexpr (kPrefetch > 0)
-          for (int i = 0; i < kPrefetch; ++i) prefetch_next();
-        for (int t = tfirst; ok && t < ntiles && !*abort_flag; t += gridDim.x) {
+          if (!dyn)
+            for (int i = 0; i < kPrefetch; ++i) prefetch_next();
+        for (int t = produce(-1); ok && t >= 0 && !*abort_flag; t = produce(t)) {
           const Tile tl = load_tile<BN>(args, t);
           const CUtensorMap* mb = (kGateUp && tl.group >= args.n_routed) ? tmBsh : tmB;
           const int a_row = (tl.group - args.group_base) * args.a_rows_per_group + tl.m_tile * C::kARows;
@@ -247,7 +318,8 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
             for (int j = 0; j < nb; ++j)
               tma_load_2d(sB + stage * C::kBBytes + j * kBBoxBytes, mb, &full[stage], kx, tl.b_row0 + j * kBBoxRows,
                           kCacheEvictLast);
-            if constexpr (kPrefetch > 0) prefetch_next();
+            if constexpr (kPrefetch > 0)
+              if (!dyn) prefetch_next();
             ++issued;
             if (++stage == kStages) {
               stage = 0;
@@ -256,6 +328,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
           }
         }
         if (*abort_flag) drain_ring(full, kStages, issued, args.timeout_ns);
+        else if (again) release_ring<kStages>(empty, stage, phase, args, abort_flag);
       }
     } else {
       // Lane 0 waits on the ring and issues the weight box (and the token boxes of
@@ -283,9 +356,10 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
         }
       };
       if constexpr (kPrefetch > 0)
-        if (lane == 0)
+        if (lane == 0 && !dyn)
           for (int i = 0; i < kPrefetch; ++i) prefetch_next();
-      for (int t = tfirst; ok && t < ntiles; t += gridDim.x) {
+      for (int t = __shfl_sync(0xffffffffu, lane == 0 ? produce(-1) : 0, 0); ok && t >= 0;
+           t = __shfl_sync(0xffffffffu, lane == 0 ? produce(t) : 0, 0)) {
         if (__shfl_sync(0xffffffffu, lane == 0 ? *abort_flag : 0, 0)) break;
         const Tile tl = load_tile<BN>(args, t);
         const bool gather = kGateUp && args.gather_perm != nullptr && tl.group < args.n_routed;
@@ -318,7 +392,8 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
               for (int j = 0; j < nb; ++j)
                 tma_load_2d(sB + stage * C::kBBytes + j * kBBoxBytes, mb, &full[stage], kx, tl.b_row0 + j * kBBoxRows,
                             kCacheEvictLast);
-            if constexpr (kPrefetch > 0) prefetch_next();
+            if constexpr (kPrefetch > 0)
+              if (!dyn) prefetch_next();
           }
           __syncwarp();
           if (gather) {
@@ -338,6 +413,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
         }
       }
       if (lane == 0 && *abort_flag) drain_ring(full, kStages, issued, args.timeout_ns);
+      else if (lane == 0 && again) release_ring<kStages>(empty, stage, phase, args, abort_flag);
     }
   } else if (warp == kWarpMma) {
     // ------------------------------------------------------------ MMA issuer
@@ -347,7 +423,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
       int acc = 0;
       uint32_t acc_phase = 0;
       bool ok = true;
-      for (int t = tfirst; ok && t < ntiles && !*abort_flag; t += gridDim.x) {
+      for (int t = consume(-1); ok && t >= 0 && !*abort_flag; t = consume(t)) {
         const Tile tl = load_tile<BN>(args, t);
         const uint32_t n_mma = max(16, (tl.nrows + 15) & ~15);
         const uint32_t idesc = idesc_bf16_f32(128, n_mma);
@@ -395,7 +471,8 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
     const int cfirst = ((warp - 2) / 4) * 16;  // this warp's first 16-column chunk
     int acc = 0;
     uint32_t acc_phase = 0;
-    for (int t = tfirst; t < ntiles; t += gridDim.x) {
+    for (int t = __shfl_sync(0xffffffffu, lane == 0 ? consume(-1) : 0, 0); t >= 0;
+         t = __shfl_sync(0xffffffffu, lane == 0 ? consume(t) : 0, 0)) {
       const Tile tl = load_tile<BN>(args, t);
       const int n_mma = max(16, (tl.nrows + 15) & ~15);
       bool ok = true;
@@ -479,6 +556,14 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tmA, const CUtensor
     tc_fence_after();
     tmem_dealloc(tmem_base, C::kTmemCols);
   }
+  const bool ok = *abort_flag == 0;
+  if (again) {
+    __syncthreads();
+    if (threadIdx.x == 0)
+      for (int i = 0; i < kNumBars; ++i) mbar_inval(&bars[i]);
+    __syncthreads();
+  }
+  return ok;
 }
 
 // Bounded wait until *p >= target (acquire); gives up when another role of the CTA
@@ -747,20 +832,57 @@ __global__ void __launch_bounds__(kThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                         const __grid_constant__ CUtensorMap tmBsh, const GemmArgs args) {
   extern __shared__ uint8_t smem_raw[];
-  gemm_body<kGateUp, kAMmas, BN, kStages>(&tmA, &tmB, &tmBsh, args, smem_raw);
+  gemm_body<kGateUp, kAMmas, BN, kStages>(&tmA, &tmB, &tmBsh, args, smem_raw, tile_first(args),
+                                          tile_count<BN>(args));
+}
+
+// The ring of the thin tiles: kThinRows-token stages, as many as fit.
+template <int kAMmas>
+constexpr int thin_stages() {
+  return (227 * 1024 - 1024 - 512) / (kAMmas * 128 * 128 + kThinRows * 128);
 }
 
 // Two token-tile widths in one launch: the width the permutation kernel chose
-// (*args.bn_select, written before this grid starts) selects the body.
+// (*args.bn_select, written before this grid starts) selects the body. With
+// args.thin_begin (kThinSplit) the list's thin tail is a second list: the last
+// CTAs, in proportion to its estimated work (a thin tile counted as half a wide
+// one), start on it with the thin ring, the others on the wide tiles, both lists
+// taken through counters, and every CTA moves to the other list when its own is
+// done.
 template <bool kGateUp, int kAMmas, int BN1, int S1, int BN2, int S2>
 __global__ void __launch_bounds__(kThreads, 1)
     grouped_gemm_dual_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                              const __grid_constant__ CUtensorMap tmBsh, const GemmArgs args) {
   extern __shared__ uint8_t smem_raw[];
-  if (*args.bn_select == BN2)
-    gemm_body<kGateUp, kAMmas, BN2, S2>(&tmA, &tmB, &tmBsh, args, smem_raw);
-  else
-    gemm_body<kGateUp, kAMmas, BN1, S1>(&tmA, &tmB, &tmBsh, args, smem_raw);
+  const int n = *args.ntiles;
+  const bool wide2 = *args.bn_select == BN2;
+  int mid = n;
+  if (kThinSplit && args.thin_begin != nullptr && args.sched != nullptr) mid = min(max(*args.thin_begin, 0), n);
+  if (mid == n) {
+    if (wide2)
+      gemm_body<kGateUp, kAMmas, BN2, S2>(&tmA, &tmB, &tmBsh, args, smem_raw, 0, n);
+    else
+      gemm_body<kGateUp, kAMmas, BN1, S1>(&tmA, &tmB, &tmBsh, args, smem_raw, 0, n);
+    return;
+  }
+  if constexpr (kThinSplit) {
+    const int G = static_cast<int>(gridDim.x);
+    const float w_thin = 0.5f * static_cast<float>(n - mid), w_wide = static_cast<float>(mid);
+    const int n_thin = mid == 0 ? G : min(max(static_cast<int>(G * w_thin / (w_thin + w_wide) + 0.5f), 1), G);
+    auto wide = [&](bool again) {
+      return wide2 ? gemm_body<kGateUp, kAMmas, BN2, S2>(&tmA, &tmB, &tmBsh, args, smem_raw, 0, mid, args.sched, again)
+                   : gemm_body<kGateUp, kAMmas, BN1, S1>(&tmA, &tmB, &tmBsh, args, smem_raw, 0, mid, args.sched, again);
+    };
+    auto thin = [&](bool again) {
+      return gemm_body<kGateUp, kAMmas, kThinRows, thin_stages<kAMmas>()>(&tmA, &tmB, &tmBsh, args, smem_raw, mid, n,
+                                                                         args.sched + 1, again);
+    };
+    if (static_cast<int>(blockIdx.x) >= G - n_thin) {
+      if (thin(true)) wide(false);
+    } else {
+      if (wide(true)) thin(false);
+    }
+  }
 }
 
 template <bool kGateUp, int kAMmas, int BN, int kStages>
@@ -772,9 +894,9 @@ cudaError_t set_attr() {
 
 template <bool kGateUp, int kAMmas, int BN1, int S1, int BN2, int S2>
 constexpr int dual_smem() {
-  return Cfg<kGateUp, kAMmas, BN1, S1>::kSmemBytes > Cfg<kGateUp, kAMmas, BN2, S2>::kSmemBytes
-             ? Cfg<kGateUp, kAMmas, BN1, S1>::kSmemBytes
-             : Cfg<kGateUp, kAMmas, BN2, S2>::kSmemBytes;
+  constexpr int a = Cfg<kGateUp, kAMmas, BN1, S1>::kSmemBytes, b = Cfg<kGateUp, kAMmas, BN2, S2>::kSmemBytes;
+  constexpr int c = kThinSplit ? Cfg<kGateUp, kAMmas, kThinRows, thin_stages<kAMmas>()>::kSmemBytes : 0;
+  return a > b ? (a > c ? a : c) : (b > c ? b : c);
 }
 
 template <bool kGateUp, int kAMmas, int BN1, int S1, int BN2, int S2>

@@ -47,6 +47,10 @@ struct GemmArgs {
   int* status;                  // device status word
   unsigned long long timeout_ns;
   const int* bn_select;         // dual-width launch: the token-tile width the permutation chose
+  const int* thin_begin;        // dual-width launch: device index from which every tile has at most
+                                //   kThinRows rows (nullptr: one tile list, taken by stride)
+  int* sched;                   // dual-width launch with thin_begin: two tile counters (wide, thin),
+                                //   zero before the launch
   const int32_t* gather_perm;   // gate/up: routed B rows are x rows perm[row] / gather_k, fetched by
   int gather_k;                 //   tile::gather4 through tmB (a one-row box map of x); nullptr = B rows as stored
 };
@@ -123,7 +127,9 @@ struct ScanArgs {
   int32_t* off;
   int4* tiles_gu;
   int4* tiles_dn;
-  int* ntiles;                  // [gu_end, dn_end, gu_shared_end, dn_shared_end]
+  int* ntiles;                  // [gu_end, dn_end, gu_shared_end, dn_shared_end, (routed rows),
+                                //  gu_thin_begin, dn_thin_begin]
+  int* sched_zero;              // when not null: 4 tile counters of the dual-width GEMMs, zeroed here
   int m_tiles_gu, m_tiles_dn;
   int bn_gu_r, bn_dn_r;         // token tile of routed groups (gate/up, down)
   int bn_gu_s, bn_dn_s;         // token tile of shared groups
@@ -162,6 +168,19 @@ static_assert(kBnLarge % 32 == 0 && kBnLarge >= 32 && kBnLarge <= 256, "large to
 constexpr int kBnAlt = MOE_BN_ALT;
 static_assert(kBnAlt == 0 || (kBnAlt % 32 == 0 && kBnAlt >= 32 && kBnAlt < kBnLarge && kBnAlt != 128 &&
                               kBnAlt != 32), "alternative token tile");
+// Thin tiles: in a longest-first list of many-token tiles the partial token tiles
+// of at most kThinRows rows come last (a skewed batch's cold experts). They only
+// stream weights, which a ring of kThinRows-token stages does with about twice the
+// bytes in flight of the wide-tile ring. With kThinSplit the dual-width launch
+// takes tiles from two counters, one per list: some CTAs start on the thin list
+// (on that ring) while the others run the wide tiles, so the weight streaming
+// overlaps the compute-bound tiles, and each CTA moves to the other list when its
+// own runs dry.
+constexpr int kThinRows = 32;
+#ifndef MOE_THIN_SPLIT
+#define MOE_THIN_SPLIT 1
+#endif
+constexpr bool kThinSplit = MOE_THIN_SPLIT != 0;
 // bn: 32 (few tokens per group), 128 or kBnLarge (gate/up) and 32 or kBnLarge
 // (down).
 cudaError_t launch_gemm_gateup(const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap& tmBsh,

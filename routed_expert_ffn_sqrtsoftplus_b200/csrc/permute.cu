@@ -25,13 +25,23 @@ constexpr int kMaxSegs = 2 * kMaxScanGroups;  // tile-list segments (shared, ful
 #define MOE_TILE_ORDER_LPT 1
 #endif
 constexpr bool kTileOrderLongestFirst = MOE_TILE_ORDER_LPT != 0;
-// Full and partial routed token tiles spread evenly over the list (1), so that the
-// compute-heavy full tiles of hot experts run beside the weight-streaming partial
-// tiles of cold ones, or full tiles first (0).
-#ifndef MOE_TILE_ORDER_MIX
-#define MOE_TILE_ORDER_MIX 0
+// In a longest-first list, the partial last token tile of a group that also has
+// full tiles follows that group's full tiles of the same weight tile (1), so that
+// the CTAs taking consecutive tiles read the weight box together, through L2; only
+// the groups without a full tile make up the longest-first tail. Or every partial
+// tile in that tail (0), where a hot expert's partial tiles read their weights from
+// HBM again.
+#ifndef MOE_TILE_ORDER_HOT_PARTIAL
+#define MOE_TILE_ORDER_HOT_PARTIAL 1
 #endif
-constexpr bool kTileOrderMix = MOE_TILE_ORDER_MIX != 0;
+constexpr bool kTileOrderHotPartial = MOE_TILE_ORDER_HOT_PARTIAL != 0;
+
+// Token tiles of routed group g (n rows) in its full-tile segment: the full ones,
+// and with `hp` (a group that has full tiles) its partial last one as well.
+__device__ __forceinline__ int full_seg_tiles(int n, int bn, bool hp) {
+  if (!hp) return n / bn;
+  return n >= bn ? (n + bn - 1) / bn : 0;
+}
 
 // Expert windows (expert parallelism): this layer instance holds routed experts
 // [e_begin, e_begin + E) of e_global; a slot whose expert lies outside the window
@@ -98,6 +108,8 @@ __global__ void __launch_bounds__(1024) perm_scan_kernel(ScanArgs a, int fused, 
   __shared__ int part_g[2][kMaxScanGroups];      // routed group of each partial-tile segment
   __shared__ int rem_s[kMaxScanGroups];          // rows of each routed group's partial token tile
   __shared__ int nseg_s[2];
+  __shared__ bool hp_list[2];
+  __shared__ int nbig_s[2];
   __shared__ int slot_e[kPermChunk];             // fused: each slot's group (-1: not this instance's)
   __shared__ int warp_tot[32];
   __shared__ int tot;
@@ -167,14 +179,18 @@ __global__ void __launch_bounds__(1024) perm_scan_kernel(ScanArgs a, int fused, 
   // costliest tiles first, so the last round holds the cheapest ones.
   //   segments 0 .. S-1          every tile of shared group j (T rows)
   //   segments S .. S+E-1        the full token tiles of routed group g, all m tiles
+  //                              (with hp: and its partial last tile, after the
+  //                              full ones of the same m tile)
   //   segments S+E .. S+E+P-1    the partial last token tile of each routed group
-  //                              that has one, by its row count descending
+  //                              that has one (with hp: of each group without a
+  //                              full tile), by its row count descending
   //                              (ties: lower group first), all m tiles
   // Thread i owns segments 2i and 2i + 1 of the scan (S + 2E <= 2 * blockDim).
   for (int list = 0; list < 2; ++list) {
     const int bnr = list == 0 ? bn_gu_r : bn_dn_r, bns = list == 0 ? bn_gu_s : bn_dn_s;
     const int mtl = list == 0 ? a.m_tiles_gu : a.m_tiles_dn;
-    for (int g = tid; g < a.E; g += blockDim.x) rem_s[g] = cnt_s[g] % bnr;
+    const bool hp = kTileOrderHotPartial && kTileOrderLongestFirst && a.sort_partial;
+    for (int g = tid; g < a.E; g += blockDim.x) rem_s[g] = (hp && cnt_s[g] >= bnr) ? 0 : cnt_s[g] % bnr;
     __syncthreads();
     if (kTileOrderLongestFirst && a.sort_partial) {
       // rank of each partial tile: longer ones first, ties by group (O(E) per thread)
@@ -196,18 +212,21 @@ __global__ void __launch_bounds__(1024) perm_scan_kernel(ScanArgs a, int fused, 
       if (has) part_g[list][rank] = tid;
     }
     const int npart = __syncthreads_count(tid < a.E && rem_s[tid] > 0);
+    const int nbig = __syncthreads_count(tid < a.E && rem_s[tid] > kThinRows);  // partial tiles before the thin ones
     const int ns = a.S + a.E + npart;
     const int sh_tiles = mtl * ((a.T + bns - 1) / bns);
     int c[2];
     for (int q = 0; q < 2; ++q) {
       const int sgi = 2 * tid + q;
-      c[q] = sgi >= ns ? 0 : sgi < a.S ? sh_tiles : sgi < a.S + a.E ? mtl * (cnt_s[sgi - a.S] / bnr) : mtl;
+      c[q] = sgi >= ns ? 0 : sgi < a.S ? sh_tiles : sgi < a.S + a.E ? mtl * full_seg_tiles(cnt_s[sgi - a.S], bnr, hp) : mtl;
     }
     const int ex = block_exclusive_scan(c[0] + c[1], warp_tot, &tot);
     if (2 * tid <= ns) seg_pre[list][2 * tid] = ex;
     if (2 * tid + 1 <= ns) seg_pre[list][2 * tid + 1] = ex + c[0];
     if (tid == 0) {
       nseg_s[list] = ns;
+      nbig_s[list] = nbig;
+      hp_list[list] = hp;
       a.ntiles[list] = tot;
     }
     __syncthreads();
@@ -215,7 +234,13 @@ __global__ void __launch_bounds__(1024) perm_scan_kernel(ScanArgs a, int fused, 
   if (tid == 0) {
     a.ntiles[2] = seg_pre[0][a.S];   // shared tiles end (= 0 without shared experts)
     a.ntiles[3] = seg_pre[1][a.S];
+    // where the thin tiles (at most kThinRows rows) begin: they end a list ordered
+    // longest first; the list's end otherwise
+    const bool sorted = kTileOrderLongestFirst && a.sort_partial;
+    for (int list = 0; list < 2; ++list)
+      a.ntiles[5 + list] = sorted ? seg_pre[list][a.S + a.E + nbig_s[list]] : seg_pre[list][nseg_s[list]];
   }
+  if (a.sched_zero != nullptr && tid < 4) a.sched_zero[tid] = 0;
   // 3. outputs
   for (int g = tid; g <= G; g += blockDim.x) {
     a.off[g] = off_s[g];
@@ -239,24 +264,13 @@ __global__ void __launch_bounds__(1024) perm_scan_kernel(ScanArgs a, int fused, 
     const int bnr = list == 0 ? bn_gu_r : bn_dn_r, bns = list == 0 ? bn_gu_s : bn_dn_s;
     int4* out = list == 0 ? a.tiles_gu : a.tiles_dn;
     const int total = pre[ns];
-    // mixed order: routed position r takes full tile floor(r NF / N) when that count
-    // steps up at r, else the next partial tile (each of the N = NF + NP once)
-    const int sh_end = pre[a.S], full_end = pre[a.S + a.E];
-    const long long NF = full_end - sh_end, NR = total - sh_end;
-    const bool mix = kTileOrderMix && a.sort_partial && NF > 0 && NR > NF;
     for (int t = tid; t < total; t += blockDim.x) {
-      int pos = t;
-      if (mix && t >= sh_end) {
-        const long long r = t - sh_end;
-        const long long f0 = r * NF / NR, f1 = (r + 1) * NF / NR;
-        pos = f1 > f0 ? sh_end + static_cast<int>(f0) : full_end + static_cast<int>(r - f0);
-      }
       int lo = 0, hi = ns - 1;
-      while (lo < hi) {  // last segment with pre <= pos
+      while (lo < hi) {  // last segment with pre <= t
         const int mid = (lo + hi + 1) >> 1;
-        if (pre[mid] <= pos) lo = mid; else hi = mid - 1;
+        if (pre[mid] <= t) lo = mid; else hi = mid - 1;
       }
-      const int local = pos - pre[lo];
+      const int local = t - pre[lo];
       int g, mt, nt;
       if (lo < a.S) {
         g = a.E + lo;
@@ -265,7 +279,7 @@ __global__ void __launch_bounds__(1024) perm_scan_kernel(ScanArgs a, int fused, 
         nt = local % ntn;
       } else if (lo < a.S + a.E) {
         g = lo - a.S;
-        const int nf = cnt_s[g] / bnr;
+        const int nf = full_seg_tiles(cnt_s[g], bnr, hp_list[list]);
         mt = local / nf;
         nt = local % nf;
       } else {

@@ -283,20 +283,29 @@ def test_nan_token_is_contained_warp_topk(cuda_device):
 
 def _check_tile_list(tiles, n_shared_end, cnt, off, E, gateup, longest_first):
     """Every group's rows covered once per weight tile; shared tiles first; with
-    many tokens per expert the partial (last) token tiles of the routed groups by
-    row count, non-increasing (the full tiles come before them or spread among
-    them, by the build's order), else the routed tiles in group order."""
+    many tokens per expert each (group, weight tile)'s token tiles adjacent, full
+    ones first, and the groups with a single token tile shorter than the widest at
+    the end, by row count non-increasing; else the routed tiles in group order."""
     g = tiles[:, 0] & 0xFFFF
     mt = tiles[:, 0] >> 16
     y, z, rows = tiles[:, 1], tiles[:, 2], tiles[:, 3]
     assert np.all(g[:n_shared_end] >= E) and np.all(g[n_shared_end:] < E)
     r = rows[n_shared_end:]
     if longest_first:
-        gr = g[n_shared_end:]
-        last = (z[n_shared_end:] - off[gr] + r) == cnt[gr]     # the group's last token tile
-        full = r == r.max()
-        part = r[last & ~full]
-        assert np.all(part[:-1] >= part[1:]), "partial tiles are not longest first"
+        gr, mr = g[n_shared_end:], mt[n_shared_end:]
+        key = gr * 65536 + mr
+        runs = np.flatnonzero(np.r_[True, key[1:] != key[:-1]])          # starts of (group, m tile) runs
+        assert len(np.unique(key[runs])) == len(runs), "a (group, m tile)'s token tiles are not adjacent"
+        ends = np.r_[runs[1:], len(key)]
+        for a_, b_ in zip(runs, ends):
+            assert np.all(r[a_:b_ - 1] >= r[a_ + 1:b_]), "full token tiles do not come first"
+        single = (ends - runs) == 1
+        cold = single & (r[runs] < r.max())                               # no full tile for sure
+        if cold.any():
+            first = int(np.argmax(cold))
+            assert np.all(cold[first:]), "groups without a full tile are not last"
+            rc = r[runs[first:]]
+            assert np.all(rc[:-1] >= rc[1:]), "the tail is not longest first"
     else:
         gr = g[n_shared_end:]
         full = r == r.max()
@@ -335,13 +344,23 @@ def test_tile_lists_are_complete_and_longest_first(tiny, cuda_device, T, hot):
         _run(layer, x)
         dev = x.device
         G = WL.E + WL.n_shared
-        nt = layer.inspect(moe.BUF_NTILES, torch.empty(4, dtype=torch.int32, device=dev)).cpu().numpy()
+        nt = layer.inspect(moe.BUF_NTILES, torch.empty(7, dtype=torch.int32, device=dev)).cpu().numpy()
         cnt = layer.inspect(moe.BUF_COUNTS, torch.empty(G, dtype=torch.int32, device=dev)).cpu().numpy()
         off = layer.inspect(moe.BUF_OFFSETS, torch.empty(G + 1, dtype=torch.int32, device=dev)).cpu().numpy()
-        for which, n, ns, gateup in ((moe.BUF_TILES_GU, nt[0], nt[2], True), (moe.BUF_TILES_DN, nt[1], nt[3], False)):
+        for which, n, ns, thin, gateup in ((moe.BUF_TILES_GU, nt[0], nt[2], nt[5], True),
+                                           (moe.BUF_TILES_DN, nt[1], nt[3], nt[6], False)):
             tl = layer.inspect(which, torch.empty((int(n), 4), dtype=torch.int32, device=dev)).cpu().numpy()
             _check_tile_list(tl.astype(np.int64), int(ns), cnt.astype(np.int64), off.astype(np.int64), WL.E, gateup,
                              longest_first=T > 32)
+            # the thin tail: tiles of routed groups of at most 32 rows in all, and every
+            # such group's tiles when the list is ordered longest first (else it is empty)
+            g = tl[:, 0] & 0xFFFF
+            assert int(ns) <= int(thin) <= int(n)
+            assert np.all(g[thin:] < WL.E) and np.all(cnt[g[thin:]] <= 32)
+            if T > 32:
+                assert np.all(cnt[g[ns:thin]] > 32)
+            else:
+                assert thin == n
     finally:
         if made is not None:
             made.close()
