@@ -116,7 +116,7 @@ class ClockSampler:
                0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
                0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
 
-    def __init__(self, index: int, period_s: float = 0.02):
+    def __init__(self, index: int, period_s: float = 0.005):
         self.samples, self.reasons, self.max_mhz = [], set(), None
         self.period, self.index = period_s, index
         self._stop = threading.Event()
