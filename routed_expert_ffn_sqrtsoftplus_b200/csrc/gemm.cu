@@ -41,6 +41,18 @@ namespace {
 #define MOE_EPI_WARPS 12
 #endif
 constexpr int kEpiWarps = MOE_EPI_WARPS;  // a multiple of 4
+// Epilogue rows staged in shared memory for 16-byte global stores where the ring
+// leaves room (1), or stored one element per lane (0). Measured on V4-Pro: the
+// gate/up's BF16 h rows gain (gate/up 1.25-1.27 ms against 1.27-1.29), the down's
+// fp32 O rows lose (0.69-0.70 against 0.67-0.68), so only the former by default.
+#ifndef MOE_EPI_STAGE
+#define MOE_EPI_STAGE 1
+#endif
+#ifndef MOE_EPI_STAGE_DOWN
+#define MOE_EPI_STAGE_DOWN 0
+#endif
+constexpr bool kEpiStage = MOE_EPI_STAGE != 0;
+constexpr bool kEpiStageDown = MOE_EPI_STAGE_DOWN != 0;
 constexpr int kEpiGroups = kEpiWarps / 4;
 constexpr int kThreads = 64 + 32 * kEpiWarps;
 static_assert(kEpiWarps % 4 == 0 && kEpiWarps >= 4 && kEpiWarps <= 16, "epilogue warps");
@@ -77,7 +89,15 @@ struct Cfg {
   static constexpr int kAccBufs = 2 * kAccCols <= 512 ? 2 : 1;
   static constexpr int kTmemCols = pow2_at_least(kAccBufs * kAccCols, 32);
   static constexpr int kBarrierBytes = 512;
-  static constexpr int kSmemBytes = 1024 + kStages * (kABytes + kBBytes) + kBarrierBytes;
+  static constexpr int kBaseBytes = 1024 + kStages * (kABytes + kBBytes) + kBarrierBytes;
+  // Epilogue staging, when it fits beside the ring: each epilogue warp turns its 16 x 32
+  // chunk into 16-byte row segments for the global stores (kEpiStage: BF16 h rows of
+  // the gate/up GEMM; fp32 O rows with kEpiStageDown).
+  static constexpr int kStageWarpBytes = kGateUp ? 16 * 32 * 2 : 16 * 32 * 4;
+  static constexpr bool kStaged = kGateUp ? kEpiStage : kEpiStageDown;
+  static constexpr int kStageBytes =
+      kStaged && kBaseBytes + kEpiWarps * kStageWarpBytes <= 227 * 1024 ? kEpiWarps * kStageWarpBytes : 0;
+  static constexpr int kSmemBytes = kBaseBytes + kStageBytes;
   static_assert(!kGateUp || kAMmas == 2, "gate/up tiles pair W1 and W3 rows");
   static_assert(kTmemCols <= 512, "TMEM holds 512 columns");
   static_assert(BN % kBBoxRows == 0 && BN >= 32 && BN <= 256, "BN");
@@ -203,6 +223,7 @@ __device__ __forceinline__ bool gemm_body(const CUtensorMap* tmA, const CUtensor
   uint32_t* tmem_base_smem = reinterpret_cast<uint32_t*>(tq_empty + kTileQ);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_base_smem + 1);
   volatile int* tq = reinterpret_cast<volatile int*>(tmem_base_smem + 2);
+  uint8_t* stage_base = reinterpret_cast<uint8_t*>(bars) + C::kBarrierBytes;  // C::kStageBytes of staging
 
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
@@ -473,6 +494,8 @@ __device__ __forceinline__ bool gemm_body(const CUtensorMap* tmA, const CUtensor
     // ------------------------------------------------------------ epilogue (warps 2..)
     const int q = warp & 3;                  // TMEM lane quarter this warp may access
     const int cfirst = ((warp - 2) / 4) * 16;  // this warp's first 16-column chunk
+    // 16-byte stores need rows and the output's column count a multiple of 8 elements
+    const bool vec_out = args.out_ld % 8 == 0 && args.m_limit % 8 == 0;
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int t = __shfl_sync(0xffffffffu, lane == 0 ? consume(-1) : 0, 0); t >= 0;
@@ -510,12 +533,31 @@ __device__ __forceinline__ bool gemm_body(const CUtensorMap* tmA, const CUtensor
             }
           } else {
             __nv_bfloat16* out = static_cast<__nv_bfloat16*>(args.out);
+            if (C::kStageBytes > 0 && vec_out) {
+              // the warp's 16 token rows x 32 columns through shared memory, then 16-byte row segments
+              __nv_bfloat16* sw = reinterpret_cast<__nv_bfloat16*>(stage_base) + (warp - 2) * 16 * 32;
 #pragma unroll
-            for (int j = 0; j < 16; ++j) {
-              const int n = c0 + j;
-              if (n < tl.nrows && m_ok) {
-                const float hv = clamped_swiglu_f32(__uint_as_float(g[j]), __uint_as_float(u[j]), args.limit);
-                out[static_cast<size_t>(tl.out_row0 + n) * args.out_ld + m] = __float2bfloat16_rn(hv);
+              for (int j = 0; j < 16; ++j)
+                sw[j * 32 + lane] =
+                    __float2bfloat16_rn(clamped_swiglu_f32(__uint_as_float(g[j]), __uint_as_float(u[j]), args.limit));
+              __syncwarp();
+              const int mw = m - lane;  // the warp's first column
+#pragma unroll
+              for (int sg = lane; sg < 64; sg += 32) {
+                const int r = sg >> 2, p = sg & 3, n = c0 + r;
+                if (n < tl.nrows && rows_ok && mw + p * 8 + 8 <= args.m_limit)
+                  *reinterpret_cast<uint4*>(out + static_cast<size_t>(tl.out_row0 + n) * args.out_ld + mw + p * 8) =
+                      *reinterpret_cast<const uint4*>(sw + r * 32 + p * 8);
+              }
+              __syncwarp();
+            } else {
+#pragma unroll
+              for (int j = 0; j < 16; ++j) {
+                const int n = c0 + j;
+                if (n < tl.nrows && m_ok) {
+                  const float hv = clamped_swiglu_f32(__uint_as_float(g[j]), __uint_as_float(u[j]), args.limit);
+                  out[static_cast<size_t>(tl.out_row0 + n) * args.out_ld + m] = __float2bfloat16_rn(hv);
+                }
               }
             }
           }
@@ -535,11 +577,28 @@ __device__ __forceinline__ bool gemm_body(const CUtensorMap* tmA, const CUtensor
             const int mi = m + i * 128;
             const bool ok_i = mi < args.m_limit && rows_ok;
             const float cb = (args.col_bias != nullptr && ok_i) ? args.col_bias[mi] : 0.0f;
+            if (C::kStageBytes > 0 && vec_out) {
+              // the warp's 16 rows x 32 columns through shared memory, then 16-byte row segments
+              float* sw = reinterpret_cast<float*>(stage_base) + (warp - 2) * 16 * 32;
 #pragma unroll
-            for (int j = 0; j < 16; ++j) {
-              const int n = c0 + j;
-              if (n < tl.nrows && ok_i)
-                out[static_cast<size_t>(tl.out_row0 + n) * args.out_ld + mi] = __uint_as_float(v[j]) + cb;
+              for (int j = 0; j < 16; ++j) sw[j * 32 + lane] = __uint_as_float(v[j]) + cb;
+              __syncwarp();
+              const int mw = mi - lane;  // the warp's first column
+#pragma unroll
+              for (int sg = lane; sg < 128; sg += 32) {
+                const int r = sg >> 3, p = sg & 7, n = c0 + r;
+                if (n < tl.nrows && rows_ok && mw + p * 4 + 4 <= args.m_limit)
+                  *reinterpret_cast<float4*>(out + static_cast<size_t>(tl.out_row0 + n) * args.out_ld + mw + p * 4) =
+                      *reinterpret_cast<const float4*>(sw + r * 32 + p * 4);
+              }
+              __syncwarp();
+            } else {
+#pragma unroll
+              for (int j = 0; j < 16; ++j) {
+                const int n = c0 + j;
+                if (n < tl.nrows && ok_i)
+                  out[static_cast<size_t>(tl.out_row0 + n) * args.out_ld + mi] = __uint_as_float(v[j]) + cb;
+              }
             }
           }
         }
@@ -562,6 +621,8 @@ __device__ __forceinline__ bool gemm_body(const CUtensorMap* tmA, const CUtensor
   }
   const bool ok = *abort_flag == 0;
   if (again) {
+    // the next body's TMA copies may land where this body's epilogue staged rows
+    fence_proxy_async_smem();
     __syncthreads();
     if (threadIdx.x == 0)
       for (int i = 0; i < kNumBars; ++i) mbar_inval(&bars[i]);
