@@ -8,8 +8,10 @@ weights resident in HBM. Prints one JSON line on rank 0.
 
   value      tokens/s over all ranks, timed with CUDA events around K steps
              (barrier + synchronize on both sides, max over ranks)
-  e2e        the same metric through moe_forward_host: the step's x copied
-             host->device and y copied back inside the timed region
+  e2e        the same metric through moe_forward_host_async (pinned host x in,
+             y out): every step's x copied host->device and its y copied back
+             inside the timed region, on the library's copy streams, overlapping
+             the neighbouring steps' layers
   roofline   the dominant kernel's algorithmic bytes per launch / its mean
              launch time (CUDA events recorded by the library on the launch
              stream during the timed steps) against the measured HBM peak
@@ -404,18 +406,23 @@ def measure(wl, steps, warmup, world, local, read_gbs=None, flush_l2=False, e2e_
     if layer.status() != moe.MOE_OK:
         raise RuntimeError(f"device status after the attribution pass of {wl.name}")
 
-    # ---- end to end through host buffers (pinned x in, y out, inside the timed region)
-    xh = x.cpu().pin_memory()
-    yh = torch.empty_like(xh).pin_memory()
+    # ---- end to end through host buffers (pinned x in, y out, inside the timed region):
+    # the pipelined host path, each step's x copied in and y copied out on the library's
+    # copy streams while the neighbouring steps' layers run; three rotating buffer pairs,
+    # since a call's buffers stay in use until two later calls have been issued
+    xh = [x.cpu().pin_memory() for _ in range(3)]
+    yh = [torch.empty_like(xh[0]).pin_memory() for _ in range(3)]
     n_e2e = e2e_steps or max(3, min(steps, 50))
-    for _ in range(2):
-        layer.forward_host(xh, yh)
+    for i in range(3):
+        layer.forward_host_async(xh[i], yh[i])
+    layer.forward_host_wait()
     torch.cuda.synchronize()
     barrier(world)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
-    for _ in range(n_e2e):
-        layer.forward_host(xh, yh)
+    for i in range(n_e2e):
+        layer.forward_host_async(xh[i % 3], yh[i % 3])
+    layer.forward_host_wait()
     e1.record(stream)
     torch.cuda.synchronize()
     barrier(world)

@@ -39,7 +39,7 @@
 extern "C" {
 #endif
 
-#define MOE_ABI_VERSION 3
+#define MOE_ABI_VERSION 4
 
 #if defined(__GNUC__)
 #define MOE_API __attribute__((visibility("default")))
@@ -219,6 +219,27 @@ MOE_API moe_status moe_forward_hashed(moe_handle* h, const void* x, const int32_
  */
 MOE_API moe_status moe_forward_host(moe_handle* h, const void* x_host, int32_t T, void* y_host,
                             int32_t* topk_idx_host, float* topk_w_host, moe_stream_t stream);
+
+/*
+ * Pipelined host path for a stream of batches: like moe_forward_host (x_host
+ * BF16 [T, hidden], y_host BF16 [T, hidden], both host memory, pinned for the
+ * copies to overlap), but the copies run on two internal streams. The layer is
+ * enqueued on `stream` after its x has arrived, and y leaves on the copy-out
+ * stream. So the copy of the next call's x and the copy-out of the previous call's
+ * y overlap this call's layer. Two device staging slots alternate between calls
+ * (the second is allocated on the first call: MOE_ERR_OOM if that fails).
+ * Ordering: x_host is read without waiting for earlier work on `stream`, and y_host
+ * is written without ordering against later work on `stream`. Call
+ * moe_forward_host_wait(h, stream) and then synchronise `stream` before reading
+ * any y_host, or reusing an x_host or y_host of a call that may still be in flight
+ * (at most the last two calls). Routing indices are not copied; hash layers and
+ * expert-window handles are not supported (MOE_ERR_INVALID_ARG, from moe_forward).
+ */
+MOE_API moe_status moe_forward_host_async(moe_handle* h, const void* x_host, int32_t T, void* y_host,
+                                  moe_stream_t stream);
+
+/* Make `stream` wait for every copy-out of moe_forward_host_async so far. */
+MOE_API moe_status moe_forward_host_wait(moe_handle* h, moe_stream_t stream);
 
 /* Synchronise the device, then report and clear the device-side status word
  * (MOE_OK, MOE_ERR_TIMEOUT or MOE_ERR_DEVICE); MOE_ERR_CUDA if the sync failed. */

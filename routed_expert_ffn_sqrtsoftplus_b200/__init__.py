@@ -35,7 +35,7 @@ EXPORTED = ("moe_create", "moe_forward", "moe_forward_host", "moe_get_status", "
             "moe_selftest_wait_timeout", "moe_get_info", "moe_profile_begin", "moe_profile_end",
             "moe_num_kernel_kinds", "moe_kernel_name", "moe_route_noalloc", "moe_quantize_mxfp8",
             "moe_set_hash_table", "moe_forward_hashed", "moe_fill_workspace", "moe_create_ep",
-            "moe_forward_partial", "moe_read_bandwidth")
+            "moe_forward_partial", "moe_read_bandwidth", "moe_forward_host_async", "moe_forward_host_wait")
 
 
 class MoEError(RuntimeError):
@@ -78,6 +78,8 @@ def lib() -> ctypes.CDLL:
             "moe_create": (I32, [ctypes.POINTER(_Config), ctypes.POINTER(_Weights), P, ctypes.POINTER(P)]),
             "moe_forward": (I32, [P, P, I32, P, P, P, P]),
             "moe_forward_host": (I32, [P, P, I32, P, P, P, P]),
+            "moe_forward_host_async": (I32, [P, P, I32, P, P]),
+            "moe_forward_host_wait": (I32, [P, P]),
             "moe_get_status": (I32, [P]),
             "moe_status_string": (ctypes.c_char_p, [I32]),
             "moe_destroy": (None, [P]),
@@ -322,6 +324,20 @@ class MoELayer:
             _need(topk_w_host, "topk_w_host", torch.float32, (T, self.top_k), "cpu")
         _check(lib().moe_forward_host(self._h, _ptr(x_host), T, _ptr(y_host), _ptr(topk_idx_host),
                                       _ptr(topk_w_host), _stream(stream)), "moe_forward_host")
+
+    def forward_host_async(self, x_host: torch.Tensor, y_host: torch.Tensor, stream=None):
+        """Pipelined host buffers in and out: the copies run on the library's own streams
+        and overlap the neighbouring calls' layers. Call forward_host_wait(stream) and
+        synchronise the stream before reading y_host or reusing a call's buffers."""
+        T = x_host.shape[0]
+        _need(x_host, "x_host", torch.bfloat16, (T, self.hidden), "cpu")
+        _need(y_host, "y_host", torch.bfloat16, (T, self.hidden), "cpu")
+        _check(lib().moe_forward_host_async(self._h, _ptr(x_host), T, _ptr(y_host), _stream(stream)),
+               "moe_forward_host_async")
+
+    def forward_host_wait(self, stream=None):
+        """Make the stream wait for every copy-out of forward_host_async so far."""
+        _check(lib().moe_forward_host_wait(self._h, _stream(stream)), "moe_forward_host_wait")
 
     # ------------------------------------------------------------------ inspection
     def inspect(self, what: int, out: torch.Tensor, stream=None) -> torch.Tensor:

@@ -113,6 +113,17 @@ struct moe_handle {
   int* status = nullptr;
   void* x_stage = nullptr;
   void* y_stage = nullptr;
+  // pipelined host path (moe_forward_host_async), set up on first use: slot 0 stages
+  // through x_stage / y_stage, slot 1 through buffers of its own
+  bool pipe_ready = false;
+  cudaStream_t pipe_in = nullptr, pipe_out = nullptr;  // host-to-device and device-to-host copies
+  cudaEvent_t pipe_copied_in[2] = {nullptr, nullptr};  // x of the slot on the device
+  cudaEvent_t pipe_done[2] = {nullptr, nullptr};       // the layer finished with the slot's x and y
+  cudaEvent_t pipe_copied_out[2] = {nullptr, nullptr}; // y of the slot on the host
+  void* pipe_x[2] = {nullptr, nullptr};
+  void* pipe_y[2] = {nullptr, nullptr};
+  int pipe_slot = 0;
+  uint64_t pipe_bytes = 0;
 
   CUtensorMap tm_w13, tm_w2, tm_xp, tm_h, tm_wg;
   CUtensorMap tm_w2w;           // W2 with 256-row boxes (wide down tiles)
@@ -184,6 +195,16 @@ struct moe_handle {
   void release() {
     for (void* p : allocs) cudaFree(p);
     allocs.clear();
+    for (int i = 0; i < 2; ++i) {
+      if (pipe_copied_in[i]) cudaEventDestroy(pipe_copied_in[i]);
+      if (pipe_done[i]) cudaEventDestroy(pipe_done[i]);
+      if (pipe_copied_out[i]) cudaEventDestroy(pipe_copied_out[i]);
+      pipe_copied_in[i] = pipe_done[i] = pipe_copied_out[i] = nullptr;
+    }
+    if (pipe_in) cudaStreamDestroy(pipe_in);
+    if (pipe_out) cudaStreamDestroy(pipe_out);
+    pipe_in = pipe_out = nullptr;
+    pipe_ready = false;
     if (hash_table != nullptr) cudaFree(hash_table);
     hash_table = nullptr;
     for (cudaEvent_t e : ev) cudaEventDestroy(e);
@@ -961,6 +982,60 @@ moe_status moe_forward_host(moe_handle* h, const void* x_host, int32_t T, void* 
   const size_t kb = static_cast<size_t>(T) * h->cfg.top_k * 4;
   if (topk_idx_host) MOE_TRY_CUDA(cudaMemcpyAsync(topk_idx_host, h->idx, kb, cudaMemcpyDeviceToHost, s));
   if (topk_w_host) MOE_TRY_CUDA(cudaMemcpyAsync(topk_w_host, h->wts, kb, cudaMemcpyDeviceToHost, s));
+  return MOE_OK;
+}
+
+moe_status moe_forward_host_async(moe_handle* h, const void* x_host, int32_t T, void* y_host, moe_stream_t stream) {
+  if (h == nullptr) return MOE_ERR_INVALID_ARG;
+  if (T < 0 || T > h->cfg.max_tokens) return MOE_ERR_INVALID_ARG;
+  if (T == 0) return MOE_OK;
+  if (x_host == nullptr || y_host == nullptr) return MOE_ERR_INVALID_ARG;
+  if (!h->pipe_ready) {
+    // two copy streams, the slots' events, and the second slot's staging buffers
+    const size_t stage = static_cast<size_t>(h->cfg.max_tokens) * h->cfg.hidden * 2;
+    bool ok = cudaStreamCreateWithFlags(&h->pipe_in, cudaStreamNonBlocking) == cudaSuccess &&
+              cudaStreamCreateWithFlags(&h->pipe_out, cudaStreamNonBlocking) == cudaSuccess;
+    for (int i = 0; ok && i < 2; ++i)
+      ok = cudaEventCreateWithFlags(&h->pipe_copied_in[i], cudaEventDisableTiming) == cudaSuccess &&
+           cudaEventCreateWithFlags(&h->pipe_done[i], cudaEventDisableTiming) == cudaSuccess &&
+           cudaEventCreateWithFlags(&h->pipe_copied_out[i], cudaEventDisableTiming) == cudaSuccess;
+    if (!ok) {
+      cudaGetLastError();
+      return MOE_ERR_CUDA;
+    }
+    if (!h->alloc(&h->pipe_x[1], stage, &h->pipe_bytes) || !h->alloc(&h->pipe_y[1], stage, &h->pipe_bytes))
+      return MOE_ERR_OOM;
+    h->pipe_x[0] = h->x_stage;
+    h->pipe_y[0] = h->y_stage;
+    h->pipe_ready = true;
+  }
+  const int k = h->pipe_slot;
+  h->pipe_slot ^= 1;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const size_t bytes = static_cast<size_t>(T) * h->cfg.hidden * 2;
+  // x into slot k once the layer two calls back has finished reading it
+  MOE_TRY_CUDA(cudaStreamWaitEvent(h->pipe_in, h->pipe_done[k], 0));
+  MOE_TRY_CUDA(cudaMemcpyAsync(h->pipe_x[k], x_host, bytes, cudaMemcpyHostToDevice, h->pipe_in));
+  MOE_TRY_CUDA(cudaEventRecord(h->pipe_copied_in[k], h->pipe_in));
+  // the layer on `stream`, after that copy and after slot k's previous y has left
+  MOE_TRY_CUDA(cudaStreamWaitEvent(s, h->pipe_copied_in[k], 0));
+  MOE_TRY_CUDA(cudaStreamWaitEvent(s, h->pipe_copied_out[k], 0));
+  const moe_status st = moe_forward(h, h->pipe_x[k], T, h->pipe_y[k], nullptr, nullptr, stream);
+  if (st != MOE_OK) return st;
+  MOE_TRY_CUDA(cudaEventRecord(h->pipe_done[k], s));
+  // y out on the copy-out stream
+  MOE_TRY_CUDA(cudaStreamWaitEvent(h->pipe_out, h->pipe_done[k], 0));
+  MOE_TRY_CUDA(cudaMemcpyAsync(y_host, h->pipe_y[k], bytes, cudaMemcpyDeviceToHost, h->pipe_out));
+  MOE_TRY_CUDA(cudaEventRecord(h->pipe_copied_out[k], h->pipe_out));
+  return MOE_OK;
+}
+
+moe_status moe_forward_host_wait(moe_handle* h, moe_stream_t stream) {
+  if (h == nullptr) return MOE_ERR_INVALID_ARG;
+  if (!h->pipe_ready) return MOE_OK;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  MOE_TRY_CUDA(cudaStreamWaitEvent(s, h->pipe_copied_out[0], 0));
+  MOE_TRY_CUDA(cudaStreamWaitEvent(s, h->pipe_copied_out[1], 0));
   return MOE_OK;
 }
 

@@ -43,7 +43,7 @@ def test_exports_are_exactly_the_header(L):
 
 
 def test_abi_version_and_strings(L):
-    assert L.moe_abi_version() == 3
+    assert L.moe_abi_version() == 4
     assert L.moe_status_string(moe.MOE_OK) == b"MOE_OK"
     assert L.moe_status_string(moe.MOE_ERR_TIMEOUT) == b"MOE_ERR_TIMEOUT"
     assert L.moe_num_kernel_kinds() == len(moe.kernel_names())
@@ -113,6 +113,8 @@ def test_create_ep_rejects_bad_windows(L):
 def test_null_handle_calls(L):
     assert L.moe_forward(None, FAKE, 1, FAKE, None, None, None) == moe.MOE_ERR_INVALID_ARG
     assert L.moe_forward_host(None, FAKE, 1, FAKE, None, None, None) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_forward_host_async(None, FAKE, 1, FAKE, None) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_forward_host_wait(None, None) == moe.MOE_ERR_INVALID_ARG
     assert L.moe_get_status(None) == moe.MOE_ERR_INVALID_ARG
     assert L.moe_inspect(None, 0, FAKE, 4, None) == moe.MOE_ERR_INVALID_ARG
     assert L.moe_set_wait_timeout(None, 10) == moe.MOE_ERR_INVALID_ARG

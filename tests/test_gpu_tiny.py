@@ -199,6 +199,30 @@ def test_forward_host_matches_device(tiny):
     assert torch.equal(yh, y.cpu()) and torch.equal(ih, idx.cpu())
 
 
+def test_forward_host_async_pipeline_matches_device(tiny):
+    """Calls of the pipelined host path with different batches back to back (copies on
+    the library's streams overlapping the neighbouring layers): every y equals the
+    device forward of its own x, bit for bit, also when the two staging slots are
+    reused several times and T changes between calls."""
+    lay, layer = tiny
+    Ts = [17, 64, 5, 64, 33, 1, 64]
+    xs, ys, ref = [], [], []
+    for i, T in enumerate(Ts):
+        x = lay["x"][:T].contiguous() if i % 2 == 0 else torch.flip(lay["x"][:T], dims=[0]).contiguous()
+        y, _, _ = _run(layer, x)
+        ref.append(y.cpu())
+        xs.append(x.cpu().pin_memory())
+        ys.append(torch.full((T, WL.H), float("nan"), dtype=torch.bfloat16).pin_memory())
+    torch.cuda.synchronize()
+    for xh, yh in zip(xs, ys):
+        layer.forward_host_async(xh, yh)
+    layer.forward_host_wait()
+    torch.cuda.synchronize()
+    assert layer.status() == moe.MOE_OK
+    for i, (yh, r) in enumerate(zip(ys, ref)):
+        assert torch.equal(yh, r), f"call {i} (T={Ts[i]})"
+
+
 def test_bounded_wait_reports_timeout(tiny):
     _, layer = tiny
     assert layer.status() == moe.MOE_OK
