@@ -23,6 +23,13 @@ namespace {
 constexpr int kTcRouterMinTokens = 256;
 // Token counts up to this use the sliced CUDA-core router and the per-token top-k.
 constexpr int kSmallRouterMaxTokens = 32;
+// Router logits of at most kSmallRouterMaxTokens tokens on the tensor cores (the
+// dense grouped-GEMM mode, K split in slices of 128) (1), or on the CUDA cores,
+// hidden-sliced (0).
+#ifndef MOE_ROUTER_TC_SMALL
+#define MOE_ROUTER_TC_SMALL 0
+#endif
+constexpr bool kRouterTcSmall = MOE_ROUTER_TC_SMALL != 0;
 // Top-k with one CTA per token up to this many tokens (the candidates of a token
 // are re-scored by 8 warps in parallel); one warp per token above (measured on
 // B200: the CTA form halves the time at T=256 and is slower from T=2048 on).
@@ -575,12 +582,36 @@ moe_status forward_impl(moe_handle* h, const void* x, const int32_t* token_ids, 
                                    c.route_scale, h->idx, h->wts, h->status, s));
     h->prof_done(s);
   } else if (T <= kSmallRouterMaxTokens) {
-    h->prof_mark(kKRouterLogits, s);
-    MOE_TRY_CUDA(launch_router_small(x, h->wg, h->zpart, T, H, E, s));
-    h->prof_done(s);
+    int nparts = 0;
+    if (kRouterTcSmall) {
+      // the logits on the tensor cores: 128-expert x 32-token tiles, K cut into
+      // H / 128 slices of two K blocks, each slice's fp32 partial sums a slice of zpart
+      GemmArgs a{};
+      a.dense_m_tiles = (E + 127) / 128;
+      a.dense_rows = T;
+      a.num_kb = H / 64;
+      a.dense_k_splits = H / 128;
+      a.split_stride = static_cast<size_t>(T) * E;
+      a.out = h->zpart;
+      a.out_ld = E;
+      a.out_rows = T;
+      a.m_limit = E;
+      a.status = h->status;
+      a.timeout_ns = h->timeout_ns;
+      const int nt = a.dense_m_tiles * a.dense_k_splits;
+      h->prof_mark(kKRouterGemm, s);
+      MOE_TRY_CUDA(launch_gemm_down(h->tm_wg, tm_x, a, 32, nt < h->num_sms ? nt : h->num_sms, s));
+      h->prof_done(s);
+      nparts = a.dense_k_splits;
+    } else {
+      h->prof_mark(kKRouterLogits, s);
+      MOE_TRY_CUDA(launch_router_small(x, h->wg, h->zpart, T, H, E, s));
+      h->prof_done(s);
+      nparts = H / router_small_slice(H);
+    }
     h->prof_mark(kKTopk, s);
-    MOE_TRY_CUDA(launch_topk_small(h->zpart, H / router_small_slice(H), x, h->wg, h->bias, T, H, E, k, c.route_scale,
-                                   kRefineDelta, h->idx, h->wts, h->z, h->status, s, h->bias));
+    MOE_TRY_CUDA(launch_topk_small(h->zpart, nparts, x, h->wg, h->bias, T, H, E, k, c.route_scale, kRefineDelta,
+                                   h->idx, h->wts, h->z, h->status, s, h->bias));
     h->prof_done(s);
   } else if (T < kTcRouterMinTokens) {
     h->prof_mark(kKRouterLogits, s);
