@@ -25,7 +25,9 @@ constexpr int kTcRouterMinTokens = 256;
 constexpr int kSmallRouterMaxTokens = 32;
 // Router logits of at most kSmallRouterMaxTokens tokens on the tensor cores (the
 // dense grouped-GEMM mode, K split in slices of 128) (1), or on the CUDA cores,
-// hidden-sliced (0).
+// hidden-sliced (0). Measured at decode: the logits take half the time on the
+// tensor cores, but the top-k then sums 40 slices instead of 5, and the step is
+// the same.
 #ifndef MOE_ROUTER_TC_SMALL
 #define MOE_ROUTER_TC_SMALL 0
 #endif
