@@ -1025,18 +1025,23 @@ moe_status moe_forward_host_async(moe_handle* h, const void* x_host, int32_t T, 
   if (x_host == nullptr || y_host == nullptr) return MOE_ERR_INVALID_ARG;
   if (!h->pipe_ready) {
     // two copy streams, the slots' events, and the second slot's staging buffers
+    // (each made once; a failed set-up is resumed by the next call)
     const size_t stage = static_cast<size_t>(h->cfg.max_tokens) * h->cfg.hidden * 2;
-    bool ok = cudaStreamCreateWithFlags(&h->pipe_in, cudaStreamNonBlocking) == cudaSuccess &&
-              cudaStreamCreateWithFlags(&h->pipe_out, cudaStreamNonBlocking) == cudaSuccess;
+    auto stream_once = [](cudaStream_t* p) {
+      return *p != nullptr || cudaStreamCreateWithFlags(p, cudaStreamNonBlocking) == cudaSuccess;
+    };
+    auto event_once = [](cudaEvent_t* p) {
+      return *p != nullptr || cudaEventCreateWithFlags(p, cudaEventDisableTiming) == cudaSuccess;
+    };
+    bool ok = stream_once(&h->pipe_in) && stream_once(&h->pipe_out);
     for (int i = 0; ok && i < 2; ++i)
-      ok = cudaEventCreateWithFlags(&h->pipe_copied_in[i], cudaEventDisableTiming) == cudaSuccess &&
-           cudaEventCreateWithFlags(&h->pipe_done[i], cudaEventDisableTiming) == cudaSuccess &&
-           cudaEventCreateWithFlags(&h->pipe_copied_out[i], cudaEventDisableTiming) == cudaSuccess;
+      ok = event_once(&h->pipe_copied_in[i]) && event_once(&h->pipe_done[i]) && event_once(&h->pipe_copied_out[i]);
     if (!ok) {
       cudaGetLastError();
       return MOE_ERR_CUDA;
     }
-    if (!h->alloc(&h->pipe_x[1], stage, &h->pipe_bytes) || !h->alloc(&h->pipe_y[1], stage, &h->pipe_bytes))
+    if ((h->pipe_x[1] == nullptr && !h->alloc(&h->pipe_x[1], stage, &h->pipe_bytes)) ||
+        (h->pipe_y[1] == nullptr && !h->alloc(&h->pipe_y[1], stage, &h->pipe_bytes)))
       return MOE_ERR_OOM;
     h->pipe_x[0] = h->x_stage;
     h->pipe_y[0] = h->y_stage;
