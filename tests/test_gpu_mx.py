@@ -50,6 +50,30 @@ def test_tiny_mx_layer_parity(tiny_mx, T):
     assert rep["rel"] < parity.TOL_Y
 
 
+@pytest.mark.parametrize("T", [300])
+def test_tiny_mx_layer_parity_hot_experts(tiny_mx, cuda_device, T):
+    """A router bias of +6 on experts 0 and 1 sends every token to both: each of
+    them gets several full 96-token MX tiles and a partial one, which the tile list
+    keeps next to the full ones (their token-tile ids, scale atoms and h rows)."""
+    lay, mxq, _ = tiny_mx
+    bias = torch.zeros(WL.E, dtype=torch.float32, device=cuda_device)
+    bias[:2] = 6.0
+    hot = dict(lay, bias=bias)
+    layer = moe.MoELayer.from_layer(hot, top_k=WL.k, max_tokens=400, mx=mxq)
+    try:
+        x = lay["x"][:T].contiguous()
+        y, idx, w = layer.forward_with_routing(x)
+        torch.cuda.synchronize()
+        assert layer.status() == moe.MOE_OK
+        cnt = np.bincount(idx.cpu().numpy().ravel(), minlength=WL.E)
+        assert cnt[0] == T and cnt[1] == T
+        rep = parity.compare_layer(dict(hot, x=x), np.arange(T), y.float().cpu().numpy(), idx.cpu().numpy(),
+                                   w.cpu().numpy(), WL.k, WL.route_scale, WL.swiglu_limit, mx_q=mxq)
+        assert rep["rel"] < parity.TOL_Y
+    finally:
+        layer.close()
+
+
 def test_mx_activation_codes_bitexact(tiny_mx):
     """The MXFP8 codes of the routed token rows equal the oracle's quantisation of x."""
     lay, mxq, layer = tiny_mx

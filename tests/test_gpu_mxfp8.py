@@ -49,6 +49,29 @@ def test_tiny_mxfp8_layer_parity(tiny_f8, T):
     assert rep["rel"] < parity.TOL_Y
 
 
+def test_tiny_mxfp8_layer_parity_hot_experts(tiny_f8, cuda_device):
+    """Every token sent to experts 0 and 1 (router bias +6): several full 96-token
+    tiles and a partial one for each of them, with E4M3 weights."""
+    lay, q, _ = tiny_f8
+    T = 300
+    bias = torch.zeros(WL.E, dtype=torch.float32, device=cuda_device)
+    bias[:2] = 6.0
+    hot = dict(lay, bias=bias)
+    layer = moe.MoELayer.from_layer(hot, top_k=WL.k, max_tokens=400, mx=q)
+    try:
+        x = lay["x"][:T].contiguous()
+        y, idx, w = layer.forward_with_routing(x)
+        torch.cuda.synchronize()
+        assert layer.status() == moe.MOE_OK
+        cnt = np.bincount(idx.cpu().numpy().ravel(), minlength=WL.E)
+        assert cnt[0] == T and cnt[1] == T
+        rep = parity.compare_layer(dict(hot, x=x), np.arange(T), y.float().cpu().numpy(), idx.cpu().numpy(),
+                                   w.cpu().numpy(), WL.k, WL.route_scale, WL.swiglu_limit, mx_q=q)
+        assert rep["rel"] < parity.TOL_Y
+    finally:
+        layer.close()
+
+
 def test_mxfp8_layer_follows_the_mxfp8_oracle(tiny_f8):
     """The GPU output is closer to the oracle's MXFP8 layer than to its BF16 layer on
     the same draw: the path computes the MXFP8 semantics, not another format's."""
