@@ -19,21 +19,22 @@ pytestmark = pytest.mark.gpu
 WL = synth.WORKLOADS["tiny"]
 
 
-def _mxq(lay):
+def _mxq(lay, fmt):
+    quant = omx.quantize_mxfp8 if fmt == "mxfp8" else omx.quantize_mxfp4_packed
     out = {}
     for n, sname in (("w1", "s1"), ("w3", "s3"), ("w2", "s2")):
-        q, sc = omx.quantize_mxfp4_packed(parity.f64(lay[n]))
+        q, sc = quant(parity.f64(lay[n]))
         out[n], out[sname] = torch.from_numpy(np.ascontiguousarray(q)), torch.from_numpy(np.ascontiguousarray(sc))
     return out
 
 
-@pytest.mark.parametrize("mx", [False, True], ids=["bf16", "mxfp4"])
+@pytest.mark.parametrize("mx", [False, "mxfp4", "mxfp8"], ids=["bf16", "mxfp4", "mxfp8"])
 @pytest.mark.parametrize("split", [16, 11])
 def test_partial_outputs_of_two_windows(cuda_device, mx, split):
     build.build()
     Tmax = 300
     lay = synth.make_layer(WL.with_tokens(Tmax), device="cpu")
-    q = _mxq(lay) if mx else None
+    q = _mxq(lay, mx) if mx else None
     lay = {k: (v.to(cuda_device) if isinstance(v, torch.Tensor) else v) for k, v in lay.items()}
     if q is not None:
         q = {k: v.to(cuda_device) for k, v in q.items()}
