@@ -106,3 +106,32 @@ def test_recorded_traffic_needs_matching_sources(tmp_path, monkeypatch):
     assert bench.recorded_traffic("w", "other") is None
     (csrc / "k.cu").write_text("kernel v2\n")
     assert bench.recorded_traffic("w", "kern") is None
+
+
+def test_peaks_from_the_measured_file_else_the_fallback(tmp_path, monkeypatch):
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.peaks() == (6650.0, 1590.0, 1400.0, "fallback")
+    (tmp_path / "MEASURED_PEAKS.json").write_text(
+        json.dumps({"hbm_gbs": 6472.5, "bf16_tflops": 1612.0, "bf16_tflops_sustained": 1401.0}))
+    assert bench.peaks() == (6472.5, 1612.0, 1401.0, "measured")
+    (tmp_path / "MEASURED_PEAKS.json").write_text(json.dumps({"hbm_gbs": 6500, "bf16_tflops": 1600}))
+    assert bench.peaks() == (6500.0, 1600.0, 1600.0, "measured")   # no sustained figure: the burst one
+
+
+def test_roofline_fractions_use_the_measured_peaks(tmp_path, monkeypatch):
+    """An HBM-bound kernel's frac is its algorithmic bytes per launch over its mean
+    launch time, against the copy figure of MEASURED_PEAKS.json, and against the
+    read-only probe when one was measured; a block-scaled contraction takes twice
+    the measured BF16 rate."""
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    (tmp_path / "MEASURED_PEAKS.json").write_text(json.dumps({"hbm_gbs": 6000.0, "bf16_tflops": 1500.0}))
+    hbm, tc, _, src = bench.peaks()
+    prof = {"gemm_fused": (30.0, 20), "gemm_gateup_mx": (20.0, 10)}     # total ms, launches
+    alg = {"kern": {"gemm_fused": (9.0e9, 1.0e12), "gemm_gateup_mx": (1.0e9, 6.0e12)},
+           "step_bytes": 0.0, "step_flops": 0.0}
+    r = bench.kernel_roofline("gemm_fused", prof, alg, hbm, tc, src, 7200.0, "nowhere")
+    assert r["bound"] == "hbm" and r["peak"] == 6000.0 and r["peak_source"].startswith("measured")
+    assert abs(r["achieved"] - 6000.0) < 1e-6 and abs(r["frac"] - 1.0) < 1e-9      # 9 GB in 1.5 ms
+    assert abs(r["frac_of_read_peak"] - 6000.0 / 7200.0) < 1e-9 and r["traffic"] is None
+    m = bench.kernel_roofline("gemm_gateup_mx", prof, alg, hbm, tc, src, 7200.0, "nowhere")
+    assert m["bound"] == "tensor" and m["peak"] == 3000.0 and abs(m["achieved"] - 3000.0) < 1e-6   # 6 TFLOP in 2 ms
