@@ -132,13 +132,8 @@ def test_top1(cuda_device, mx):
 
 
 def test_widest_hidden(cuda_device):
-    """Outputs compared on 6 tokens per batch (about 100k elements, like the full-size
-    tests' samples). The bound caps the largest error over the compared elements,
-    whose expected size grows with their number: the float64 layer with only h and y
-    rounded to BF16 already reaches 2.3 % of RMS over the 655k elements of 40
-    tokens of this shape."""
     wl = synth.Workload("cfg_h16k", T=0, H=16384, I=128, E=8, k=2, seed=2011)
-    _check(wl, [3, 40, 200], cuda_device, sample=6)
+    _check(wl, [3, 40, 200], cuda_device)
 
 
 def test_widest_expert(cuda_device):
