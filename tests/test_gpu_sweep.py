@@ -1,6 +1,7 @@
-"""A seeded sweep of small layer configurations against the oracle, through the C
-ABI: BF16, MXFP4 and MXFP8 routed experts; 0 to 2 shared experts; top-k 1 to 8;
-hidden 128 to 512 (multiples of 128, some not of 256); expert width 128 or 256;
+"""A seeded sweep of layer configurations against the oracle, through the C ABI:
+BF16, MXFP4 and MXFP8 routed experts; 0 to 2 shared experts; top-k 1 to 16;
+8 to 512 routed experts; hidden 128 to 2048 (multiples of 128, some not of 256);
+expert width 128 to 512;
 uniform and skewed routers (a per-expert bias, so that a few experts take several
 token tiles and many get a handful of rows); and token counts from one to many
 tokens per expert, so that each case runs the routing, permutation, tile-list,
@@ -35,7 +36,26 @@ def _cases(n=24, seed=20241203):
     return out
 
 
-CASES = _cases()
+def _large_cases(n=12, seed=20241204):
+    """Larger layers: many experts, wider k and widths, up to 1200 tokens (several
+    permutation chunks, both many-token tile widths, the thin-tile split)."""
+    rng = np.random.default_rng(seed)
+    out = []
+    for i in range(n):
+        fmt = str(rng.choice(["bf16", "mxfp4", "mxfp8"]))
+        # block-scaled layers kept smaller: the oracle's codec quantises them on the host
+        E = int(rng.choice([128, 256, 384, 512] if fmt == "bf16" else [128, 256]))
+        k = int(rng.choice([4, 6, 8, 12, 16]))
+        H = int(rng.choice([512, 768, 1024, 2048] if fmt == "bf16" else [512, 768, 1024]))
+        I = int(rng.choice([256, 512] if fmt == "bf16" else [256]))
+        S = int(rng.integers(0, 3))
+        skew = bool(rng.integers(0, 2))
+        Ts = sorted({int(rng.integers(1, 33)), int(rng.integers(200, 601)), int(rng.integers(601, 1201))})
+        out.append((f"L{i}-{fmt}-E{E}k{k}H{H}I{I}S{S}{'-skew' if skew else ''}", E, k, H, I, S, fmt, skew, Ts))
+    return out
+
+
+CASES = _cases() + _large_cases()
 
 
 def _quantised(lay, fmt):
@@ -50,7 +70,9 @@ def _quantised(lay, fmt):
 @pytest.mark.parametrize("name,E,k,H,I,S,fmt,skew,Ts", CASES, ids=[c[0] for c in CASES])
 def test_sweep_case(cuda_device, name, E, k, H, I, S, fmt, skew, Ts):
     build.build()
-    wl = synth.Workload(name, T=0, H=H, I=I, E=E, k=k, n_shared=S, seed=3000 + int(name.split("-")[0][1:]))
+    tag = name.split("-")[0]
+    wl = synth.Workload(name, T=0, H=H, I=I, E=E, k=k, n_shared=S,
+                        seed=(3000 if tag[0] == "c" else 3100) + int(tag[1:]))
     Tmax = max(Ts)
     lay = synth.make_layer(wl.with_tokens(Tmax), device="cpu")
     if skew:
